@@ -1,0 +1,55 @@
+"""Planted-mistake check of the oracle pins (CPU only).
+
+Each entry plants one plausible slip in a private copy of the oracle module and
+asserts that at least one pin in ``test_oracle_pins`` fails on it.
+"""
+
+import importlib.util
+import inspect
+import os
+import types
+
+import pytest
+
+import tests.test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(__file__)), "oracle", "mla_oracle.py")
+
+MUTATIONS = {
+    "rope_rotation_sign": ("x1 * c - x2 * s, x2 * c + x1 * s", "x1 * c + x2 * s, x2 * c - x1 * s"),
+    "rope_interleaved_pairs": ("x1, x2 = x[..., :h], x[..., h:]\n    return np.concat",
+                               "x1, x2 = x[..., 0::2], x[..., 1::2]\n    return np.concat"),
+    "rope_frequency_exponent": ("return base ** (-(2.0 * m) / d_r)", "return base ** (-(1.0 * m) / d_r)"),
+    "scale_without_rope_dims": ("1.0 / math.sqrt(d_h + d_r)", "1.0 / math.sqrt(d_h)"),
+    "shared_key_dropped": ("k = np.concatenate([k_c, k_r_rot], axis=1)",
+                           "k = np.concatenate([k_c, 0 * k_r_rot], axis=1)"),
+    "mask_off_by_one": ("visible = j_idx <= (T_k - T_q + t_idx)", "visible = j_idx < (T_k - T_q + t_idx)"),
+    "value_uses_key_weight": ("v_c = c_kv @ wv.T", "v_c = c_kv @ wk.T"),
+    "query_position_shift": ("qpos = np.arange(L - T_q, L)", "qpos = np.arange(L - T_q, L) - 1"),
+    "merge_weights_linear": ("w = np.exp(lse_parts - m)", "w = (lse_parts - m + 1)"),
+    "absorb_transposed": ("out[:, i, :] = q_c[:, i, :] @ w_uk[i]",
+                          "out[:, i, :] = (q_c[:, i, :] @ w_uk[i])[:, ::-1]"),
+}
+
+
+def _mutated_module(old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, old
+    mod = types.ModuleType("mla_oracle_mutant")
+    exec(compile(src.replace(old, new), "mla_oracle_mutant", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, monkeypatch):
+    mod = _mutated_module(*MUTATIONS[name])
+    monkeypatch.setattr(pins, "O", mod)
+    failures = 0
+    for fname, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not fname.startswith("test_"):
+            continue
+        try:
+            fn()
+        except Exception:
+            failures += 1
+    assert failures >= 1, f"no pin caught mutation {name}"
