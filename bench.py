@@ -1,0 +1,369 @@
+#!/usr/bin/env python3
+"""Benchmark of one MLA decode step (absorb_q -> rope_append -> decode -> up_v)
+on the DeepSeek-V2 decode workload, printed as one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload v2_decode|varlen|long|multi_token|tiny]
+
+N > 1 runs under torch.distributed.run, one process per GPU.  Sequences are
+independent, so every rank runs its own full copy of the workload (weak scaling)
+with no data-path collective; the process group is only used for the barrier
+around the timed region and the max-over-ranks of the device time.
+
+--impl reference times the fp64 CPU oracle on rank 0 on a bounded sample of the
+same workload (a few heads of one sequence per step).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode tokens/s + achieved HBM TB/s & TFLOP/s vs roofline (1×B200)"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="v2_decode")
+    ap.add_argument("--kernel-impl", type=int, default=0, help="mla_config_t.impl (0 auto)")
+    ap.add_argument("--max-splits", type=int, default=0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML polling thread)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [k for k, v in self.REASONS.items() if self.reasons & v and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# the oracle arm
+# ---------------------------------------------------------------------------
+
+def oracle_sample_rate(spec, steps, warmup, heads_per_step=8, budget_s=None):
+    """Time the fp64 oracle on `heads_per_step` heads of one sequence per step.
+
+    Returns (tokens/s, seconds, description).  A token's output needs all n_h
+    heads, so a step credits heads_per_step / n_h of each of its T_q tokens."""
+    from oracle.evaluate import reference
+    b = 0
+    heads_all = list(range(spec.n_h))
+    done_heads, t_total, k = 0, 0.0, 0
+    for i in range(warmup + steps):
+        hs = [heads_all[(i * heads_per_step + j) % spec.n_h] for j in range(heads_per_step)]
+        t0 = time.perf_counter()
+        reference(spec, b, heads=hs)
+        dt = time.perf_counter() - t0
+        if i >= warmup:
+            t_total += dt
+            done_heads += len(hs)
+            k += 1
+            if budget_s is not None and t_total > budget_s:
+                break
+    tokens = done_heads / spec.n_h * spec.T_q
+    desc = (f"{k} steps x {heads_per_step} of {spec.n_h} heads of sequence {b} "
+            f"(context {int(spec.seq_lens[b])}, T_q={spec.T_q}), explicit K/V reconstruction in fp64")
+    return tokens / t_total, t_total, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from mla_latent_kv_38_b200.workloads import config_specs
+    spec = config_specs()[args.workload]
+    rate, secs, desc = oracle_sample_rate(spec, args.steps, args.warmup)
+    line = {
+        "metric": METRIC, "impl": "reference", "value": rate, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name},
+        "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def decode_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mla_latent_kv_38_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.startswith(("decode", "sm100")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload, kernel_hash):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current decode kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    for line in open(p):
+        parts = line.split("#")[0].split()
+        if len(parts) == 3 and parts[0] == workload and parts[1] == kernel_hash:
+            return int(parts[2])
+    return None
+
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+    from mla_latent_kv_38_b200 import binding as M
+    from mla_latent_kv_38_b200.runner import DeviceCase
+    from mla_latent_kv_38_b200.workloads import config_specs
+
+    spec = config_specs()[args.workload]
+    dc = DeviceCase(spec, impl=args.kernel_impl, max_splits=args.max_splits, device=f"cuda:{local}")
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    launches_decode = M.mla_decode_launches(dc.cfg, spec.B, spec.T_q, args.max_splits)
+    launches_per_step = 3 + launches_decode       # absorb_q, rope_append, up_v + decode
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    def max_over_ranks(x):
+        if pg is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up
+    for _ in range(max(args.warmup, 3)):
+        dc.reset_step_inputs()
+        dc.step()
+    torch.cuda.synchronize(dev)
+    st = dc.decode_status() | dc.append_status()
+    if st:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with sampler:
+        for k in range(K):
+            flush.zero_()                         # L2 flush outside the timed events
+            dc.q_r.copy_(dc.q_r_pre)
+            s = dc.spec
+            ev[k][0].record(stream)
+            M.mla_absorb_q(dc.cfg, dc.q_c, dc.w_uk, dc.q_abs, s.n_tok)
+            M.mla_rope_append(dc.cfg, dc.q_r, dc.k_r_new, dc.c_kv_new, dc.positions, dc.rope_table,
+                              dc.max_pos, dc.block_table, s.max_blocks, dc.pool, s.num_blocks, s.B,
+                              s.T_q, dc.status)
+            ev[k][1].record(stream)
+            dc.decode_only()
+            ev[k][2].record(stream)
+            M.mla_up_v(dc.cfg, dc.latent, dc.w_uv, dc.out, s.n_tok)
+            ev[k][3].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    step_ms = sum(e[0].elapsed_time(e[3]) for e in ev)
+    decode_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    step_ms = max_over_ranks(step_ms)
+    tokens_per_step = spec.n_tok
+    value = world * tokens_per_step * K / (step_ms / 1e3)
+
+    # end to end through the public API with host buffers
+    h_in = [torch.from_numpy(a.view(np.int16)).pin_memory() for a in
+            (dc.h_q_c, dc.h_q_r, dc.h_k_r_new, dc.h_c_kv_new)]
+    h_pos = torch.from_numpy(dc.h_positions).pin_memory()
+    d_in = [dc.q_c, dc.q_r, dc.k_r_new, dc.c_kv_new]
+    h_out = torch.empty(dc.out.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h_in) + h_pos.numel() * 4
+    d2h = h_out.numel() * 2
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    for k in range(K):
+        flush.zero_()
+        e0.record(stream)
+        for h, d in zip(h_in, d_in):
+            d.view(torch.int16).copy_(h, non_blocking=True)
+        dc.positions.copy_(h_pos, non_blocking=True)
+        dc.step()
+        h_out.copy_(dc.out, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e2e_ms)
+    e2e_value = world * tokens_per_step * K / (e2e_ms / 1e3)
+
+    peaks, peak_src = load_peaks()
+    bytes_alg = spec.algorithmic_bytes()
+    flops_alg = spec.algorithmic_flops()
+    dec_s = decode_ms / 1e3
+    hbm_gbs = bytes_alg / dec_s / 1e9
+    tflops = flops_alg / dec_s / 1e12
+    t_hbm = bytes_alg / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops_alg / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": hbm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": hbm_gbs / peaks["hbm_gbs"]}
+    else:
+        roof = {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"]}
+    khash = decode_source_hash()
+    roof["traffic"] = profiled_traffic(args.workload, khash)
+    roof["peak_source"] = f"MEASURED_PEAKS.json ({peak_src})"
+    roof["kernel"] = "mla_decode (decode + split merge)"
+    roof["roofline_time_us"] = 1e6 * max(t_hbm, t_tc)
+    roof["decode_us"] = decode_ms * 1e3
+
+    if rank != 0:
+        if pg is not None:
+            pg.destroy_process_group()
+        return 0
+
+    cpu = None
+    if world == 1:
+        rate, secs, desc = oracle_sample_rate(spec, steps=4, warmup=1, budget_s=20.0)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": step_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": spec.name, "B": spec.B, "T_q": spec.T_q, "n_h": spec.n_h,
+                   "d_c": spec.d_c, "d_r": spec.d_r, "block_size": spec.block_size,
+                   "context": [int(spec.seq_lens.min()), int(spec.seq_lens.max())],
+                   "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "decode_hbm_tbs": hbm_gbs / 1e3, "decode_tflops": tflops,
+        "decode_tflops_frac_sustained": tflops / peaks.get("bf16_tflops_sustained", 1e9),
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * K,
+        "clocks": sampler.summary(),
+        "decode_kernel_hash": khash,
+    }
+    print(json.dumps(line))
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,187 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) MLA latent-KV decode library.
+ *
+ * One decode step of Multi-head Latent Attention over a paged latent cache:
+ *
+ *   mla_absorb_q     q_abs = W^UK^T q^C, per head
+ *   mla_rope_append  RoPE on q^R and k^R, then c^KV || k^R appended to the cache
+ *   mla_decode       causal softmax of the absorbed scores over the cached rows,
+ *                    weighted sum of the latent rows (split-KV + LSE merge)
+ *   mla_up_v         o = W^UV latent, per head
+ *
+ * Sources (page title, section / equation):
+ *   [notes]  "MLA(Multi-head Latent Attention): DeepSeek-V2 논문정리":
+ *            eq. (9)-(11); "Key에 대한 수식 전개"; "Value에 대한 수식 전개";
+ *            "Decoupled Rotary Position Embedding"; "MLA 코드 구현".
+ *   [ru]     "Техотчёт DeepSeek-V2 (2024): MLA и экономика инференса":
+ *            "Идея 1", "Идея 2: отделённый RoPE", "Сколько получилось".
+ *   [v3]     DeepSeek-V3 report notes, "Multi-Head Attention 및 Output 계산
+ *            (식 10, 11)", eq. (10).
+ *   [review] "DeepSeek-V2 review", 2.1 (absorption, T = max(B/BW, F/P)),
+ *            2.3 (Decoupled RoPE).
+ *
+ * Conventions for every call
+ *   - Element type mla_bf16 is the raw 16-bit pattern of a bfloat16.
+ *   - All tensor pointers are DEVICE pointers unless a parameter says "host".
+ *     The caller allocates and owns every buffer; the library never allocates
+ *     device memory.  mla_decode takes a caller-provided workspace whose size
+ *     mla_decode_workspace_bytes() returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous on that stream.
+ *   - Return value: MLA_OK (0) or a negative MLA_ERR_* code.  Every argument
+ *     check that needs no device data happens on the host before any launch;
+ *     a rejected call launches nothing and writes nothing.
+ *   - Checks that need device data (positions, block indices, sequence
+ *     lengths) run in the kernels: an offending row is skipped (never read or
+ *     written out of bounds) and a bit is OR-ed into a device status word
+ *     (MLA_STATUS_* bits).  Read it with mla_read_status().
+ *   - Layouts are row-major and densely packed in the order written.
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t mla_bf16;
+
+/* Head shapes of one attention layer.  DeepSeek-V2: n_h = 128, d_c = 512,
+ * d_h = 128, d_r = 64 ([ru] "Сколько получилось"; [v3]).  block_size is the
+ * number of cache rows per page (64).  scale <= 0 selects 1/sqrt(d_h + d_r)
+ * ([v3] eq. (10); [ru] "Идея 2").  impl selects among this library's own
+ * decode kernels; all of them compute the same function. */
+typedef struct {
+    int n_h;
+    int d_c;
+    int d_h;
+    int d_r;
+    int block_size;
+    float scale;
+    int impl; /* mla_decode kernel: 0 = best for the shape, 1 = portable
+                 SIMT kernel (any supported shape), 2 = tcgen05 kernel
+                 (d_c = 512, d_r = 64, n_h a multiple of 64 only) */
+} mla_config_t;
+
+enum {
+    MLA_OK = 0,
+    MLA_ERR_NULL = -1,        /* a required pointer is NULL                   */
+    MLA_ERR_CONFIG = -2,      /* unsupported head shape / block size          */
+    MLA_ERR_SIZE = -3,        /* a count is out of range (n_tok, B, T_q ...)  */
+    MLA_ERR_WORKSPACE = -4,   /* workspace too small or misaligned            */
+    MLA_ERR_LAUNCH = -5,      /* a CUDA launch or runtime call failed         */
+    MLA_ERR_UNSUPPORTED = -6, /* device is not sm_100 or feature unavailable  */
+    MLA_ERR_ALIGN = -7        /* a pointer breaks the 16-byte alignment rule  */
+};
+
+/* Device status word bits (see mla_read_status). */
+enum {
+    MLA_STATUS_BAD_POSITION = 1,  /* position < 0 or beyond the RoPE table    */
+    MLA_STATUS_BAD_BLOCK = 2,     /* block-table entry outside [0, num_blocks) */
+    MLA_STATUS_BAD_SEQ_LEN = 4,   /* seq_len < T_q or beyond the block table  */
+    MLA_STATUS_TIMEOUT = 8        /* a bounded device wait ran out            */
+};
+
+/* Constraints shared by every call: d_c, d_r and d_h multiples of 8,
+ * 8 <= d_c <= 512, 8 <= d_r <= 64, 8 <= d_h <= 256, block_size = 64,
+ * 1 <= n_h <= 1024.  Every tensor pointer 16-byte aligned. */
+
+/* Human-readable name of a return code. */
+const char* mla_status_str(int code);
+
+/* Compute capability check: returns MLA_OK when the current device is sm_100. */
+int mla_check_device(void);
+
+/* RoPE table on the HOST: host_table[p * d_r + m] = cos(p * f_m) and
+ * host_table[p * d_r + d_r/2 + m] = sin(p * f_m) for p < max_pos and
+ * f_m = base^(-2m/d_r), m < d_r/2, evaluated in double and rounded to float
+ * ([notes] "MLA 코드 구현", build_rope_cache).  The caller copies it to the
+ * device and passes it to mla_rope_append.  host_table holds max_pos * d_r
+ * floats. */
+int mla_rope_table(int d_r, double base, int max_pos, float* host_table);
+
+/* q_abs[n, i, :] = W^UK_i^T q_c[n, i, :]  ([notes] "Key에 대한 수식 전개";
+ * [ru] "Идея 1").
+ *   q_c   (n_tok, n_h, d_h)  bf16
+ *   w_uk  (n_h, d_h, d_c)    bf16; W^UK_i = w_uk[i] maps a latent to head i's key
+ *   q_abs (n_tok, n_h, d_c)  bf16 out (float accumulation, RNE rounding)
+ * n_tok = B * T_q, token n = b * T_q + t.  1 <= n_tok <= 65536. */
+int mla_absorb_q(const mla_config_t* cfg, const mla_bf16* q_c, const mla_bf16* w_uk,
+                 mla_bf16* q_abs, int n_tok, void* stream);
+
+/* Decoupled RoPE and paged append ([review] 2.3; [ru] "Идея 2"; [notes]
+ * "Decoupled Rotary Position Embedding", "MLA 코드 구현" forward).
+ * For token n = b * T_q + t with p = positions[n]:
+ *   q_r[n, i, :] <- RoPE(q_r[n, i, :], p) for every head i (skipped if q_r NULL)
+ *   pool[blk][p % block_size][0 : d_c]        <- c_kv[n, :]           (bit copy)
+ *   pool[blk][p % block_size][d_c : d_c+d_r]  <- RoPE(k_r[n, :], p)
+ * with blk = block_table[b * max_blocks_per_seq + p / block_size].
+ * RoPE pairs element m with m + d_r/2 (half split) and uses float32 products
+ * and sums without fused multiply-add on the float32 table, then rounds to
+ * bf16 (round to nearest even).
+ *   q_r        (n_tok, n_h, d_r) bf16, in place, may be NULL
+ *   k_r        (n_tok, d_r) bf16;  c_kv (n_tok, d_c) bf16
+ *   positions  (n_tok) int32
+ *   rope_table (max_pos, d_r) float32 from mla_rope_table
+ *   block_table (B, max_blocks_per_seq) int32
+ *   pool       (num_blocks, block_size, d_c + d_r) bf16
+ *   dev_status one int32 on the device (may be NULL): MLA_STATUS_* bits are
+ *              OR-ed in for rows whose position or block index is invalid;
+ *              those rows are not written. */
+int mla_rope_append(const mla_config_t* cfg, mla_bf16* q_r, const mla_bf16* k_r,
+                    const mla_bf16* c_kv, const int32_t* positions,
+                    const float* rope_table, int max_pos,
+                    const int32_t* block_table, int max_blocks_per_seq,
+                    mla_bf16* pool, int num_blocks, int B, int T_q,
+                    int32_t* dev_status, void* stream);
+
+/* Bytes of workspace mla_decode needs for these sizes (256-byte aligned
+ * pointer required).  max_splits as for mla_decode. */
+size_t mla_decode_workspace_bytes(const mla_config_t* cfg, int B, int T_q, int max_splits);
+
+/* Absorbed MLA decode over the paged cache ([v3] eq. (10) with [notes]
+ * "Key에 대한 수식 전개" and "Value에 대한 수식 전개"):
+ *   s[b,t,i,j] = scale * (q_abs[b,t,i,:] . pool_row(b,j)[0:d_c]
+ *                         + q_r[b,t,i,:] . pool_row(b,j)[d_c:d_c+d_r])
+ * for keys j <= seq_lens[b] - T_q + t (generalised causal mask, [notes]
+ * "MLA 코드 구현" forward), softmax over j, and
+ *   out_latent[b,t,i,:] = sum_j p[b,t,i,j] pool_row(b,j)[0:d_c]     (bf16)
+ *   out_lse[b,t,i]      = log sum_j exp(s[b,t,i,j])                  (float32)
+ *   q_abs (B*T_q, n_h, d_c) bf16;  q_r (B*T_q, n_h, d_r) bf16 (already RoPE'd)
+ *   pool, block_table as for mla_rope_append; seq_lens (B) int32, the cache
+ *   length AFTER the step's append, 1 <= T_q <= seq_lens[b].
+ *   max_splits: upper bound on key-range splits per query row (0 = choose).
+ * The key ranges are split across thread blocks; fp32 partial results in the
+ * workspace are merged by a log-sum-exp reduction kernel.  The workspace
+ * starts with the device status word (mla_read_status).  T_q <= 16. */
+int mla_decode(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q_r,
+               const mla_bf16* pool, int num_blocks, const int32_t* block_table,
+               int max_blocks_per_seq, const int32_t* seq_lens, int B, int T_q,
+               int max_splits, void* workspace, size_t ws_bytes,
+               mla_bf16* out_latent, float* out_lse, void* stream);
+
+/* Number of kernel launches one mla_decode call with these arguments makes
+ * (decode, optional scheduling and merge kernels); negative on bad arguments. */
+int mla_decode_launches(const mla_config_t* cfg, int B, int T_q, int max_splits);
+
+/* o[n, i, :] = W^UV_i latent[n, i, :]  ([notes] "Value에 대한 수식 전개").
+ *   latent (n_tok, n_h, d_c) bf16;  w_uv (n_h, d_h, d_c) bf16
+ *   out    (n_tok, n_h, d_h) bf16 (float accumulation, RNE rounding) */
+int mla_up_v(const mla_config_t* cfg, const mla_bf16* latent, const mla_bf16* w_uv,
+             mla_bf16* out, int n_tok, void* stream);
+
+/* Zero a device status word (async on stream). */
+int mla_clear_status(int32_t* dev_status, void* stream);
+
+/* Copy a device status word to *host_status; synchronises `stream`.  For
+ * mla_decode the word is the first int32 of the workspace. */
+int mla_read_status(const int32_t* dev_status, int32_t* host_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H */

@@ -1,0 +1,79 @@
+// Shared device helpers of the MLA decode library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mla.h"
+
+namespace mla {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ float bf2f(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// float -> bf16 bits, round to nearest even (hardware conversion)
+__device__ __forceinline__ uint16_t f2bf(float f) {
+    __nv_bfloat16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&h);
+}
+
+// two floats -> packed bf16x2 (lo in the low half)
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    return static_cast<uint32_t>(f2bf(lo)) | (static_cast<uint32_t>(f2bf(hi)) << 16);
+}
+
+__device__ __forceinline__ void unpack8(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// 2^x on the special-function unit (PTX ex2.approx; 2^-inf = +0)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ void raise_status(int32_t* st, int bits) {
+    if (st != nullptr) atomicOr(st, bits);
+}
+
+// Parameters of one decode launch (shared by the SIMT and tcgen05 kernels).
+struct DecodeParams {
+    const uint16_t* q_abs;      // (n_tok, n_h, d_c)
+    const uint16_t* q_r;        // (n_tok, n_h, d_r)
+    const uint16_t* pool;       // (num_blocks, block_size, d_c + d_r)
+    const int32_t* block_table; // (B, max_blocks)
+    const int32_t* seq_lens;    // (B)
+    uint16_t* out_latent;       // (n_tok, n_h, d_c)
+    float* out_lse;             // (n_tok, n_h)
+    float* part_o;              // (splits, n_tok, n_h, d_c) fp32
+    float* part_lse;            // (splits, n_tok, n_h)
+    int32_t* status;
+    int n_h, d_c, d_r, block_size;
+    int num_blocks, max_blocks, B, T_q, n_tok, splits;
+    float scale_log2;           // scale * log2(e)
+};
+
+}  // namespace mla

@@ -1,0 +1,224 @@
+// Portable absorbed-MLA decode (CUDA cores, float32), any supported head shape,
+// plus the split-KV log-sum-exp merge used by every decode kernel.
+//
+// Scores follow DeepSeek-V3 report notes eq. (10) with the absorbed query of
+// "MLA(Multi-head Latent Attention): DeepSeek-V2 논문정리", "Key에 대한 수식
+// 전개": s_j = scale * (q_abs . c_j + q^R . k^R_j); the output is the
+// probability-weighted latent sum of "Value에 대한 수식 전개" (W^UV is applied
+// afterwards by mla_up_v).  The causal limit of query t is
+// seq_len - T_q + t ("MLA 코드 구현", generalised causal mask).
+//
+// Layout of the work: grid (split, token, head group of 8).  Each warp owns one
+// head; the 8 warps share each 32-row key tile staged in shared memory with
+// 16-byte loads.  Online softmax in the exp2 domain.
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mla {
+
+constexpr int kSimtHeads = 8;
+constexpr int kSimtKeys = 32;
+
+__global__ void __launch_bounds__(256)
+decode_simt_kernel(DecodeParams P) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int D = P.d_c + P.d_r;
+    const int row_vec = D / 8 + 1;                       // padded row, in uint4
+    uint4* Ks = reinterpret_cast<uint4*>(smem_raw);      // [32][row_vec]
+    float* Qs = reinterpret_cast<float*>(Ks + kSimtKeys * row_vec);  // [8][D]
+
+    const int split = blockIdx.x, n = blockIdx.y, hg = blockIdx.z;
+    const int b = n / P.T_q, t = n - b * P.T_q;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int head = hg * kSimtHeads + warp;
+    const bool head_ok = head < P.n_h;
+
+    int L = P.seq_lens[b];
+    const bool len_ok = L >= P.T_q && L <= P.max_blocks * P.block_size;
+    if (!len_ok && threadIdx.x == 0 && split == 0 && hg == 0 && t == 0)
+        raise_status(P.status, MLA_STATUS_BAD_SEQ_LEN);
+    const int kv_len = len_ok ? L - P.T_q + t + 1 : 0;
+    const int ntiles = (kv_len + kSimtKeys - 1) / kSimtKeys;
+    const int per = (ntiles + P.splits - 1) / P.splits;
+    const int tile0 = split * per;
+    const int tile1 = min(ntiles, tile0 + per);
+
+    // stage the query rows, pre-multiplied by scale*log2(e)
+    for (int e = threadIdx.x; e < kSimtHeads * D; e += blockDim.x) {
+        const int w = e / D, c = e - w * D;
+        const int hh = hg * kSimtHeads + w;
+        float v = 0.f;
+        if (hh < P.n_h) {
+            v = c < P.d_c ? bf2f(P.q_abs[(static_cast<size_t>(n) * P.n_h + hh) * P.d_c + c])
+                          : bf2f(P.q_r[(static_cast<size_t>(n) * P.n_h + hh) * P.d_r + (c - P.d_c)]);
+        }
+        Qs[e] = v * P.scale_log2;
+    }
+
+    const int nchunk = P.d_c >> 3;                      // 8-column latent chunks
+    float o[2][8];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) o[u][k] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    const float* q = Qs + warp * D;
+
+    for (int tile = tile0; tile < tile1; ++tile) {
+        __syncthreads();
+        // cooperative load of 32 cache rows through the block table
+        for (int e = threadIdx.x; e < kSimtKeys * (D / 8); e += blockDim.x) {
+            const int j = e / (D / 8), v = e - j * (D / 8);
+            const int key = tile * kSimtKeys + j;
+            uint4 val = make_uint4(0, 0, 0, 0);
+            if (key < kv_len) {
+                const int blk = P.block_table[static_cast<size_t>(b) * P.max_blocks + key / P.block_size];
+                if (blk >= 0 && blk < P.num_blocks) {
+                    const uint4* src = reinterpret_cast<const uint4*>(
+                        P.pool + (static_cast<size_t>(blk) * P.block_size + key % P.block_size) * D);
+                    val = src[v];
+                } else if (v == 0) {
+                    raise_status(P.status, MLA_STATUS_BAD_BLOCK);
+                }
+            }
+            Ks[j * row_vec + v] = val;
+        }
+        __syncthreads();
+        if (!head_ok) continue;
+
+        // scores: lane j scores key j
+        const int key = tile * kSimtKeys + lane;
+        float s = 0.f;
+        const uint4* krow = Ks + lane * row_vec;
+        for (int v = 0; v < D / 8; ++v) {
+            float kf[8];
+            unpack8(krow[v], kf);
+            const float4 qa = *reinterpret_cast<const float4*>(q + 8 * v);
+            const float4 qb = *reinterpret_cast<const float4*>(q + 8 * v + 4);
+            s = fmaf(qa.x, kf[0], s); s = fmaf(qa.y, kf[1], s);
+            s = fmaf(qa.z, kf[2], s); s = fmaf(qa.w, kf[3], s);
+            s = fmaf(qb.x, kf[4], s); s = fmaf(qb.y, kf[5], s);
+            s = fmaf(qb.z, kf[6], s); s = fmaf(qb.w, kf[7], s);
+        }
+        if (key >= kv_len) s = -INFINITY;
+        const float m_new = fmaxf(m_run, warp_max(s));
+        const float alpha = ex2(m_run - m_new);
+        const float p = ex2(s - m_new);
+        l_run = l_run * alpha + warp_sum(p);
+        m_run = m_new;
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) o[u][k] *= alpha;
+        for (int j = 0; j < kSimtKeys; ++j) {
+            const float pj = __shfl_sync(0xffffffffu, p, j);
+            if (pj == 0.f) continue;   // warp-uniform
+            const uint4* vrow = Ks + j * row_vec;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int ch = lane + 32 * u;
+                if (ch < nchunk) {
+                    float vf[8];
+                    unpack8(vrow[ch], vf);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) o[u][k] = fmaf(pj, vf[k], o[u][k]);
+                }
+            }
+        }
+    }
+
+    if (!head_ok) return;
+    const size_t row = static_cast<size_t>(n) * P.n_h + head;
+    const bool empty = l_run == 0.f;
+    const float inv_l = empty ? 0.f : 1.f / l_run;
+    const float lse = empty ? -INFINITY : (m_run + __log2f(l_run)) * kLn2;
+    if (P.splits == 1) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int ch = lane + 32 * u;
+            if (ch < nchunk) {
+                uint4 w;
+                w.x = pack_bf16x2(o[u][0] * inv_l, o[u][1] * inv_l);
+                w.y = pack_bf16x2(o[u][2] * inv_l, o[u][3] * inv_l);
+                w.z = pack_bf16x2(o[u][4] * inv_l, o[u][5] * inv_l);
+                w.w = pack_bf16x2(o[u][6] * inv_l, o[u][7] * inv_l);
+                reinterpret_cast<uint4*>(P.out_latent + row * P.d_c)[ch] = w;
+            }
+        }
+        if (lane == 0) P.out_lse[row] = lse;
+    } else {
+        float* po = P.part_o + (static_cast<size_t>(split) * P.n_tok * P.n_h + row) * P.d_c;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int ch = lane + 32 * u;
+            if (ch < nchunk) {
+                float4* d = reinterpret_cast<float4*>(po + 8 * ch);
+                d[0] = make_float4(o[u][0] * inv_l, o[u][1] * inv_l, o[u][2] * inv_l, o[u][3] * inv_l);
+                d[1] = make_float4(o[u][4] * inv_l, o[u][5] * inv_l, o[u][6] * inv_l, o[u][7] * inv_l);
+            }
+        }
+        if (lane == 0) P.part_lse[static_cast<size_t>(split) * P.n_tok * P.n_h + row] = lse;
+    }
+}
+
+// Split-KV merge: o = sum_s w_s o_s / sum_s w_s, lse = max + log sum_s w_s with
+// w_s = exp(lse_s - max).  One block per (token, head).
+__global__ void __launch_bounds__(128)
+merge_splits_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                    uint16_t* __restrict__ out_latent, float* __restrict__ out_lse,
+                    int rows, int d_c, int splits) {
+    const int row = blockIdx.x;
+    float m = -INFINITY;
+    for (int s = 0; s < splits; ++s) m = fmaxf(m, part_lse[static_cast<size_t>(s) * rows + row]);
+    float z = 0.f;
+    for (int s = 0; s < splits; ++s) {
+        const float ls = part_lse[static_cast<size_t>(s) * rows + row];
+        z += (ls == -INFINITY) ? 0.f : ex2((ls - m) * kLog2e);
+    }
+    const float inv_z = z > 0.f ? 1.f / z : 0.f;
+    for (int c = threadIdx.x * 4; c < d_c; c += blockDim.x * 4) {
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        for (int s = 0; s < splits; ++s) {
+            const float ls = part_lse[static_cast<size_t>(s) * rows + row];
+            if (ls == -INFINITY) continue;
+            const float w = ex2((ls - m) * kLog2e) * inv_z;
+            const float4 v = *reinterpret_cast<const float4*>(
+                part_o + (static_cast<size_t>(s) * rows + row) * d_c + c);
+            a0 = fmaf(w, v.x, a0); a1 = fmaf(w, v.y, a1);
+            a2 = fmaf(w, v.z, a2); a3 = fmaf(w, v.w, a3);
+        }
+        uint2 pk;
+        pk.x = pack_bf16x2(a0, a1);
+        pk.y = pack_bf16x2(a2, a3);
+        *reinterpret_cast<uint2*>(out_latent + static_cast<size_t>(row) * d_c + c) = pk;
+    }
+    if (threadIdx.x == 0) out_lse[row] = z > 0.f ? m + logf(z) : -INFINITY;
+}
+
+size_t simt_smem_bytes(int d_c, int d_r) {
+    const int D = d_c + d_r;
+    return static_cast<size_t>(kSimtKeys) * (D / 8 + 1) * 16 + static_cast<size_t>(kSimtHeads) * D * 4;
+}
+
+cudaError_t launch_decode_simt(const DecodeParams& P, cudaStream_t stream) {
+    const size_t smem = simt_smem_bytes(P.d_c, P.d_r);
+    cudaError_t e = cudaFuncSetAttribute(decode_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    dim3 grid(P.splits, P.n_tok, (P.n_h + kSimtHeads - 1) / kSimtHeads);
+    decode_simt_kernel<<<grid, 256, smem, stream>>>(P);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || P.splits == 1) return e;
+    return launch_merge(P.part_o, P.part_lse, P.out_latent, P.out_lse, P.n_tok * P.n_h, P.d_c,
+                        P.splits, stream);
+}
+
+cudaError_t launch_merge(const float* part_o, const float* part_lse, uint16_t* out_latent,
+                         float* out_lse, int rows, int d_c, int splits, cudaStream_t stream) {
+    merge_splits_kernel<<<rows, 128, 0, stream>>>(part_o, part_lse, out_latent, out_lse, rows, d_c,
+                                                  splits);
+    return cudaGetLastError();
+}
+
+}  // namespace mla

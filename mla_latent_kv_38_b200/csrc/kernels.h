@@ -1,0 +1,28 @@
+// Internal launchers (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mla {
+
+struct DecodeParams;
+
+cudaError_t launch_rope_append(uint16_t* q_r, const uint16_t* k_r, const uint16_t* c_kv,
+                               const int32_t* positions, const float* table, int max_pos,
+                               const int32_t* block_table, int max_blocks, uint16_t* pool,
+                               int num_blocks, int n_tok, int T_q, int n_h, int d_c, int d_r,
+                               int block_size, int32_t* status, cudaStream_t stream);
+
+size_t simt_smem_bytes(int d_c, int d_r);
+cudaError_t launch_decode_simt(const DecodeParams& P, cudaStream_t stream);
+cudaError_t launch_merge(const float* part_o, const float* part_lse, uint16_t* out_latent,
+                         float* out_lse, int rows, int d_c, int splits, cudaStream_t stream);
+
+cudaError_t launch_absorb_q_simt(const uint16_t* q_c, const uint16_t* w_uk, uint16_t* q_abs,
+                                 int n_tok, int n_h, int d_h, int d_c, cudaStream_t stream);
+cudaError_t launch_up_v_simt(const uint16_t* latent, const uint16_t* w_uv, uint16_t* out,
+                             int n_tok, int n_h, int d_h, int d_c, cudaStream_t stream);
+
+}  // namespace mla

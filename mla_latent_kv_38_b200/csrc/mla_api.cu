@@ -1,0 +1,232 @@
+// Host side of the C ABI declared in include/mla.h: argument checks, workspace
+// layout, kernel selection and launches.  No device memory is allocated here.
+
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100_decode.h"
+
+namespace {
+
+using mla::DecodeParams;
+
+constexpr int kMaxSplits = 256;
+constexpr int kB200Sms = 148;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int check_config(const mla_config_t* c) {
+    if (c == nullptr) return MLA_ERR_NULL;
+    if (c->n_h < 1 || c->n_h > 1024) return MLA_ERR_CONFIG;
+    if (c->d_c < 8 || c->d_c > 512 || c->d_c % 8) return MLA_ERR_CONFIG;
+    if (c->d_r < 8 || c->d_r > 64 || c->d_r % 8) return MLA_ERR_CONFIG;
+    if (c->d_h < 8 || c->d_h > 256 || c->d_h % 8) return MLA_ERR_CONFIG;
+    if (c->block_size != 64) return MLA_ERR_CONFIG;
+    if (c->impl < 0 || c->impl > 2) return MLA_ERR_CONFIG;
+    if (!(c->scale == c->scale)) return MLA_ERR_CONFIG;  // NaN
+    return MLA_OK;
+}
+
+float effective_scale(const mla_config_t* c) {
+    return c->scale > 0.f ? c->scale : static_cast<float>(1.0 / sqrt(static_cast<double>(c->d_h + c->d_r)));
+}
+
+int choose_splits(const mla_config_t* c, int B, int T_q, int max_splits) {
+    if (max_splits > 0) return max_splits < kMaxSplits ? max_splits : kMaxSplits;
+    const long work = static_cast<long>(B) * T_q * ((c->n_h + 7) / 8);
+    long s = (8L * kB200Sms + work - 1) / work;
+    if (s < 1) s = 1;
+    if (s > 64) s = 64;
+    return static_cast<int>(s);
+}
+
+struct WsLayout {
+    size_t part_o, part_lse, sm100, total;
+};
+
+WsLayout ws_layout(const mla_config_t* c, int B, int T_q, int splits) {
+    WsLayout w;
+    const size_t rows = static_cast<size_t>(B) * T_q * c->n_h;
+    const size_t simt_o = splits > 1 ? round256(static_cast<size_t>(splits) * rows * c->d_c * 4) : 0;
+    const size_t simt_l = splits > 1 ? round256(static_cast<size_t>(splits) * rows * 4) : 0;
+    w.part_o = 256;
+    w.part_lse = w.part_o + simt_o;
+    w.sm100 = w.part_lse + simt_l;
+    w.total = w.sm100 + round256(mla::sm100_workspace_bytes(c->n_h, c->d_c, B, T_q));
+    return w;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_LAUNCH; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_str(int code) {
+    switch (code) {
+        case MLA_OK: return "ok";
+        case MLA_ERR_NULL: return "null pointer";
+        case MLA_ERR_CONFIG: return "unsupported configuration";
+        case MLA_ERR_SIZE: return "size out of range";
+        case MLA_ERR_WORKSPACE: return "workspace too small or misaligned";
+        case MLA_ERR_LAUNCH: return "CUDA launch or runtime error";
+        case MLA_ERR_UNSUPPORTED: return "device or feature not supported";
+        case MLA_ERR_ALIGN: return "pointer not 16-byte aligned";
+        default: return "unknown status";
+    }
+}
+
+int mla_check_device(void) {
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_UNSUPPORTED;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MLA_ERR_UNSUPPORTED;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return MLA_ERR_UNSUPPORTED;
+    return (major == 10 && minor == 0) ? MLA_OK : MLA_ERR_UNSUPPORTED;
+}
+
+int mla_rope_table(int d_r, double base, int max_pos, float* host_table) {
+    if (host_table == nullptr) return MLA_ERR_NULL;
+    if (d_r < 2 || d_r % 2 || max_pos < 1 || !(base > 0.0)) return MLA_ERR_SIZE;
+    const int h = d_r / 2;
+    for (int m = 0; m < h; ++m) {
+        const double f = pow(base, -2.0 * m / d_r);
+        for (int p = 0; p < max_pos; ++p) {
+            const double th = static_cast<double>(p) * f;
+            host_table[static_cast<size_t>(p) * d_r + m] = static_cast<float>(cos(th));
+            host_table[static_cast<size_t>(p) * d_r + h + m] = static_cast<float>(sin(th));
+        }
+    }
+    return MLA_OK;
+}
+
+int mla_absorb_q(const mla_config_t* cfg, const mla_bf16* q_c, const mla_bf16* w_uk,
+                 mla_bf16* q_abs, int n_tok, void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!q_c || !w_uk || !q_abs) return MLA_ERR_NULL;
+    if (!aligned16(q_c) || !aligned16(w_uk) || !aligned16(q_abs)) return MLA_ERR_ALIGN;
+    if (n_tok < 1 || n_tok > 65536) return MLA_ERR_SIZE;
+    return cuda_rc(mla::launch_absorb_q_simt(q_c, w_uk, q_abs, n_tok, cfg->n_h, cfg->d_h, cfg->d_c,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+int mla_rope_append(const mla_config_t* cfg, mla_bf16* q_r, const mla_bf16* k_r,
+                    const mla_bf16* c_kv, const int32_t* positions, const float* rope_table,
+                    int max_pos, const int32_t* block_table, int max_blocks_per_seq,
+                    mla_bf16* pool, int num_blocks, int B, int T_q, int32_t* dev_status,
+                    void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!k_r || !c_kv || !positions || !rope_table || !block_table || !pool) return MLA_ERR_NULL;
+    if ((q_r && !aligned16(q_r)) || !aligned16(k_r) || !aligned16(c_kv) || !aligned16(pool))
+        return MLA_ERR_ALIGN;
+    if (!aligned4(positions) || !aligned4(rope_table) || !aligned4(block_table) ||
+        (dev_status && !aligned4(dev_status)))
+        return MLA_ERR_ALIGN;
+    if (B < 1 || T_q < 1 || static_cast<long>(B) * T_q > (1L << 24)) return MLA_ERR_SIZE;
+    if (max_pos < 1 || max_blocks_per_seq < 1 || num_blocks < 1) return MLA_ERR_SIZE;
+    return cuda_rc(mla::launch_rope_append(q_r, k_r, c_kv, positions, rope_table, max_pos, block_table,
+                                           max_blocks_per_seq, pool, num_blocks, B * T_q, T_q,
+                                           cfg->n_h, cfg->d_c, cfg->d_r, cfg->block_size, dev_status,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+size_t mla_decode_workspace_bytes(const mla_config_t* cfg, int B, int T_q, int max_splits) {
+    if (check_config(cfg) || B < 1 || T_q < 1 || max_splits < 0) return 0;
+    return ws_layout(cfg, B, T_q, choose_splits(cfg, B, T_q, max_splits)).total;
+}
+
+int mla_decode(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q_r,
+               const mla_bf16* pool, int num_blocks, const int32_t* block_table,
+               int max_blocks_per_seq, const int32_t* seq_lens, int B, int T_q, int max_splits,
+               void* workspace, size_t ws_bytes, mla_bf16* out_latent, float* out_lse,
+               void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!q_abs || !q_r || !pool || !block_table || !seq_lens || !workspace || !out_latent || !out_lse)
+        return MLA_ERR_NULL;
+    if (!aligned16(q_abs) || !aligned16(q_r) || !aligned16(pool) || !aligned16(out_latent) ||
+        !aligned4(out_lse) || !aligned4(block_table) || !aligned4(seq_lens))
+        return MLA_ERR_ALIGN;
+    if (B < 1 || T_q < 1 || T_q > 16 || static_cast<long>(B) * T_q > 65535) return MLA_ERR_SIZE;
+    if (num_blocks < 1 || max_blocks_per_seq < 1 || max_splits < 0) return MLA_ERR_SIZE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLA_ERR_WORKSPACE;
+    const int splits = choose_splits(cfg, B, T_q, max_splits);
+    const WsLayout w = ws_layout(cfg, B, T_q, splits);
+    if (ws_bytes < w.total) return MLA_ERR_WORKSPACE;
+
+    char* ws = static_cast<char*>(workspace);
+    DecodeParams P;
+    P.q_abs = q_abs;
+    P.q_r = q_r;
+    P.pool = pool;
+    P.block_table = block_table;
+    P.seq_lens = seq_lens;
+    P.out_latent = out_latent;
+    P.out_lse = out_lse;
+    P.part_o = reinterpret_cast<float*>(ws + w.part_o);
+    P.part_lse = reinterpret_cast<float*>(ws + w.part_lse);
+    P.status = reinterpret_cast<int32_t*>(ws);
+    P.n_h = cfg->n_h;
+    P.d_c = cfg->d_c;
+    P.d_r = cfg->d_r;
+    P.block_size = cfg->block_size;
+    P.num_blocks = num_blocks;
+    P.max_blocks = max_blocks_per_seq;
+    P.B = B;
+    P.T_q = T_q;
+    P.n_tok = B * T_q;
+    P.splits = splits;
+    P.scale_log2 = effective_scale(cfg) * mla::kLog2e;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    const bool sm100_shape = mla::sm100_supports(cfg->n_h, cfg->d_c, cfg->d_r);
+    if (cfg->impl == 2 && !sm100_shape) return MLA_ERR_CONFIG;
+    const bool use_sm100 = cfg->impl == 2 || (cfg->impl == 0 && sm100_shape);
+    if (use_sm100) {
+        if (mla_check_device() != MLA_OK) return MLA_ERR_UNSUPPORTED;
+        return cuda_rc(mla::launch_decode_sm100(P, ws + w.sm100, max_splits, st));
+    }
+    return cuda_rc(mla::launch_decode_simt(P, st));
+}
+
+int mla_decode_launches(const mla_config_t* cfg, int B, int T_q, int max_splits) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (B < 1 || T_q < 1 || T_q > 16 || max_splits < 0) return MLA_ERR_SIZE;
+    const bool sm100_shape = mla::sm100_supports(cfg->n_h, cfg->d_c, cfg->d_r);
+    if (cfg->impl == 2 && !sm100_shape) return MLA_ERR_CONFIG;
+    if (cfg->impl == 2 || (cfg->impl == 0 && sm100_shape))
+        return mla::sm100_launches(B, T_q, max_splits);
+    return choose_splits(cfg, B, T_q, max_splits) > 1 ? 2 : 1;
+}
+
+int mla_up_v(const mla_config_t* cfg, const mla_bf16* latent, const mla_bf16* w_uv, mla_bf16* out,
+             int n_tok, void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!latent || !w_uv || !out) return MLA_ERR_NULL;
+    if (!aligned16(latent) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_ALIGN;
+    if (n_tok < 1 || n_tok > 65536) return MLA_ERR_SIZE;
+    return cuda_rc(mla::launch_up_v_simt(latent, w_uv, out, n_tok, cfg->n_h, cfg->d_h, cfg->d_c,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int mla_clear_status(int32_t* dev_status, void* stream) {
+    if (!dev_status) return MLA_ERR_NULL;
+    return cuda_rc(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)));
+}
+
+int mla_read_status(const int32_t* dev_status, int32_t* host_status, void* stream) {
+    if (!dev_status || !host_status) return MLA_ERR_NULL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(host_status, dev_status, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return MLA_ERR_LAUNCH;
+    return cuda_rc(cudaStreamSynchronize(st));
+}
+
+}  // extern "C"

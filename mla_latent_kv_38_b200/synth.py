@@ -118,3 +118,59 @@ def permutation(seed: int, n: int) -> np.ndarray:
 def weight_std(fan_in: int) -> float:
     """Standard deviation 1/sqrt(fan_in) for the up-projection weights."""
     return 1.0 / float(np.sqrt(fan_in))
+
+
+# ---------------------------------------------------------------------------
+# The same generator evaluated with torch on a CUDA device, for bulk inputs.
+# Integer steps use int64 with wrapping multiplication (the same bits as the
+# unsigned arithmetic above) and masked shifts for the logical right shifts.
+# ---------------------------------------------------------------------------
+
+def _i64(v: int) -> int:
+    v &= (1 << 64) - 1
+    return v - (1 << 64) if v >= (1 << 63) else v
+
+
+def _torch_mix(z):
+    import torch
+
+    def shr(x, k):
+        return (x >> k) & ((1 << (64 - k)) - 1)
+
+    z = (z ^ shr(z, 30)) * _i64(int(_M1))
+    z = (z ^ shr(z, 27)) * _i64(int(_M2))
+    return z ^ shr(z, 31)
+
+
+def normal_bf16_torch(seed: int, tid: int, count: int, start: int = 0, std: float = 1.0,
+                      device="cuda", chunk: int = 1 << 24):
+    """bf16 tensor of `count` draws for flat indices [start, start+count); the
+    same values as :func:`normal_bf16` up to the last bit of the float64
+    log/cos, which bf16 rounding hides except with probability ~2^-44."""
+    import torch
+
+    key = _i64(int(_key(seed, tid)))
+    golden = _i64(int(_GOLDEN))
+    out = torch.empty(count, dtype=torch.bfloat16, device=device)
+    for c0 in range(0, count, chunk):
+        n = min(chunk, count - c0)
+        i = torch.arange(start + c0, start + c0 + n, dtype=torch.int64, device=device)
+        u1 = _torch_mix(key + (2 * i + 1) * golden)
+        u2 = _torch_mix(key + (2 * i + 2) * golden)
+        f1 = ((u1 >> 11) & ((1 << 53) - 1)).to(torch.float64).add_(1.0).mul_(1.0 / 9007199254740992.0)
+        f2 = ((u2 >> 11) & ((1 << 53) - 1)).to(torch.float64).add_(1.0).mul_(1.0 / 9007199254740992.0)
+        z = torch.sqrt(-2.0 * torch.log(f1)) * torch.cos((2.0 * np.pi) * f2) * std
+        out[c0:c0 + n] = _torch_f64_to_bf16(z)
+    return out
+
+
+def _torch_f64_to_bf16(z):
+    """float64 -> bf16 with one rounding (round half to even on the float64
+    significand), matching :func:`to_bf16_bits`."""
+    import torch
+
+    b = z.view(torch.int64)
+    lsb = (b >> 45) & 1
+    r = (b + ((1 << 44) - 1) + lsb) & ~((1 << 45) - 1)
+    f = r.view(torch.float64).to(torch.float32)  # exact
+    return f.to(torch.bfloat16)                  # exact

@@ -1,0 +1,94 @@
+"""CPU-side checks of the C ABI library: it builds for sm_100a, loads, exports
+every function include/mla.h declares, and rejects bad arguments on the host
+before touching a device (so these calls are safe without a GPU)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from mla_latent_kv_38_b200 import build
+from oracle import mla_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def M():
+    build.build()
+    from mla_latent_kv_38_b200 import binding
+    return binding
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "mla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(M):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(M._lib, n), n
+    assert set(M.EXPORTED) == set(names)
+
+
+def test_status_strings(M):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
+        assert M.mla_status_str(code) not in ("", "unknown status")
+    assert M.mla_status_str(-99) == "unknown status"
+
+
+def test_library_rope_table_matches_oracle_table(M):
+    for d_r, max_pos in ((16, 300), (64, 5000)):
+        lib = M.mla_rope_table(d_r, 10000.0, max_pos).numpy()
+        ref = O.rope_table_f32(max_pos, d_r)
+        ulps = np.abs(lib.view(np.int32).astype(np.int64) - ref.view(np.int32).astype(np.int64))
+        assert ulps.max() <= 1
+        assert (ulps > 0).mean() < 1e-3
+
+
+FAKE = 0x10000  # 16-byte aligned non-null value; never dereferenced by these calls
+
+
+def _cfg(M, **kw):
+    base = dict(n_h=128, d_c=512, d_h=128, d_r=64)
+    base.update(kw)
+    return M.MlaConfig(**base)
+
+
+def test_host_validation_without_device(M):
+    raw = M.raw_call
+    cfg = _cfg(M)
+    bad_block = _cfg(M, block_size=32)
+    bad_dc = _cfg(M, d_c=520)
+    p = ctypes.c_void_p(FAKE)
+    assert raw("mla_absorb_q", ctypes.byref(bad_block), p, p, p, 4, None) == -2
+    assert raw("mla_absorb_q", ctypes.byref(bad_dc), p, p, p, 4, None) == -2
+    assert raw("mla_absorb_q", ctypes.byref(cfg), None, p, p, 4, None) == -1
+    assert raw("mla_absorb_q", ctypes.byref(cfg), ctypes.c_void_p(FAKE + 2), p, p, 4, None) == -7
+    assert raw("mla_absorb_q", ctypes.byref(cfg), p, p, p, 0, None) == -3
+    assert raw("mla_up_v", ctypes.byref(cfg), p, p, p, 70000, None) == -3
+    ws = M.mla_decode_workspace_bytes(cfg, 32, 1, 0)
+    assert ws >= 256 and ws % 256 == 0
+    assert M.mla_decode_workspace_bytes(cfg, 32, 1, 4) >= M.mla_decode_workspace_bytes(cfg, 32, 1, 1)
+    args = [ctypes.byref(cfg), p, p, p, 10, p, 1, p, 32, 1, 0, p, ws - 1, p, p, None]
+    assert raw("mla_decode", *args) == -4
+    args[12] = ws
+    args[11] = ctypes.c_void_p(FAKE + 16)          # workspace must be 256-byte aligned
+    assert raw("mla_decode", *args) == -4
+    args[11] = p
+    args[9] = 17                                    # T_q > 16
+    assert raw("mla_decode", *args) == -3
+    args[9] = 1
+    args[1] = None
+    assert raw("mla_decode", *args) == -1
+    impl_tc_tiny = _cfg(M, n_h=4, d_c=64, d_h=32, d_r=16, impl=2)
+    args = [ctypes.byref(impl_tc_tiny), p, p, p, 10, p, 1, p, 1, 1, 0, p,
+            M.mla_decode_workspace_bytes(impl_tc_tiny, 1, 1, 0), p, p, None]
+    assert raw("mla_decode", *args) == -2           # tcgen05 kernel needs the V2 shape
+    assert raw("mla_rope_table", 64, ctypes.c_double(10000.0), 0, p) == -3
+    assert raw("mla_clear_status", None, None) == -1

@@ -1,0 +1,216 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Bars: bit-exact for the cache append and the page-table gather; for floating
+point, max-abs error <= 2e-2 and mean relative error sum|gpu-ref|/sum|ref|
+<= 5e-3 on the head output o and on the latent output, and |lse error| <= 1e-2.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from mla_latent_kv_38_b200.workloads import CaseSpec, config_specs
+from oracle import mla_oracle as O
+from oracle.evaluate import reference
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+MEAN_REL = 5e-3
+LSE_ABS = 1e-2
+
+
+@pytest.fixture(scope="module")
+def M():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from mla_latent_kv_38_b200 import build
+    build.build()
+    from mla_latent_kv_38_b200 import binding
+    return binding
+
+
+def _dc(spec, **kw):
+    from mla_latent_kv_38_b200.runner import DeviceCase
+    return DeviceCase(spec, **kw)
+
+
+def _f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def assert_close(got, want, what):
+    err = np.abs(got - want)
+    max_abs = float(err.max())
+    mre = float(err.sum() / max(np.abs(want).sum(), 1e-300))
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    assert max_abs <= MAX_ABS and mre <= MEAN_REL, f"{what}: max_abs={max_abs:.3e} mean_rel={mre:.3e}"
+    return max_abs, mre
+
+
+def check_sequences(dc, seqs, heads=None):
+    s = dc.spec
+    out = _f64(dc.out).reshape(s.B, s.T_q, s.n_h, s.d_h)
+    lat = _f64(dc.latent).reshape(s.B, s.T_q, s.n_h, s.d_c)
+    lse = dc.lse.cpu().numpy().astype(np.float64).reshape(s.B, s.T_q, s.n_h)
+    hs = list(range(s.n_h)) if heads is None else list(heads)
+    for b in seqs:
+        ref = reference(s, b, heads=hs)
+        assert_close(out[b][:, hs], ref["o"], f"o seq {b}")
+        assert_close(lat[b][:, hs], ref["latent"], f"latent seq {b}")
+        d = np.abs(lse[b][:, hs] - ref["lse"]).max()
+        assert d <= LSE_ABS, f"lse seq {b}: {d:.3e}"
+
+
+V2 = dict(n_h=128, d_c=512, d_h=128, d_r=64)
+
+SMALL_CASES = {
+    "tiny_config": config_specs()["tiny"],
+    "v2_ragged": CaseSpec(**V2, seq_lens=np.array([1, 63, 64, 65, 300], np.int32), seed=1),
+    "v2_permuted": CaseSpec(**V2, seq_lens=np.array([700, 129, 2], np.int32), seed=2,
+                            permute_blocks=True),
+    "v2_multi_token": CaseSpec(**V2, seq_lens=np.array([4, 5, 67, 200], np.int32), T_q=4, seed=3),
+    "tiny_multi_token": CaseSpec(n_h=4, d_c=64, d_h=32, d_r=16,
+                                 seq_lens=np.array([2, 64, 129], np.int32), T_q=2, seed=4),
+    "odd_heads": CaseSpec(n_h=12, d_c=128, d_h=64, d_r=32, seq_lens=np.array([33, 97], np.int32),
+                          seed=5),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL_CASES))
+@pytest.mark.parametrize("impl", [0, 1])
+def test_full_path_small(M, name, impl):
+    spec = SMALL_CASES[name]
+    dc = _dc(spec, impl=impl)
+    dc.step()
+    torch.cuda.synchronize()
+    assert dc.decode_status() == 0 and dc.append_status() == 0
+    check_sequences(dc, range(spec.B))
+
+
+@pytest.mark.parametrize("name", sorted(SMALL_CASES))
+def test_append_and_gather_bit_exact(M, name):
+    spec = SMALL_CASES[name]
+    dc = _dc(spec)
+    dc.step()
+    torch.cuda.synchronize()
+    pool = dc.bits(dc.pool)
+    table = dc.block_table_np
+    tab = O.rope_table_f32(dc.max_pos, spec.d_r)
+    for b, L in enumerate(spec.seq_lens):
+        L = int(L)
+        rows = O.gather_rows(pool, table, b, L, spec.block_size)     # through the block table
+        assert np.array_equal(rows[:, :spec.d_c], spec.c_kv_rows(b, 0, L))
+        want_kr = O.rope_emulate_bf16(spec.k_r_rows(b, 0, L), np.arange(L), tab)
+        assert np.array_equal(rows[:, spec.d_c:], want_kr)
+    # the step's query RoPE, in place
+    q_r = dc.bits(dc.q_r)
+    want_q = O.rope_emulate_bf16(spec.q_r(), spec.positions()[:, None], tab)
+    assert np.array_equal(q_r, want_q)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 7])
+@pytest.mark.parametrize("impl", [0, 1])
+def test_split_count_invariance(M, splits, impl):
+    spec = CaseSpec(**V2, seq_lens=np.array([1000, 37, 513], np.int32), seed=6)
+    dc = _dc(spec, impl=impl, max_splits=splits)
+    dc.step()
+    torch.cuda.synchronize()
+    check_sequences(dc, range(spec.B))
+
+
+def test_absorb_q_parity(M):
+    spec = CaseSpec(**V2, seq_lens=np.array([64] * 5, np.int32), T_q=3, seed=7)
+    dc = _dc(spec, fill_history=False)
+    M.mla_absorb_q(dc.cfg, dc.q_c, dc.w_uk, dc.q_abs, spec.n_tok)
+    torch.cuda.synchronize()
+    want = O.absorb_q(O.bf16_to_f64(spec.q_c()), O.bf16_to_f64(spec.w_uk()))
+    assert_close(_f64(dc.q_abs), want, "q_abs")
+
+
+def test_up_v_parity(M):
+    from mla_latent_kv_38_b200 import synth
+    spec = CaseSpec(**V2, seq_lens=np.array([64] * 9, np.int32), seed=8)
+    dc = _dc(spec, fill_history=False)
+    lat_bits = synth.normal_bf16(8, 99, (spec.n_tok, spec.n_h, spec.d_c), std=0.05)
+    lat = torch.from_numpy(lat_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    M.mla_up_v(dc.cfg, lat, dc.w_uv, dc.out, spec.n_tok)
+    torch.cuda.synchronize()
+    want = O.up_v(O.bf16_to_f64(lat_bits), O.bf16_to_f64(spec.w_uv()))
+    assert_close(_f64(dc.out), want, "up_v")
+
+
+def test_device_checks_flag_bad_rows(M):
+    spec = CaseSpec(**V2, seq_lens=np.array([130, 70], np.int32), seed=9)
+    dc = _dc(spec)
+    # sequence 1 claims fewer rows than its query tokens need
+    dc.seq_lens[1] = 0
+    M.mla_clear_status(dc.ws)
+    dc.decode_only()
+    assert dc.decode_status() & M.MLA_STATUS_BAD_SEQ_LEN
+    # a block-table entry outside the pool
+    dc.seq_lens[1] = 70
+    dc.block_table[0, 1] = spec.num_blocks + 5
+    M.mla_clear_status(dc.ws)
+    dc.decode_only()
+    assert dc.decode_status() & M.MLA_STATUS_BAD_BLOCK
+    # an append through the bad entry (sequence 0, block 1) and one position
+    # beyond the RoPE table (sequence 1): both rows skipped and flagged
+    M.mla_clear_status(dc.status)
+    dc.positions[0] = 64 + 3
+    dc.positions[1] = dc.max_pos + 1
+    dc.step()
+    st = dc.append_status()
+    assert st & M.MLA_STATUS_BAD_POSITION and st & M.MLA_STATUS_BAD_BLOCK
+    torch.cuda.synchronize()
+
+
+def test_host_argument_errors(M):
+    spec = CaseSpec(**V2, seq_lens=np.array([64], np.int32), seed=10)
+    dc = _dc(spec, fill_history=False)
+    with pytest.raises(M.MlaError) as e:
+        M.mla_decode(dc.cfg, dc.q_abs, dc.q_r, dc.pool, spec.num_blocks, dc.block_table,
+                     spec.max_blocks, dc.seq_lens, 1, 1, 0, dc.ws, 16, dc.latent, dc.lse)
+    assert e.value.code == -4
+    with pytest.raises(M.MlaError) as e:
+        M.mla_decode(dc.cfg, dc.q_abs, dc.q_r, dc.pool, spec.num_blocks, dc.block_table,
+                     spec.max_blocks, dc.seq_lens, 1, 17, 0, dc.ws, dc.ws_bytes, dc.latent, dc.lse)
+    assert e.value.code == -3
+    bad = M.MlaConfig(128, 512, 128, 64, block_size=32)
+    with pytest.raises(M.MlaError) as e:
+        M.mla_absorb_q(bad, dc.q_c, dc.w_uk, dc.q_abs, 1)
+    assert e.value.code == -2
+
+
+# ---------------------------------------------------------------------------
+# Full sizes of the five workloads, in the benchmark's launch configuration,
+# checked on sampled sequences and heads.
+# ---------------------------------------------------------------------------
+
+FULL = {
+    "v2_decode": ([0, 17, 31], [0, 1, 63, 64, 127]),
+    "varlen": ([0, 5, 77, 127], [0, 64, 127]),
+    "long": ([0, 3], [0, 127]),
+    "multi_token": ([0, 63], [0, 65, 127]),
+    "tiny": ([0], None),
+}
+
+
+@pytest.mark.parametrize("name", ["tiny", "v2_decode", "multi_token", "long", "varlen"])
+def test_full_size_sampled(M, name):
+    spec = config_specs()[name]
+    seqs, heads = FULL[name]
+    dc = _dc(spec)
+    dc.step()
+    torch.cuda.synchronize()
+    assert dc.decode_status() == 0 and dc.append_status() == 0
+    check_sequences(dc, seqs, heads)
+    # page-table gather of the sampled sequences' cache rows, bit exact
+    pool = dc.bits(dc.pool)
+    tab = O.rope_table_f32(dc.max_pos, spec.d_r)
+    for b in seqs[:2]:
+        L = int(spec.seq_lens[b])
+        rows = O.gather_rows(pool, dc.block_table_np, b, L, spec.block_size)
+        assert np.array_equal(rows[:, :spec.d_c], spec.c_kv_rows(b, 0, L))
+        assert np.array_equal(rows[:, spec.d_c:],
+                              O.rope_emulate_bf16(spec.k_r_rows(b, 0, L), np.arange(L), tab))
