@@ -167,6 +167,36 @@ int mla_decode(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q
  * (decode, optional scheduling and merge kernels); negative on bad arguments. */
 int mla_decode_launches(const mla_config_t* cfg, int B, int T_q, int max_splits);
 
+/* mla_decode for callers that cannot allocate device memory: the pages have
+ * no counterpart; this is a deployment variant of the same computation.
+ * Callers inside frameworks that own every device allocation, plugins that
+ * are handed only their input and output buffers, or hosts that must not grow
+ * device memory after start-up cannot provide mla_decode's workspace.  This
+ * call takes no workspace and allocates nothing: it runs the portable decode
+ * kernel (the impl = 1 kernel, whatever cfg->impl says) and keeps its split-KV
+ * partial results in a fixed 16 MiB device array inside this library, which
+ * every GPU that loads the library holds until the process exits.
+ *   Arguments as for mla_decode, except:
+ *   splits      key-range splits per query row, 1..256 (no automatic choice);
+ *               when splits > 1 the partials need
+ *               splits * B * T_q * n_h * (4 * d_c + 4) bytes (plus 256-byte
+ *               rounding) and a call needing more than 16 MiB returns
+ *               MLA_ERR_SIZE without launching anything.
+ *   dev_status  optional device int32 that device-side checks OR
+ *               MLA_STATUS_* bits into (NULL: not reported).
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  All calls share the one array, which
+ * keeps the last call's contents (each call fully writes what it reads, so
+ * nothing needs clearing); calls that overlap on the GPU, on different streams
+ * or from different host threads, race on it and must be serialised by the
+ * caller. */
+int mla_decode_noalloc(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q_r,
+                       const mla_bf16* pool, int num_blocks, const int32_t* block_table,
+                       int max_blocks_per_seq, const int32_t* seq_lens, int B, int T_q,
+                       int splits, mla_bf16* out_latent, float* out_lse,
+                       int32_t* dev_status, void* stream);
+
 /* o[n, i, :] = W^UV_i latent[n, i, :]  ([notes] "Value에 대한 수식 전개").
  *   latent (n_tok, n_h, d_c) bf16;  w_uv (n_h, d_h, d_c) bf16
  *   out    (n_tok, n_h, d_h) bf16 (float accumulation, RNE rounding) */

@@ -27,7 +27,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 EXPORTED = (
     "mla_status_str", "mla_check_device", "mla_rope_table", "mla_absorb_q",
     "mla_rope_append", "mla_decode_workspace_bytes", "mla_decode", "mla_decode_launches",
-    "mla_up_v",
+    "mla_decode_noalloc", "mla_up_v",
     "mla_clear_status", "mla_read_status",
 )
 
@@ -73,6 +73,8 @@ _lib.mla_decode_workspace_bytes.restype = _sz
 _lib.mla_decode_workspace_bytes.argtypes = [_cfgp, _i, _i, _i]
 _lib.mla_decode.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, _vp, _sz, _vp, _vp, _vp]
 _lib.mla_decode_launches.argtypes = [_cfgp, _i, _i, _i]
+_lib.mla_decode_noalloc.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp,
+                                    _vp]
 _lib.mla_up_v.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp]
 _lib.mla_clear_status.argtypes = [_vp, _vp]
 _lib.mla_read_status.argtypes = [_vp, _vp, _vp]
@@ -146,6 +148,17 @@ def mla_decode_launches(cfg: MlaConfig, B: int, T_q: int, max_splits: int = 0) -
     if n < 0:
         raise MlaError("mla_decode_launches", n)
     return n
+
+
+def mla_decode_noalloc(cfg: MlaConfig, q_abs, q_r, pool, num_blocks: int, block_table,
+                       max_blocks_per_seq: int, seq_lens, B: int, T_q: int, splits: int,
+                       out_latent, out_lse, dev_status=None, stream=None):
+    """mla_decode without a workspace, for callers that cannot allocate: the
+    split partials live in the library's fixed 16 MiB device array."""
+    _check("mla_decode_noalloc", _lib.mla_decode_noalloc(
+        ctypes.byref(cfg), _ptr(q_abs), _ptr(q_r), _ptr(pool), int(num_blocks), _ptr(block_table),
+        int(max_blocks_per_seq), _ptr(seq_lens), int(B), int(T_q), int(splits), _ptr(out_latent),
+        _ptr(out_lse), _ptr(dev_status), _stream(stream)))
 
 
 def mla_up_v(cfg: MlaConfig, latent, w_uv, out, n_tok: int, stream=None):
