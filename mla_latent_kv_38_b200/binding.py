@@ -16,7 +16,7 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmla_b200.so")
+LIB_PATH = os.environ.get("MLA_B200_LIB") or os.path.join(_HERE, "libmla_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(

@@ -46,50 +46,59 @@ namespace mla {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kStages = 2;
 constexpr int kClusters = 74;                     // 148 SMs / 2
 constexpr int kDc = 512, kDr = 64, kRow = 576;    // row = c^KV || k^R
-constexpr int kBlk = 64;                          // keys per page = per tile
+constexpr int kPage = 64;                         // cache rows per page
+constexpr int kTile = 32;                         // keys per tile (half a page)
+constexpr int kStages = 4;                        // TMA ring depth
+constexpr int kSBuf = 4;                          // S accumulators in tensor memory
+constexpr int kPBuf = 2;                          // P operand buffers
 
-constexpr uint32_t kChunk = 8192;                 // 64 rows x 128 B
-constexpr uint32_t kQBytes = 9 * kChunk;          // 64 heads x 576
-constexpr uint32_t kSRegion = 9 * 4096;           // 32 keys x 576
-constexpr uint32_t kVRegion = 4 * kChunk;         // 64 keys x 256 latent columns
+constexpr uint32_t kQChunk = 8192;                // 64 heads x 128 B
+constexpr uint32_t kQBytes = 9 * kQChunk;         // 64 heads x 576 columns
+constexpr uint32_t kSChunk = 2048;                // 16 keys x 128 B
+constexpr uint32_t kSRegion = 9 * kSChunk;        // this CTA's 16 keys x 576
+constexpr uint32_t kVSlot = 4096;                 // 32 keys x 128 B
+constexpr uint32_t kVRegion = 4 * kVSlot;         // 32 keys x 256 latent columns
 constexpr uint32_t kStageBytes = kSRegion + kVRegion;
+constexpr uint32_t kPBytes = 4096;                // 64 heads x 32 keys bf16 (64-byte swizzle)
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffStage = kOffQ + kQBytes;
 constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;
-constexpr uint32_t kOffXmax = kOffP + kChunk;     // 2 x 128 floats
-constexpr uint32_t kOffXsum = kOffXmax + 1024;    // 128 floats
+constexpr uint32_t kOffXmax = kOffP + kPBuf * kPBytes;   // 2 x 128 floats
+constexpr uint32_t kOffXsum = kOffXmax + 1024;           // 128 floats
 constexpr uint32_t kOffBar = kOffXsum + 512;
-constexpr uint32_t kOffMisc = kOffBar + 8 * 16;   // tmem base, abort flag
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+constexpr uint32_t kOffMisc = kOffBar + 8 * 32;          // tmem base, abort flag
+constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;    // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 enum {
     BAR_Q_FULL = 0,
     BAR_Q_EMPTY = 1,
-    BAR_KV_FULL = 2,   // + stage
-    BAR_KV_EMPTY = 4,  // + stage
-    BAR_S_FULL = 6,    // + buffer
-    BAR_S_FREE = 8,    // + buffer
-    BAR_P_FULL = 10,
-    BAR_P_FREE = 11,
-    BAR_DRAIN = 12
+    BAR_KV_FULL = 2,                     // + stage
+    BAR_KV_EMPTY = BAR_KV_FULL + kStages,
+    BAR_S_FULL = BAR_KV_EMPTY + kStages, // + S buffer
+    BAR_S_FREE = BAR_S_FULL + kSBuf,
+    BAR_P_FULL = BAR_S_FREE + kSBuf,     // + P buffer
+    BAR_P_FREE = BAR_P_FULL + kPBuf,
+    BAR_DRAIN = BAR_P_FREE + kPBuf,
+    NUM_BARS = BAR_DRAIN + 1
 };
+static_assert(NUM_BARS <= 32, "barrier area");
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 0;
-constexpr uint32_t kTmemS = 256;
+constexpr uint32_t kTmemO = 0;                    // 2 x 128 columns (paired layout)
+constexpr uint32_t kTmemS = 256;                  // kSBuf x 16 columns
 
-constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 64, 0, 0);
+constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, kTile, 0, 0);
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 256, 0, 1);
 
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
 
 struct Sm100Params {
-    CUtensorMap tm_pool_s;    // pool as [rows][576], box 64 cols x 32 rows
-    CUtensorMap tm_pool_v;    // pool as [rows][576], box 64 cols x 64 rows
+    CUtensorMap tm_pool_s;    // pool as [rows][576], box 64 cols x 16 rows
+    CUtensorMap tm_pool_v;    // pool as [rows][576], box 64 cols x 32 rows
     CUtensorMap tm_qa;        // q_abs as [n_tok*n_h][512], box 64 x 64
     CUtensorMap tm_qr;        // q_r   as [n_tok*n_h][64],  box 64 x 64
     const int32_t* block_table;
@@ -121,7 +130,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, volatil
     }
 }
 
-// First unit whose tile range contains global tile g (prefix is non-decreasing).
+// Unit whose tile range contains global tile g (prefix is non-decreasing).
 __device__ __forceinline__ int find_unit(const int32_t* prefix, int U, int g) {
     int lo = 0, hi = U - 1;
     while (lo < hi) {
@@ -131,7 +140,33 @@ __device__ __forceinline__ int find_unit(const int32_t* prefix, int U, int g) {
     return lo;
 }
 
-// latent column chunk (64 wide) that V-region slot i of CTA `rank` holds
+// Walks a cluster's tiles [g0, g1) unit by unit.
+struct TileCursor {
+    const int32_t* prefix;
+    int g, g0, g1, u;
+    __device__ void init(const int32_t* pf, int U, int g0_, int g1_) {
+        prefix = pf;
+        g = g0_;
+        g0 = g0_;
+        g1 = g1_;
+        u = g0_ < g1_ ? find_unit(pf, U, g0_) : 0;
+        skip();
+    }
+    __device__ void skip() {
+        while (g < g1 && prefix[u + 1] <= g) ++u;
+    }
+    __device__ bool done() const { return g >= g1; }
+    __device__ int j() const { return g - prefix[u]; }   // tile index within the unit
+    __device__ bool seg_first() const { return g == g0 || g == prefix[u]; }
+    __device__ bool seg_last() const { return g + 1 == g1 || g + 1 == prefix[u + 1]; }
+    __device__ void next() {
+        ++g;
+        skip();
+    }
+};
+
+// latent column chunk (64 wide) that V-region slot i of CTA `rank` holds:
+// P.V instruction h takes N columns [0,128) from CTA 0 and [128,256) from CTA 1
 __device__ __forceinline__ int owned_chunk(uint32_t rank, int i) {
     return 4 * (i >> 1) + 2 * static_cast<int>(rank) + (i & 1);
 }
@@ -158,12 +193,14 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             ptx::mbar_init(bar(BAR_KV_FULL + s), 1);
             ptx::mbar_init(bar(BAR_KV_EMPTY + s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kSBuf; ++b) {
             ptx::mbar_init(bar(BAR_S_FULL + b), 1);
-            ptx::mbar_init(bar(BAR_S_FREE + b), 8);
+            ptx::mbar_init(bar(BAR_S_FREE + b), 8);   // 4 softmax warps x 2 CTAs
         }
-        ptx::mbar_init(bar(BAR_P_FULL), 8);
-        ptx::mbar_init(bar(BAR_P_FREE), 1);
+        for (int b = 0; b < kPBuf; ++b) {
+            ptx::mbar_init(bar(BAR_P_FULL + b), 8);
+            ptx::mbar_init(bar(BAR_P_FREE + b), 1);
+        }
         ptx::mbar_init(bar(BAR_DRAIN), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -196,101 +233,119 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         if (lane == 0 && g0 < g1) {
             const uint64_t pol_stream = ptx::l2_policy_evict_first();
             const uint64_t pol_q = ptx::l2_policy_evict_last();
+            TileCursor c;
+            c.init(p.prefix, p.U, g0, g1);
             int it = 0, uc = 0;
-            int u = find_unit(p.prefix, p.U, g0);
-            for (int g = g0; g < g1; ++u) {
-                const int ubeg = p.prefix[u], uend = p.prefix[u + 1];
-                if (uend <= g) continue;
-                const int t0 = g - ubeg, t1 = min(g1, uend) - ubeg;
-                const int bt = u / p.n_hb, hb = u - bt * p.n_hb;
+            for (; !c.done(); ++it) {
+                const int u = c.u, j = c.j();
                 const int b = p.unit_meta[u].w;
-                const int qrow = bt * p.n_h + hb * 128 + 64 * static_cast<int>(rank);
-                if (!wait_bar(bar(BAR_Q_EMPTY), (uc & 1) ^ 1, abort_flag, p.status)) break;
-                if (rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_Q_FULL), 2 * kQBytes);
-                const uint32_t qf = leader_bar(BAR_Q_FULL);
-                for (int c = 0; c < 8; ++c)
-                    ptx::tma_load_2d_pair(sbase + kOffQ + c * kChunk, &p.tm_qa, 64 * c, qrow, qf, pol_q);
-                ptx::tma_load_2d_pair(sbase + kOffQ + 8 * kChunk, &p.tm_qr, 0, qrow, qf, pol_q);
-                bool ok = true;
-                for (int j = t0; j < t1; ++j, ++it) {
-                    const int st = it % kStages;
-                    if (!wait_bar(bar(BAR_KV_EMPTY + st), ((it / kStages) & 1) ^ 1, abort_flag, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    if (rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), 2 * kStageBytes);
-                    int blk = p.block_table[static_cast<size_t>(b) * p.max_blocks + j];
-                    if (blk < 0 || blk >= p.num_blocks) {
-                        raise_status(p.status, MLA_STATUS_BAD_BLOCK);
-                        blk = 0;
-                    }
-                    const uint32_t kf = leader_bar(BAR_KV_FULL + st);
-                    const uint32_t stage = sbase + kOffStage + st * kStageBytes;
-                    const int row_s = blk * kBlk + 32 * static_cast<int>(rank);
-                    for (int c = 0; c < 9; ++c)
-                        ptx::tma_load_2d_pair(stage + c * 4096, &p.tm_pool_s, 64 * c, row_s, kf, pol_stream);
-                    for (int i = 0; i < 4; ++i)
-                        ptx::tma_load_2d_pair(stage + kSRegion + i * kChunk, &p.tm_pool_v,
-                                              64 * owned_chunk(rank, i), blk * kBlk, kf, pol_stream);
+                if (c.seg_first()) {
+                    const int bt = u / p.n_hb, hb = u - bt * p.n_hb;
+                    const int qrow = bt * p.n_h + hb * 128 + 64 * static_cast<int>(rank);
+                    if (!wait_bar(bar(BAR_Q_EMPTY), (uc & 1) ^ 1, abort_flag, p.status)) break;
+                    if (rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_Q_FULL), 2 * kQBytes);
+                    const uint32_t qf = leader_bar(BAR_Q_FULL);
+                    for (int cc = 0; cc < 8; ++cc)
+                        ptx::tma_load_2d_pair(sbase + kOffQ + cc * kQChunk, &p.tm_qa, 64 * cc, qrow, qf, pol_q);
+                    ptx::tma_load_2d_pair(sbase + kOffQ + 8 * kQChunk, &p.tm_qr, 0, qrow, qf, pol_q);
                 }
-                if (!ok) break;
-                ++uc;
-                g = ubeg + t1;
+                const int st = it % kStages;
+                if (!wait_bar(bar(BAR_KV_EMPTY + st), ((it / kStages) & 1) ^ 1, abort_flag, p.status)) break;
+                if (rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), 2 * kStageBytes);
+                int blk = p.block_table[static_cast<size_t>(b) * p.max_blocks + (j >> 1)];
+                if (blk < 0 || blk >= p.num_blocks) {
+                    raise_status(p.status, MLA_STATUS_BAD_BLOCK);
+                    blk = 0;
+                }
+                const uint32_t kf = leader_bar(BAR_KV_FULL + st);
+                const uint32_t stage = sbase + kOffStage + st * kStageBytes;
+                const int row0 = blk * kPage + kTile * (j & 1);
+                const int row_s = row0 + 16 * static_cast<int>(rank);
+                for (int cc = 0; cc < 9; ++cc)
+                    ptx::tma_load_2d_pair(stage + cc * kSChunk, &p.tm_pool_s, 64 * cc, row_s, kf, pol_stream);
+                for (int i = 0; i < 4; ++i)
+                    ptx::tma_load_2d_pair(stage + kSRegion + i * kVSlot, &p.tm_pool_v,
+                                          64 * owned_chunk(rank, i), row0, kf, pol_stream);
+                if (c.seg_last()) ++uc;
+                c.next();
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (rank == 0 && lane == 0 && g0 < g1) {
-            int it = 0, uc = 0;
+            TileCursor cs, cp;
+            cs.init(p.prefix, p.U, g0, g1);
+            cp.init(p.prefix, p.U, g0, g1);
+            int its = 0, itp = 0, ucs = 0;
             bool ok = true;
-            auto pv = [&](int i, bool first) -> bool {
-                if (!wait_bar(bar(BAR_P_FULL), i & 1, abort_flag, p.status)) return false;
-                ptx::tc_fence_after();
-                const uint32_t vbase = sbase + kOffStage + (i % kStages) * kStageBytes + kSRegion;
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t a = ptx::smem_desc_sw128(sbase + kOffP + 32 * kk, 16, 1024);
-                        const uint64_t bdesc = ptx::smem_desc_sw128(vbase + 16384 * h + 2048 * kk, kChunk, 1024);
-                        ptx::mma_pair_ss(tmem_base + kTmemO + 128 * h, a, bdesc, kIdescPV,
-                                         (first && kk == 0) ? 0u : 1u);
+            uint64_t last = ptx::global_timer_ns();
+            while (!cp.done()) {
+                bool progress = false;
+                // S(its) = Q K^T once its keys have landed and its accumulator is free
+                if (!cs.done()) {
+                    const int st = its % kStages, sb = its % kSBuf;
+                    bool ready = !cs.seg_first() || ptx::mbar_test_wait(bar(BAR_Q_FULL), ucs & 1);
+                    ready = ready && ptx::mbar_test_wait(bar(BAR_KV_FULL + st), (its / kStages) & 1);
+                    ready = ready && ptx::mbar_test_wait(bar(BAR_S_FREE + sb), ((its / kSBuf) & 1) ^ 1);
+                    if (ready) {
+                        ptx::tc_fence_after();
+                        const uint32_t sreg = sbase + kOffStage + st * kStageBytes;
+                        const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffQ, 16, 1024);
+                        const uint64_t b0 = ptx::smem_desc_sw128(sreg, 16, 1024);
+#pragma unroll 4
+                        for (int kk = 0; kk < 36; ++kk) {
+                            const int c = kk >> 2, k4 = kk & 3;
+                            // descriptor start addresses advance in 16-byte units
+                            const uint64_t a = a0 + static_cast<uint64_t>((c * kQChunk + 32 * k4) >> 4);
+                            const uint64_t bd = b0 + static_cast<uint64_t>((c * kSChunk + 32 * k4) >> 4);
+                            ptx::mma_pair_ss(tmem_base + kTmemS + 16 * sb, a, bd, kIdescS, kk > 0 ? 1u : 0u);
+                        }
+                        ptx::mma_commit_pair(bar(BAR_S_FULL + sb), 0x3);
+                        if (cs.seg_last()) {
+                            ptx::mma_commit_pair(bar(BAR_Q_EMPTY), 0x3);
+                            ++ucs;
+                        }
+                        ++its;
+                        cs.next();
+                        progress = true;
                     }
-                ptx::mma_commit_pair(bar(BAR_KV_EMPTY + i % kStages), 0x3);
-                ptx::mma_commit_pair(bar(BAR_P_FREE), 0x3);
-                return true;
-            };
-            int u = find_unit(p.prefix, p.U, g0);
-            for (int g = g0; g < g1 && ok; ++u) {
-                const int ubeg = p.prefix[u], uend = p.prefix[u + 1];
-                if (uend <= g) continue;
-                const int t0 = g - ubeg, t1 = min(g1, uend) - ubeg;
-                const int n = t1 - t0;
-                if (!wait_bar(bar(BAR_Q_FULL), uc & 1, abort_flag, p.status)) { ok = false; break; }
-                for (int jj = 0; jj < n; ++jj, ++it) {
-                    const int st = it % kStages, sb = it & 1;
-                    if (!wait_bar(bar(BAR_KV_FULL + st), (it / kStages) & 1, abort_flag, p.status) ||
-                        !wait_bar(bar(BAR_S_FREE + sb), ((it >> 1) & 1) ^ 1, abort_flag, p.status)) {
+                }
+                // O (+)= P V once the softmax has written P(itp)
+                if (itp < its) {
+                    const int pb = itp % kPBuf;
+                    if (ptx::mbar_test_wait(bar(BAR_P_FULL + pb), (itp / kPBuf) & 1)) {
+                        ptx::tc_fence_after();
+                        const bool first = cp.seg_first();
+                        const uint32_t vbase = sbase + kOffStage + (itp % kStages) * kStageBytes + kSRegion;
+                        const uint64_t a0 = ptx::smem_desc_sw64(sbase + kOffP + pb * kPBytes, 16, 512);
+                        const uint64_t b0 = ptx::smem_desc_sw128(vbase, kVSlot, 1024);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int kk = 0; kk < 2; ++kk) {
+                                const uint64_t a = a0 + static_cast<uint64_t>((32 * kk) >> 4);
+                                const uint64_t bd = b0 + static_cast<uint64_t>((8192 * h + 2048 * kk) >> 4);
+                                ptx::mma_pair_ss(tmem_base + kTmemO + 128 * h, a, bd, kIdescPV,
+                                                 (first && kk == 0) ? 0u : 1u);
+                            }
+                        ptx::mma_commit_pair(bar(BAR_KV_EMPTY + itp % kStages), 0x3);
+                        ptx::mma_commit_pair(bar(BAR_P_FREE + pb), 0x3);
+                        ++itp;
+                        cp.next();
+                        progress = true;
+                    }
+                }
+                if (progress) {
+                    last = ptx::global_timer_ns();
+                } else {
+                    if (*abort_flag) { ok = false; break; }
+                    if (ptx::global_timer_ns() - last > kTimeoutNs) {
+                        *abort_flag = 1;
+                        raise_status(p.status, MLA_STATUS_TIMEOUT);
                         ok = false;
                         break;
                     }
-                    ptx::tc_fence_after();
-                    const uint32_t sreg = sbase + kOffStage + st * kStageBytes;
-#pragma unroll 4
-                    for (int kk = 0; kk < 36; ++kk) {
-                        const int c = kk >> 2, k4 = kk & 3;
-                        const uint64_t a = ptx::smem_desc_sw128(sbase + kOffQ + c * kChunk + 32 * k4, 16, 1024);
-                        const uint64_t bdesc = ptx::smem_desc_sw128(sreg + c * 4096 + 32 * k4, 16, 1024);
-                        ptx::mma_pair_ss(tmem_base + kTmemS + 32 * sb, a, bdesc, kIdescS, kk > 0 ? 1u : 0u);
-                    }
-                    ptx::mma_commit_pair(bar(BAR_S_FULL + sb), 0x3);
-                    if (jj == n - 1) ptx::mma_commit_pair(bar(BAR_Q_EMPTY), 0x3);
-                    if (jj > 0 && !pv(it - 1, jj == 1)) { ok = false; break; }
                 }
-                if (!ok) break;
-                if (!pv(it - 1, n == 1)) { ok = false; break; }
-                ++uc;
-                g = ubeg + t1;
             }
             if (!ok) {
                 // let every issued MMA finish before the teardown frees anything
@@ -309,38 +364,37 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
         float* xmax = reinterpret_cast<float*>(smem + kOffXmax);
         float* xsum = reinterpret_cast<float*>(smem + kOffXsum);
-        unsigned char* P = smem + kOffP;
-        const uint32_t s_free_l[2] = {leader_bar(BAR_S_FREE), leader_bar(BAR_S_FREE + 1)};
-        const uint32_t p_full_l = leader_bar(BAR_P_FULL);
+        TileCursor c;
+        c.init(p.prefix, p.U, g0, g1);
         int it = 0;
         bool ok = true;
-        int u = g0 < g1 ? find_unit(p.prefix, p.U, g0) : 0;
-        for (int g = g0; g < g1 && ok; ++u) {
-            const int ubeg = p.prefix[u], uend = p.prefix[u + 1];
-            if (uend <= g) continue;
-            const int t0 = g - ubeg, t1 = min(g1, uend) - ubeg;
+        while (!c.done() && ok) {
+            const int u = c.u;
             const int4 meta = p.unit_meta[u];
             const int kv_len = meta.x;
+            const int jfirst = c.j();
             float m_used = -INFINITY, l_part = 0.f;
-            for (int j = t0; j < t1; ++j, ++it) {
-                const int sb = it & 1;
-                ok = wait_bar(bar(BAR_S_FULL + sb), (it >> 1) & 1, abort_flag, p.status);
+            bool seg_last = false;
+            do {
+                const int j = c.j();
+                const int sb = it % kSBuf;
+                ok = wait_bar(bar(BAR_S_FULL + sb), (it / kSBuf) & 1, abort_flag, p.status);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 ptx::tc_fence_after();
-                uint32_t r[32];
-                ptx::tmem_ld32(t_lane + kTmemS + 32 * sb, r);
+                uint32_t r[16];
+                ptx::tmem_ld16(t_lane + kTmemS + 16 * sb, r);
                 ptx::tmem_wait_ld();
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive_cluster(s_free_l[sb]);
+                if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_S_FREE + sb));
 
-                const int key0 = j * kBlk + (hi ? 32 : 0);
-                float s[32];
+                const int key0 = j * kTile + (hi ? 16 : 0);
+                float s[16];
                 float mx = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    s[c] = (key0 + c < kv_len) ? __uint_as_float(r[c]) * p.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, s[c]);
+                for (int q = 0; q < 16; ++q) {
+                    s[q] = (key0 + q < kv_len) ? __uint_as_float(r[q]) * p.scale_log2 : -INFINITY;
+                    mx = fmaxf(mx, s[q]);
                 }
                 float* xb = xmax + (it & 1) * 128;
                 xb[l] = mx;
@@ -350,22 +404,26 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 bool resc = false;
                 if (mx > m_used + kRescaleThreshold) {
                     new_m = mx;
-                    resc = j > t0;
+                    resc = j > jfirst;
                 }
                 const float alpha = ex2(m_used - new_m);
                 m_used = new_m;
-                uint32_t pk[16];
+                uint32_t pk[8];
                 float ps = 0.f;
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const float p0 = ex2(s[c] - m_used), p1 = ex2(s[c + 1] - m_used);
+                for (int q = 0; q < 16; q += 2) {
+                    const float p0 = ex2(s[q] - m_used), p1 = ex2(s[q + 1] - m_used);
                     ps += p0 + p1;
-                    pk[c >> 1] = pack_bf16x2(p0, p1);
+                    pk[q >> 1] = pack_bf16x2(p0, p1);
                 }
                 l_part = l_part * alpha + ps;
 
-                // P.V of the previous block must be done: P buffer free, O stable
-                ok = wait_bar(bar(BAR_P_FREE), (it & 1) ^ 1, abort_flag, p.status);
+                const int pb = it % kPBuf;
+                // P buffer pb is free once P.V(it - 2) has completed
+                ok = wait_bar(bar(BAR_P_FREE + pb), ((it / kPBuf) & 1) ^ 1, abort_flag, p.status);
+                // a rescale of O needs P.V(it - 1) complete as well
+                if (ok && resc)
+                    ok = wait_bar(bar(BAR_P_FREE + (pb ^ 1)), ((it - 1) / kPBuf) & 1, abort_flag, p.status);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 ptx::tc_fence_after();
                 if (resc) {
@@ -375,40 +433,46 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                         ptx::tmem_ld32(t_lane + kTmemO + 32 * q, o);
                         ptx::tmem_wait_ld();
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                         ptx::tmem_st32(t_lane + kTmemO + 32 * q, o);
                     }
                     ptx::tmem_wait_st();
                 }
-                // rows past the end of the keys hold stale data: zero this CTA's
-                // P.V operand rows for them (P is zero there already)
-                const int valid = kv_len - j * kBlk;
-                if (valid < kBlk) {
-                    const int bad = kBlk - valid;
+                // keys past the end hold stale rows: zero this CTA's P.V operand
+                // rows for them (their P is zero already)
+                const int valid = kv_len - j * kTile;
+                if (valid < kTile) {
+                    const int bad = kTile - valid;
                     uint4* vreg = reinterpret_cast<uint4*>(smem + kOffStage + (it % kStages) * kStageBytes + kSRegion);
                     for (int e = l; e < 4 * bad * 8; e += 128) {
                         const int slot = e / (bad * 8), rem = e - slot * bad * 8;
-                        const int row = valid + rem / 8, ch = rem & 7;
-                        vreg[(slot * kChunk + row * 128) / 16 + ch] = make_uint4(0, 0, 0, 0);
+                        const int row = valid + (rem >> 3), ch = rem & 7;
+                        vreg[(slot * kVSlot + row * 128) / 16 + ch] = make_uint4(0, 0, 0, 0);
                     }
                 }
-                // P row m, keys (hi ? 32 : 0) + [0, 32) in 128-byte-swizzled K-major layout
+                // P row m, keys (hi ? 16 : 0) + [0, 16): K-major, 64-byte rows,
+                // 64-byte swizzle (16-byte chunk index XOR (row >> 1) & 3)
+                unsigned char* Pb = smem + kOffP + pb * kPBytes;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int chunk = (hi ? 4 : 0) + q4;
-                    const int phys = chunk ^ (m & 7);
-                    *reinterpret_cast<uint4*>(P + m * 128 + phys * 16) =
-                        make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    const int chunk = (hi ? 2 : 0) + q2;
+                    const int phys = chunk ^ ((m >> 1) & 3);
+                    *reinterpret_cast<uint4*>(Pb + m * 64 + phys * 16) =
+                        make_uint4(pk[4 * q2], pk[4 * q2 + 1], pk[4 * q2 + 2], pk[4 * q2 + 3]);
                 }
                 ptx::fence_proxy_async_smem();
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive_cluster(p_full_l);
-            }
+                if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_P_FULL + pb));
+                seg_last = c.seg_last();
+                ++it;
+                c.next();
+            } while (!seg_last);
             if (!ok) break;
 
-            // ---- epilogue of this unit segment
-            ok = wait_bar(bar(BAR_P_FREE), (it & 1) ^ 1, abort_flag, p.status);
+            // ---- epilogue of this unit segment: wait for P.V of its last tile
+            const int e = it - 1;
+            ok = wait_bar(bar(BAR_P_FREE + e % kPBuf), (e / kPBuf) & 1, abort_flag, p.status);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             ptx::tc_fence_after();
             xsum[l] = l_part;
@@ -455,7 +519,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 else p.part_lse[slot * 128 + head_in_unit] = lse;
             }
             ptx::tc_fence_before();
-            g = ubeg + t1;
         }
     }
 
@@ -494,9 +557,9 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, 
             b = bt / T_q;
             const int t = bt - b * T_q;
             const int L = seq_lens[b];
-            if (L >= T_q && L <= max_blocks * kBlk) {
+            if (L >= T_q && L <= max_blocks * kPage) {
                 kv = L - T_q + t + 1;
-                tiles = (kv + kBlk - 1) / kBlk;
+                tiles = (kv + kTile - 1) / kTile;
             } else if (t == 0 && (u % n_hb) == 0) {
                 raise_status(status, MLA_STATUS_BAD_SEQ_LEN);
             }
@@ -653,8 +716,8 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int /*max_split
     Sm100Params k;
     const uint64_t pool_rows = static_cast<uint64_t>(P.num_blocks) * P.block_size;
     const uint64_t q_rows = static_cast<uint64_t>(P.n_tok) * P.n_h;
-    if (!make_map_2d(&k.tm_pool_s, P.pool, kRow, pool_rows, kRow * 2, 64, 32) ||
-        !make_map_2d(&k.tm_pool_v, P.pool, kRow, pool_rows, kRow * 2, 64, 64) ||
+    if (!make_map_2d(&k.tm_pool_s, P.pool, kRow, pool_rows, kRow * 2, 64, 16) ||
+        !make_map_2d(&k.tm_pool_v, P.pool, kRow, pool_rows, kRow * 2, 64, 32) ||
         !make_map_2d(&k.tm_qa, P.q_abs, kDc, q_rows, kDc * 2, 64, 64) ||
         !make_map_2d(&k.tm_qr, P.q_r, kDr, q_rows, kDr * 2, 64, 64))
         return cudaErrorInvalidValue;
