@@ -48,61 +48,56 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kClusters = 74;                     // 148 SMs / 2
 constexpr int kDc = 512, kDr = 64, kRow = 576;    // row = c^KV || k^R
-constexpr int kPage = 64;                         // cache rows per page
-constexpr int kTile = 32;                         // keys per tile (half a page)
-constexpr int kStages = 4;                        // TMA ring depth
-constexpr int kSBuf = 4;                          // S accumulators in tensor memory
-constexpr int kPBuf = 2;                          // P operand buffers
+constexpr int kPage = 64;                         // cache rows per page (TMA box height)
+constexpr int kTilePages = 4;                     // a tile = 4 pages = 256 keys (MMA N)
+constexpr int kRing = 7;                          // 16 KB entries in the load ring
 
-constexpr uint32_t kQChunk = 8192;                // 64 heads x 128 B
-constexpr uint32_t kQBytes = 9 * kQChunk;         // 64 heads x 576 columns
-constexpr uint32_t kSChunk = 2048;                // 16 keys x 128 B
-constexpr uint32_t kSRegion = 9 * kSChunk;        // this CTA's 16 keys x 576
-constexpr uint32_t kVSlot = 4096;                 // 32 keys x 128 B
-constexpr uint32_t kVRegion = 4 * kVSlot;         // 32 keys x 256 latent columns
-constexpr uint32_t kStageBytes = kSRegion + kVRegion;
-constexpr uint32_t kPBytes = 4096;                // 64 heads x 32 keys bf16 (64-byte swizzle)
+constexpr uint32_t kBox = 8192;                   // one page x 64 columns (128 B rows)
+constexpr uint32_t kEntry = 2 * kBox;             // ring entry: 2 boxes
+constexpr uint32_t kQBytes = 9 * kBox;            // 64 heads x 576 columns
+constexpr uint32_t kPBytes = 4 * kBox;            // 64 heads x 256 keys (4 blocks of 64 keys)
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffStage = kOffQ + kQBytes;
-constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;
-constexpr uint32_t kOffXmax = kOffP + kPBuf * kPBytes;   // 2 x 128 floats
-constexpr uint32_t kOffXsum = kOffXmax + 1024;           // 128 floats
+constexpr uint32_t kOffRing = kOffQ + kQBytes;
+constexpr uint32_t kOffP = kOffRing + kRing * kEntry;
+constexpr uint32_t kOffXmax = kOffP + kPBytes;    // 2 x 128 floats
+constexpr uint32_t kOffXsum = kOffXmax + 1024;    // 128 floats
 constexpr uint32_t kOffBar = kOffXsum + 512;
-constexpr uint32_t kOffMisc = kOffBar + 8 * 32;          // tmem base, abort flag
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;    // + alignment slack
+constexpr uint32_t kOffMisc = kOffBar + 8 * 32;   // tmem base, abort flag
+constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 enum {
     BAR_Q_FULL = 0,
     BAR_Q_EMPTY = 1,
-    BAR_KV_FULL = 2,                     // + stage
-    BAR_KV_EMPTY = BAR_KV_FULL + kStages,
-    BAR_S_FULL = BAR_KV_EMPTY + kStages, // + S buffer
-    BAR_S_FREE = BAR_S_FULL + kSBuf,
-    BAR_P_FULL = BAR_S_FREE + kSBuf,     // + P buffer
-    BAR_P_FREE = BAR_P_FULL + kPBuf,
-    BAR_DRAIN = BAR_P_FREE + kPBuf,
+    BAR_RING_FULL = 2,                       // + slot (leader: both CTAs' bytes)
+    BAR_RING_EMPTY = BAR_RING_FULL + kRing,  // + slot (each CTA, MMA commit)
+    BAR_S_FULL = BAR_RING_EMPTY + kRing,     // + S buffer
+    BAR_S_FREE = BAR_S_FULL + 2,             // + S buffer (leader, 8 warps)
+    BAR_P_FULL = BAR_S_FREE + 2,             // leader, 8 warps
+    BAR_P_FREE = BAR_P_FULL + 1,             // each CTA, MMA commit
+    BAR_TAIL_READY = BAR_P_FREE + 1,         // each CTA, MMA thread arrives remotely
+    BAR_TAIL_DONE = BAR_TAIL_READY + 1,      // leader, 8 warps
+    BAR_DRAIN = BAR_TAIL_DONE + 1,
     NUM_BARS = BAR_DRAIN + 1
 };
 static_assert(NUM_BARS <= 32, "barrier area");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;                    // 2 x 128 columns (paired layout)
-constexpr uint32_t kTmemS = 256;                  // kSBuf x 16 columns
+constexpr uint32_t kTmemS = 256;                  // 2 x 128 columns
 
-constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, kTile, 0, 0);
+constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 256, 0, 0);
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 256, 0, 1);
 
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
 
 struct Sm100Params {
-    CUtensorMap tm_pool_s;    // pool as [rows][576], box 64 cols x 16 rows
-    CUtensorMap tm_pool_v;    // pool as [rows][576], box 64 cols x 32 rows
+    CUtensorMap tm_pool;      // pool as [rows][576], box 64 cols x 64 rows
     CUtensorMap tm_qa;        // q_abs as [n_tok*n_h][512], box 64 x 64
     CUtensorMap tm_qr;        // q_r   as [n_tok*n_h][64],  box 64 x 64
     const int32_t* block_table;
-    const int32_t* prefix;    // (U + 1) exclusive prefix of tiles per unit
+    const int32_t* prefix;    // (U + 1) exclusive prefix of pages per unit
     const int4* unit_meta;    // (U) {kv_len, first cluster, parts, batch index}
     uint16_t* out_latent;
     float* out_lse;
@@ -130,7 +125,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, volatil
     }
 }
 
-// Unit whose tile range contains global tile g (prefix is non-decreasing).
+// Unit whose page range contains global page g (prefix is non-decreasing).
 __device__ __forceinline__ int find_unit(const int32_t* prefix, int U, int g) {
     int lo = 0, hi = U - 1;
     while (lo < hi) {
@@ -140,8 +135,18 @@ __device__ __forceinline__ int find_unit(const int32_t* prefix, int U, int g) {
     return lo;
 }
 
-// Walks a cluster's tiles [g0, g1) unit by unit.
-struct TileCursor {
+// One tile of a cluster's work: up to 4 consecutive pages of one unit.
+struct Tile {
+    int u;          // unit
+    int page0;      // first page, within the unit
+    int np;         // pages in this tile (1..4)
+    bool first;     // first tile of a unit segment (new Q, O starts from zero)
+    bool last;      // last tile of a unit segment (epilogue follows)
+    bool unit_end;  // the unit's last page is in this tile
+};
+
+// Walks a cluster's pages [g0, g1) as tiles.
+struct TileWalker {
     const int32_t* prefix;
     int g, g0, g1, u;
     __device__ void init(const int32_t* pf, int U, int g0_, int g1_) {
@@ -150,25 +155,29 @@ struct TileCursor {
         g0 = g0_;
         g1 = g1_;
         u = g0_ < g1_ ? find_unit(pf, U, g0_) : 0;
-        skip();
-    }
-    __device__ void skip() {
         while (g < g1 && prefix[u + 1] <= g) ++u;
     }
     __device__ bool done() const { return g >= g1; }
-    __device__ int j() const { return g - prefix[u]; }   // tile index within the unit
-    __device__ bool seg_first() const { return g == g0 || g == prefix[u]; }
-    __device__ bool seg_last() const { return g + 1 == g1 || g + 1 == prefix[u + 1]; }
-    __device__ void next() {
-        ++g;
-        skip();
+    __device__ Tile next() {
+        Tile t;
+        const int ubeg = prefix[u], uend = prefix[u + 1];
+        t.u = u;
+        t.page0 = g - ubeg;
+        t.first = (g == g0) || (g == ubeg);
+        const int seg_end = min(g1, uend);   // tiles start at the segment start
+        t.np = min(kTilePages, seg_end - g);
+        t.last = g + t.np == seg_end;
+        t.unit_end = g + t.np == uend;
+        g += t.np;
+        while (g < g1 && prefix[u + 1] <= g) ++u;
+        return t;
     }
 };
 
-// latent column chunk (64 wide) that V-region slot i of CTA `rank` holds:
-// P.V instruction h takes N columns [0,128) from CTA 0 and [128,256) from CTA 1
-__device__ __forceinline__ int owned_chunk(uint32_t rank, int i) {
-    return 4 * (i >> 1) + 2 * static_cast<int>(rank) + (i & 1);
+// latent column chunk (64 wide) that a CTA contributes to P.V instruction h:
+// N columns [0,128) come from CTA 0, [128,256) from CTA 1
+__device__ __forceinline__ int owned_chunk(uint32_t rank, int h, int i) {
+    return 4 * h + 2 * static_cast<int>(rank) + i;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -189,25 +198,24 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     if (threadIdx.x == 0) {
         ptx::mbar_init(bar(BAR_Q_FULL), 1);
         ptx::mbar_init(bar(BAR_Q_EMPTY), 1);
-        for (int s = 0; s < kStages; ++s) {
-            ptx::mbar_init(bar(BAR_KV_FULL + s), 1);
-            ptx::mbar_init(bar(BAR_KV_EMPTY + s), 1);
+        for (int s = 0; s < kRing; ++s) {
+            ptx::mbar_init(bar(BAR_RING_FULL + s), 1);
+            ptx::mbar_init(bar(BAR_RING_EMPTY + s), 1);
         }
-        for (int b = 0; b < kSBuf; ++b) {
+        for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(bar(BAR_S_FULL + b), 1);
             ptx::mbar_init(bar(BAR_S_FREE + b), 8);   // 4 softmax warps x 2 CTAs
         }
-        for (int b = 0; b < kPBuf; ++b) {
-            ptx::mbar_init(bar(BAR_P_FULL + b), 8);
-            ptx::mbar_init(bar(BAR_P_FREE + b), 1);
-        }
+        ptx::mbar_init(bar(BAR_P_FULL), 8);
+        ptx::mbar_init(bar(BAR_P_FREE), 1);
+        ptx::mbar_init(bar(BAR_TAIL_READY), 1);
+        ptx::mbar_init(bar(BAR_TAIL_DONE), 8);
         ptx::mbar_init(bar(BAR_DRAIN), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        ptx::prefetch_tmap(&p.tm_pool_s);
-        ptx::prefetch_tmap(&p.tm_pool_v);
+        ptx::prefetch_tmap(&p.tm_pool);
         ptx::prefetch_tmap(&p.tm_qa);
         ptx::prefetch_tmap(&p.tm_qr);
     }
@@ -221,131 +229,176 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    // this cluster's contiguous range of global tiles; with fewer tiles than
+    // this cluster's contiguous range of global pages; with fewer pages than
     // clusters only the first `total` clusters work, so no range is empty
     const int total = p.prefix[p.U];
     const int Ce = min(p.C, total);
     const int g0 = cluster < Ce ? static_cast<int>((static_cast<long long>(cluster) * total) / Ce) : 0;
     const int g1 = cluster < Ce ? static_cast<int>((static_cast<long long>(cluster + 1) * total) / Ce) : 0;
 
+    // Ring order, shared by the producer and the MMA issuer:
+    //   S(0), S(1), V(0), S(2), V(1), ..., S(n-1), V(n-2), V(n-1)
+    // S(i): 9 entries (column chunk c of this CTA's pages 2r, 2r+1 of tile i);
+    // V(i): 2 entries per page (latent chunks owned for P.V instruction h).
+
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0 && g0 < g1) {
-            const uint64_t pol_stream = ptx::l2_policy_evict_first();
-            const uint64_t pol_q = ptx::l2_policy_evict_last();
-            TileCursor c;
-            c.init(p.prefix, p.U, g0, g1);
-            int it = 0, uc = 0;
-            for (; !c.done(); ++it) {
-                const int u = c.u, j = c.j();
-                const int b = p.unit_meta[u].w;
-                if (c.seg_first()) {
-                    const int bt = u / p.n_hb, hb = u - bt * p.n_hb;
-                    const int qrow = bt * p.n_h + hb * 128 + 64 * static_cast<int>(rank);
-                    if (!wait_bar(bar(BAR_Q_EMPTY), (uc & 1) ^ 1, abort_flag, p.status)) break;
-                    if (rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_Q_FULL), 2 * kQBytes);
-                    const uint32_t qf = leader_bar(BAR_Q_FULL);
-                    for (int cc = 0; cc < 8; ++cc)
-                        ptx::tma_load_2d_pair(sbase + kOffQ + cc * kQChunk, &p.tm_qa, 64 * cc, qrow, qf, pol_q);
-                    ptx::tma_load_2d_pair(sbase + kOffQ + 8 * kQChunk, &p.tm_qr, 0, qrow, qf, pol_q);
-                }
-                const int st = it % kStages;
-                if (!wait_bar(bar(BAR_KV_EMPTY + st), ((it / kStages) & 1) ^ 1, abort_flag, p.status)) break;
-                if (rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), 2 * kStageBytes);
-                int blk = p.block_table[static_cast<size_t>(b) * p.max_blocks + (j >> 1)];
-                if (blk < 0 || blk >= p.num_blocks) {
-                    raise_status(p.status, MLA_STATUS_BAD_BLOCK);
-                    blk = 0;
-                }
-                const uint32_t kf = leader_bar(BAR_KV_FULL + st);
-                const uint32_t stage = sbase + kOffStage + st * kStageBytes;
-                const int row0 = blk * kPage + kTile * (j & 1);
-                const int row_s = row0 + 16 * static_cast<int>(rank);
-                for (int cc = 0; cc < 9; ++cc)
-                    ptx::tma_load_2d_pair(stage + cc * kSChunk, &p.tm_pool_s, 64 * cc, row_s, kf, pol_stream);
-                for (int i = 0; i < 4; ++i)
-                    ptx::tma_load_2d_pair(stage + kSRegion + i * kVSlot, &p.tm_pool_v,
-                                          64 * owned_chunk(rank, i), row0, kf, pol_stream);
-                if (c.seg_last()) ++uc;
-                c.next();
+        const uint64_t pol_stream = ptx::l2_policy_evict_first();
+        const uint64_t pol_q = ptx::l2_policy_evict_last();
+        TileWalker w;
+        w.init(p.prefix, p.U, g0, g1);
+        Tile cur{}, prev{};
+        bool have_prev = false;
+        int e = 0, uc = 0;
+        bool ok = g0 < g1;
+        // lane 0 waits/arms barriers; lanes 0..1 each issue one box of an entry
+        auto issue_entry = [&](int rows0, int rows1, bool has0, bool has1, int col0, int col1, uint32_t tx_total) -> bool {
+            const int slot = e % kRing;
+            bool good = true;
+            if (lane == 0) good = wait_bar(bar(BAR_RING_EMPTY + slot), ((e / kRing) & 1) ^ 1, abort_flag, p.status);
+            good = __shfl_sync(0xffffffffu, good, 0);
+            if (!good) return false;
+            if (lane == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_RING_FULL + slot), tx_total);
+            __syncwarp();
+            const uint32_t dst = sbase + kOffRing + slot * kEntry;
+            const uint32_t full = leader_bar(BAR_RING_FULL + slot);
+            if (lane == 0 && has0) ptx::tma_load_2d_pair(dst, &p.tm_pool, col0, rows0, full, pol_stream);
+            if (lane == 1 && has1) ptx::tma_load_2d_pair(dst + kBox, &p.tm_pool, col1, rows1, full, pol_stream);
+            ++e;
+            return true;
+        };
+        auto page_row = [&](const Tile& t, int pg) -> int {
+            // cache row of page pg (0..3) of tile t; invalid entries are flagged and clamped
+            const int b = p.unit_meta[t.u].w;
+            int blk = p.block_table[static_cast<size_t>(b) * p.max_blocks + t.page0 + pg];
+            if (blk < 0 || blk >= p.num_blocks) {
+                raise_status(p.status, MLA_STATUS_BAD_BLOCK);
+                blk = 0;
             }
+            return blk * kPage;
+        };
+        while (ok && (!w.done() || have_prev)) {
+            const bool has_cur = !w.done();
+            if (has_cur) {
+                cur = w.next();
+                if (cur.first) {
+                    // new unit segment: load Q (this CTA's 64 heads)
+                    bool good = true;
+                    if (lane == 0) good = wait_bar(bar(BAR_Q_EMPTY), (uc & 1) ^ 1, abort_flag, p.status);
+                    good = __shfl_sync(0xffffffffu, good, 0);
+                    if (!good) { ok = false; break; }
+                    const int bt = cur.u / p.n_hb, hb = cur.u - bt * p.n_hb;
+                    const int qrow = bt * p.n_h + hb * 128 + 64 * static_cast<int>(rank);
+                    if (lane == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_Q_FULL), 2 * kQBytes);
+                    __syncwarp();
+                    const uint32_t qf = leader_bar(BAR_Q_FULL);
+                    if (lane < 8) ptx::tma_load_2d_pair(sbase + kOffQ + lane * kBox, &p.tm_qa, 64 * lane, qrow, qf, pol_q);
+                    if (lane == 8) ptx::tma_load_2d_pair(sbase + kOffQ + 8 * kBox, &p.tm_qr, 0, qrow, qf, pol_q);
+                    ++uc;
+                }
+                // S(cur): 9 column chunks of pages 2r, 2r+1
+                const bool h0 = 2 * static_cast<int>(rank) < cur.np, h1 = 2 * static_cast<int>(rank) + 1 < cur.np;
+                const int r0 = h0 ? page_row(cur, 2 * rank) : 0;
+                const int r1 = h1 ? page_row(cur, 2 * rank + 1) : 0;
+                const uint32_t tx = static_cast<uint32_t>(cur.np) * kBox;   // both CTAs together
+                for (int c = 0; c < 9 && ok; ++c)
+                    ok = issue_entry(r0, r1, h0, h1, 64 * c, 64 * c, tx);
+                if (!ok) break;
+            }
+            if (have_prev) {
+                // V(prev): per page, per P.V instruction h: 2 latent chunks, all 64 keys
+                for (int pg = 0; pg < prev.np && ok; ++pg) {
+                    const int r = page_row(prev, pg);
+                    for (int h = 0; h < 2 && ok; ++h)
+                        ok = issue_entry(r, r, true, true, 64 * owned_chunk(rank, h, 0), 64 * owned_chunk(rank, h, 1),
+                                         2 * kEntry);
+                }
+                if (!ok) break;
+            }
+            have_prev = has_cur;
+            prev = cur;
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (rank == 0 && lane == 0 && g0 < g1) {
-            TileCursor cs, cp;
-            cs.init(p.prefix, p.U, g0, g1);
-            cp.init(p.prefix, p.U, g0, g1);
-            int its = 0, itp = 0, ucs = 0;
+            TileWalker w;
+            w.init(p.prefix, p.U, g0, g1);
+            Tile cur{}, prev{};
+            bool have_prev = false;
+            int e = 0, i = 0, uc = 0, tails = 0;
             bool ok = true;
-            uint64_t last = ptx::global_timer_ns();
-            while (!cp.done()) {
-                bool progress = false;
-                // S(its) = Q K^T once its keys have landed and its accumulator is free
-                if (!cs.done()) {
-                    const int st = its % kStages, sb = its % kSBuf;
-                    bool ready = !cs.seg_first() || ptx::mbar_test_wait(bar(BAR_Q_FULL), ucs & 1);
-                    ready = ready && ptx::mbar_test_wait(bar(BAR_KV_FULL + st), (its / kStages) & 1);
-                    ready = ready && ptx::mbar_test_wait(bar(BAR_S_FREE + sb), ((its / kSBuf) & 1) ^ 1);
-                    if (ready) {
+            auto wait_entry = [&](int idx) -> bool {
+                return wait_bar(bar(BAR_RING_FULL + idx % kRing), (idx / kRing) & 1, abort_flag, p.status);
+            };
+            while (ok && (!w.done() || have_prev)) {
+                const bool has_cur = !w.done();
+                if (has_cur) {
+                    cur = w.next();
+                    const int sb = i & 1;
+                    if (cur.first && !(ok = wait_bar(bar(BAR_Q_FULL), uc & 1, abort_flag, p.status))) break;
+                    if (!(ok = wait_bar(bar(BAR_S_FREE + sb), ((i >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+                    const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffQ, 16, 1024);
+                    for (int c = 0; c < 9; ++c) {
+                        if (!(ok = wait_entry(e))) break;
                         ptx::tc_fence_after();
-                        const uint32_t sreg = sbase + kOffStage + st * kStageBytes;
-                        const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffQ, 16, 1024);
-                        const uint64_t b0 = ptx::smem_desc_sw128(sreg, 16, 1024);
-#pragma unroll 4
-                        for (int kk = 0; kk < 36; ++kk) {
-                            const int c = kk >> 2, k4 = kk & 3;
-                            // descriptor start addresses advance in 16-byte units
-                            const uint64_t a = a0 + static_cast<uint64_t>((c * kQChunk + 32 * k4) >> 4);
-                            const uint64_t bd = b0 + static_cast<uint64_t>((c * kSChunk + 32 * k4) >> 4);
-                            ptx::mma_pair_ss(tmem_base + kTmemS + 16 * sb, a, bd, kIdescS, kk > 0 ? 1u : 0u);
+                        const uint64_t b0 = ptx::smem_desc_sw128(sbase + kOffRing + (e % kRing) * kEntry, 16, 1024);
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const uint64_t a = a0 + static_cast<uint64_t>((c * kBox + 32 * k4) >> 4);
+                            const uint64_t bd = b0 + static_cast<uint64_t>((32 * k4) >> 4);
+                            ptx::mma_pair_ss(tmem_base + kTmemS + 128 * sb, a, bd, kIdescS, (c | k4) ? 1u : 0u);
                         }
-                        ptx::mma_commit_pair(bar(BAR_S_FULL + sb), 0x3);
-                        if (cs.seg_last()) {
-                            ptx::mma_commit_pair(bar(BAR_Q_EMPTY), 0x3);
-                            ++ucs;
-                        }
-                        ++its;
-                        cs.next();
-                        progress = true;
+                        ptx::mma_commit_pair(bar(BAR_RING_EMPTY + e % kRing), 0x3);
+                        ++e;
                     }
+                    if (!ok) break;
+                    ptx::mma_commit_pair(bar(BAR_S_FULL + sb), 0x3);
+                    if (cur.last) {
+                        ptx::mma_commit_pair(bar(BAR_Q_EMPTY), 0x3);
+                        ++uc;
+                    }
+                    ++i;
                 }
-                // O (+)= P V once the softmax has written P(itp)
-                if (itp < its) {
-                    const int pb = itp % kPBuf;
-                    if (ptx::mbar_test_wait(bar(BAR_P_FULL + pb), (itp / kPBuf) & 1)) {
-                        ptx::tc_fence_after();
-                        const bool first = cp.seg_first();
-                        const uint32_t vbase = sbase + kOffStage + (itp % kStages) * kStageBytes + kSRegion;
-                        const uint64_t a0 = ptx::smem_desc_sw64(sbase + kOffP + pb * kPBytes, 16, 512);
-                        const uint64_t b0 = ptx::smem_desc_sw128(vbase, kVSlot, 1024);
+                if (have_prev) {
+                    // P.V of the previous tile, once its P is written
+                    const int ip = i - 1 - (has_cur ? 1 : 0);
+                    if (!(ok = wait_bar(bar(BAR_P_FULL), ip & 1, abort_flag, p.status))) break;
+                    const int4 meta = p.unit_meta[prev.u];
+                    const bool tail = prev.unit_end && (meta.x % kPage) != 0;
+                    ptx::tc_fence_after();
+                    const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffP, 16, 1024);
+                    for (int pg = 0; pg < prev.np && ok; ++pg) {
+                        if (tail && pg == prev.np - 1) {
+                            // the unit's last page holds rows past the end: once its two
+                            // V entries have landed, the softmax warps of both CTAs zero
+                            // those rows (entries are consumed in ring order, so the
+                            // earlier pages' slots are already free for these loads)
+                            if (!(ok = wait_entry(e) && wait_entry(e + 1))) break;
+                            ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 0));
+                            ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 1));
+                            if (!(ok = wait_bar(bar(BAR_TAIL_DONE), tails & 1, abort_flag, p.status))) break;
+                            ++tails;
+                        }
+                        for (int h = 0; h < 2; ++h) {
+                            if (!(ok = wait_entry(e))) break;
+                            ptx::tc_fence_after();
+                            const uint64_t b0 = ptx::smem_desc_sw128(sbase + kOffRing + (e % kRing) * kEntry, kBox, 1024);
 #pragma unroll
-                        for (int h = 0; h < 2; ++h)
-#pragma unroll
-                            for (int kk = 0; kk < 2; ++kk) {
-                                const uint64_t a = a0 + static_cast<uint64_t>((32 * kk) >> 4);
-                                const uint64_t bd = b0 + static_cast<uint64_t>((8192 * h + 2048 * kk) >> 4);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint64_t a = a0 + static_cast<uint64_t>((pg * kBox + 32 * kk) >> 4);
+                                const uint64_t bd = b0 + static_cast<uint64_t>((2048 * kk) >> 4);
                                 ptx::mma_pair_ss(tmem_base + kTmemO + 128 * h, a, bd, kIdescPV,
-                                                 (first && kk == 0) ? 0u : 1u);
+                                                 (prev.first && pg == 0 && kk == 0) ? 0u : 1u);
                             }
-                        ptx::mma_commit_pair(bar(BAR_KV_EMPTY + itp % kStages), 0x3);
-                        ptx::mma_commit_pair(bar(BAR_P_FREE + pb), 0x3);
-                        ++itp;
-                        cp.next();
-                        progress = true;
+                            ptx::mma_commit_pair(bar(BAR_RING_EMPTY + e % kRing), 0x3);
+                            ++e;
+                        }
                     }
+                    if (!ok) break;
+                    ptx::mma_commit_pair(bar(BAR_P_FREE), 0x3);
                 }
-                if (progress) {
-                    last = ptx::global_timer_ns();
-                } else {
-                    if (*abort_flag) { ok = false; break; }
-                    if (ptx::global_timer_ns() - last > kTimeoutNs) {
-                        *abort_flag = 1;
-                        raise_status(p.status, MLA_STATUS_TIMEOUT);
-                        ok = false;
-                        break;
-                    }
-                }
+                have_prev = has_cur;
+                prev = cur;
             }
             if (!ok) {
                 // let every issued MMA finish before the teardown frees anything
@@ -364,161 +417,176 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
         float* xmax = reinterpret_cast<float*>(smem + kOffXmax);
         float* xsum = reinterpret_cast<float*>(smem + kOffXsum);
-        TileCursor c;
-        c.init(p.prefix, p.U, g0, g1);
-        int it = 0;
+        TileWalker w;
+        w.init(p.prefix, p.U, g0, g1);
+        int i = 0, tails = 0;
+        int v_before = 0;      // V ring entries of tiles before i
         bool ok = true;
-        while (!c.done() && ok) {
-            const int u = c.u;
-            const int4 meta = p.unit_meta[u];
-            const int kv_len = meta.x;
-            const int jfirst = c.j();
-            float m_used = -INFINITY, l_part = 0.f;
-            bool seg_last = false;
-            do {
-                const int j = c.j();
-                const int sb = it % kSBuf;
-                ok = wait_bar(bar(BAR_S_FULL + sb), (it / kSBuf) & 1, abort_flag, p.status);
-                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                ptx::tc_fence_after();
-                uint32_t r[16];
-                ptx::tmem_ld16(t_lane + kTmemS + 16 * sb, r);
-                ptx::tmem_wait_ld();
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_S_FREE + sb));
-
-                const int key0 = j * kTile + (hi ? 16 : 0);
-                float s[16];
-                float mx = -INFINITY;
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    s[q] = (key0 + q < kv_len) ? __uint_as_float(r[q]) * p.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, s[q]);
-                }
-                float* xb = xmax + (it & 1) * 128;
-                xb[l] = mx;
-                ptx::named_bar_sync(1, 128);
-                mx = fmaxf(mx, xb[l ^ 64]);
-                float new_m = m_used;
-                bool resc = false;
-                if (mx > m_used + kRescaleThreshold) {
-                    new_m = mx;
-                    resc = j > jfirst;
-                }
-                const float alpha = ex2(m_used - new_m);
-                m_used = new_m;
-                uint32_t pk[8];
-                float ps = 0.f;
-#pragma unroll
-                for (int q = 0; q < 16; q += 2) {
-                    const float p0 = ex2(s[q] - m_used), p1 = ex2(s[q + 1] - m_used);
-                    ps += p0 + p1;
-                    pk[q >> 1] = pack_bf16x2(p0, p1);
-                }
-                l_part = l_part * alpha + ps;
-
-                const int pb = it % kPBuf;
-                // P buffer pb is free once P.V(it - 2) has completed
-                ok = wait_bar(bar(BAR_P_FREE + pb), ((it / kPBuf) & 1) ^ 1, abort_flag, p.status);
-                // a rescale of O needs P.V(it - 1) complete as well
-                if (ok && resc)
-                    ok = wait_bar(bar(BAR_P_FREE + (pb ^ 1)), ((it - 1) / kPBuf) & 1, abort_flag, p.status);
-                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                ptx::tc_fence_after();
-                if (resc) {
-#pragma unroll 1
-                    for (int q = 0; q < 8; ++q) {
-                        uint32_t o[32];
-                        ptx::tmem_ld32(t_lane + kTmemO + 32 * q, o);
-                        ptx::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        ptx::tmem_st32(t_lane + kTmemO + 32 * q, o);
-                    }
-                    ptx::tmem_wait_st();
-                }
-                // keys past the end hold stale rows: zero this CTA's P.V operand
-                // rows for them (their P is zero already)
-                const int valid = kv_len - j * kTile;
-                if (valid < kTile) {
-                    const int bad = kTile - valid;
-                    uint4* vreg = reinterpret_cast<uint4*>(smem + kOffStage + (it % kStages) * kStageBytes + kSRegion);
-                    for (int e = l; e < 4 * bad * 8; e += 128) {
-                        const int slot = e / (bad * 8), rem = e - slot * bad * 8;
-                        const int row = valid + (rem >> 3), ch = rem & 7;
-                        vreg[(slot * kVSlot + row * 128) / 16 + ch] = make_uint4(0, 0, 0, 0);
-                    }
-                }
-                // P row m, keys (hi ? 16 : 0) + [0, 16): K-major, 64-byte rows,
-                // 64-byte swizzle (16-byte chunk index XOR (row >> 1) & 3)
-                unsigned char* Pb = smem + kOffP + pb * kPBytes;
-#pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2) {
-                    const int chunk = (hi ? 2 : 0) + q2;
-                    const int phys = chunk ^ ((m >> 1) & 3);
-                    *reinterpret_cast<uint4*>(Pb + m * 64 + phys * 16) =
-                        make_uint4(pk[4 * q2], pk[4 * q2 + 1], pk[4 * q2 + 2], pk[4 * q2 + 3]);
-                }
-                ptx::fence_proxy_async_smem();
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_P_FULL + pb));
-                seg_last = c.seg_last();
-                ++it;
-                c.next();
-            } while (!seg_last);
-            if (!ok) break;
-
-            // ---- epilogue of this unit segment: wait for P.V of its last tile
-            const int e = it - 1;
-            ok = wait_bar(bar(BAR_P_FREE + e % kPBuf), (e / kPBuf) & 1, abort_flag, p.status);
+        float m_used = -INFINITY, l_part = 0.f;
+        while (ok && !w.done()) {
+            const Tile t = w.next();
+            const bool is_cluster_last = w.done();
+            const int4 meta = p.unit_meta[t.u];
+            // keys of this tile that belong to this segment
+            const int key_end = min(meta.x, kPage * (t.page0 + t.np));
+            if (t.first) {
+                m_used = -INFINITY;
+                l_part = 0.f;
+            }
+            const int sb = i & 1;
+            ok = wait_bar(bar(BAR_S_FULL + sb), (i >> 1) & 1, abort_flag, p.status);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             ptx::tc_fence_after();
-            xsum[l] = l_part;
+            uint32_t r[128];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t (&rq)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q]);
+                ptx::tmem_ld32(t_lane + kTmemS + 128 * sb + 32 * q, rq);
+            }
+            ptx::tmem_wait_ld();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_S_FREE + sb));
+
+            const int key0 = kPage * t.page0 + (hi ? 128 : 0);
+            float mx = -INFINITY;
+#pragma unroll
+            for (int q = 0; q < 128; ++q) {
+                const float v = (key0 + q < key_end) ? __uint_as_float(r[q]) * p.scale_log2 : -INFINITY;
+                r[q] = __float_as_uint(v);
+                mx = fmaxf(mx, v);
+            }
+            float* xb = xmax + (i & 1) * 128;
+            xb[l] = mx;
             ptx::named_bar_sync(1, 128);
-            const float lsum = l_part + xsum[l ^ 64];
-            const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-            const float lse = lsum > 0.f ? (m_used + __log2f(lsum)) * kLn2 : -INFINITY;
-            const int bt = u / p.n_hb, hb = u - bt * p.n_hb;
-            const int head_in_unit = 64 * static_cast<int>(rank) + m;
-            const bool whole = meta.z == 1;
-            const size_t grow = static_cast<size_t>(bt) * p.n_h + hb * 128 + head_in_unit;
-            const size_t slot = static_cast<size_t>(cluster) + u;
+            mx = fmaxf(mx, xb[l ^ 64]);
+            float new_m = m_used;
+            bool resc = false;
+            if (mx > m_used + kRescaleThreshold) {
+                new_m = mx;
+                resc = !t.first;
+            }
+            const float alpha = ex2(m_used - new_m);
+            m_used = new_m;
+            float ps = 0.f;
+#pragma unroll
+            for (int q = 0; q < 128; q += 2) {
+                const float p0 = ex2(__uint_as_float(r[q]) - m_used), p1 = ex2(__uint_as_float(r[q + 1]) - m_used);
+                ps += p0 + p1;
+                r[q >> 1] = pack_bf16x2(p0, p1);
+            }
+            l_part = l_part * alpha + ps;
+
+            // P.V of the previous tile must be complete: P buffer free, O stable
+            ok = wait_bar(bar(BAR_P_FREE), (i & 1) ^ 1, abort_flag, p.status);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            ptx::tc_fence_after();
+            if (resc) {
 #pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-                const int col0 = 256 * h + (hi ? 128 : 0);
-#pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 8; ++q) {
                     uint32_t o[32];
-                    ptx::tmem_ld32(t_lane + kTmemO + 128 * h + 32 * q, o);
+                    ptx::tmem_ld32(t_lane + kTmemO + 32 * q, o);
                     ptx::tmem_wait_ld();
-                    const int col = col0 + 32 * q;
-                    if (whole) {
-                        uint4* dst = reinterpret_cast<uint4*>(p.out_latent + grow * kDc + col);
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            uint4 w;
-                            w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-                            w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-                            w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-                            w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-                            dst[v] = w;
-                        }
-                    } else {
-                        float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * 128 + head_in_unit) * kDc + col);
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                    ptx::tmem_st32(t_lane + kTmemO + 32 * q, o);
+                }
+                ptx::tmem_wait_st();
+            }
+            // P row m, keys (hi ? 128 : 0) + [0, 128): blocks of 64 keys, K-major,
+            // 128-byte rows, 128-byte swizzle (chunk index XOR row & 7)
 #pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
-                                                 __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
-                    }
+            for (int blk = 0; blk < 2; ++blk) {
+                unsigned char* Pb = smem + kOffP + ((hi ? 2 : 0) + blk) * kBox + m * 128;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const int phys = ch ^ (m & 7);
+                    const int w0 = 32 * blk + 4 * ch;
+                    *reinterpret_cast<uint4*>(Pb + phys * 16) = make_uint4(r[w0], r[w0 + 1], r[w0 + 2], r[w0 + 3]);
                 }
             }
-            if (!hi) {
-                if (whole) p.out_lse[grow] = lse;
-                else p.part_lse[slot * 128 + head_in_unit] = lse;
-            }
+            ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_P_FULL));
+
+            // ring position of this tile's V entries (same order as the producer)
+            const int v_start = 9 * (i + (is_cluster_last ? 1 : 2)) + v_before;
+            v_before += 2 * t.np;
+            if (t.unit_end && (meta.x % kPage) != 0) {
+                // zero rows past the end in this CTA's two V entries of the last page
+                ok = wait_bar(bar(BAR_TAIL_READY), tails & 1, abort_flag, p.status);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                ++tails;
+                const int valid = meta.x - kPage * (t.page0 + t.np - 1);
+                const int bad = kPage - valid;
+                const int et = v_start + 2 * (t.np - 1);
+                for (int x = l; x < 2 * 2 * bad * 8; x += 128) {
+                    const int ent = x / (2 * bad * 8);
+                    const int rem = x - ent * 2 * bad * 8;
+                    const int half = rem / (bad * 8);
+                    const int rem2 = rem - half * bad * 8;
+                    const int row = valid + (rem2 >> 3), ch = rem2 & 7;
+                    uint4* dst = reinterpret_cast<uint4*>(smem + kOffRing + ((et + ent) % kRing) * kEntry +
+                                                          half * kBox + row * 128) + ch;
+                    *dst = make_uint4(0, 0, 0, 0);
+                }
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_TAIL_DONE));
+            }
+
+            if (t.last) {
+                // ---- epilogue of this unit segment: wait for P.V of this tile
+                ok = wait_bar(bar(BAR_P_FREE), i & 1, abort_flag, p.status);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                ptx::tc_fence_after();
+                xsum[l] = l_part;
+                ptx::named_bar_sync(1, 128);
+                const float lsum = l_part + xsum[l ^ 64];
+                const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+                const float lse = lsum > 0.f ? (m_used + __log2f(lsum)) * kLn2 : -INFINITY;
+                const int bt = t.u / p.n_hb, hb = t.u - bt * p.n_hb;
+                const int head_in_unit = 64 * static_cast<int>(rank) + m;
+                const bool whole = meta.z == 1;
+                const size_t grow = static_cast<size_t>(bt) * p.n_h + hb * 128 + head_in_unit;
+                const size_t slot = static_cast<size_t>(cluster) + t.u;
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    const int col0 = 256 * h + (hi ? 128 : 0);
+#pragma unroll 1
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t o[32];
+                        ptx::tmem_ld32(t_lane + kTmemO + 128 * h + 32 * q, o);
+                        ptx::tmem_wait_ld();
+                        const int col = col0 + 32 * q;
+                        if (whole) {
+                            uint4* dst = reinterpret_cast<uint4*>(p.out_latent + grow * kDc + col);
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                uint4 wv;
+                                wv.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+                                wv.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+                                wv.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+                                wv.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+                                dst[v] = wv;
+                            }
+                        } else {
+                            float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * 128 + head_in_unit) * kDc + col);
+#pragma unroll
+                            for (int v = 0; v < 8; ++v)
+                                dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                                     __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
+                        }
+                    }
+                }
+                if (!hi) {
+                    if (whole) p.out_lse[grow] = lse;
+                    else p.part_lse[slot * 128 + head_in_unit] = lse;
+                }
+                ptx::tc_fence_before();
+            }
+            ++i;
         }
     }
 
@@ -559,7 +627,7 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, 
             const int L = seq_lens[b];
             if (L >= T_q && L <= max_blocks * kPage) {
                 kv = L - T_q + t + 1;
-                tiles = (kv + kTile - 1) / kTile;
+                tiles = (kv + kPage - 1) / kPage;
             } else if (t == 0 && (u % n_hb) == 0) {
                 raise_status(status, MLA_STATUS_BAD_SEQ_LEN);
             }
@@ -716,8 +784,7 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int /*max_split
     Sm100Params k;
     const uint64_t pool_rows = static_cast<uint64_t>(P.num_blocks) * P.block_size;
     const uint64_t q_rows = static_cast<uint64_t>(P.n_tok) * P.n_h;
-    if (!make_map_2d(&k.tm_pool_s, P.pool, kRow, pool_rows, kRow * 2, 64, 16) ||
-        !make_map_2d(&k.tm_pool_v, P.pool, kRow, pool_rows, kRow * 2, 64, 32) ||
+    if (!make_map_2d(&k.tm_pool, P.pool, kRow, pool_rows, kRow * 2, 64, 64) ||
         !make_map_2d(&k.tm_qa, P.q_abs, kDc, q_rows, kDc * 2, 64, 64) ||
         !make_map_2d(&k.tm_qr, P.q_r, kDr, q_rows, kDr * 2, 64, 64))
         return cudaErrorInvalidValue;

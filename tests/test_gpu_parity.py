@@ -109,6 +109,17 @@ def test_append_and_gather_bit_exact(M, name):
     assert np.array_equal(q_r, want_q)
 
 
+def test_many_units_whole_and_split(M):
+    # 300 units of 9 pages each (last page partial): most units fit inside one
+    # cluster's page range (written directly), the rest straddle two clusters
+    spec = CaseSpec(**V2, seq_lens=np.full(300, 517, np.int32), seed=12, permute_blocks=True)
+    dc = _dc(spec)
+    dc.step()
+    torch.cuda.synchronize()
+    assert dc.decode_status() == 0
+    check_sequences(dc, [0, 1, 150, 298, 299])
+
+
 @pytest.mark.parametrize("splits", [1, 2, 3, 7])
 @pytest.mark.parametrize("impl", [0, 1])
 def test_split_count_invariance(M, splits, impl):
