@@ -96,6 +96,7 @@ struct Sm100Params {
     CUtensorMap tm_pool;      // pool as [rows][576], box 64 cols x 64 rows
     CUtensorMap tm_qa;        // q_abs as [n_tok*n_h][512], box 64 x 64
     CUtensorMap tm_qr;        // q_r   as [n_tok*n_h][64],  box 64 x 64
+    const uint16_t* pool;     // for L2 prefetches of whole pages
     const int32_t* block_table;
     const int32_t* prefix;    // (U + 1) exclusive prefix of pages per unit
     const int4* unit_meta;    // (U) {kv_len, first cluster, parts, batch index}
@@ -243,30 +244,24 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
+        // Each step's entries (S(cur): 9, V(prev): 2 per page) are listed first,
+        // then issued up to kBatch at a time: lane 0 waits for their slots and
+        // arms the barriers, lanes 2j and 2j+1 issue the two boxes of entry j.
+        constexpr int kBatch = 4;
+        constexpr int kMaxStep = 9 + 2 * kTilePages;
         const uint64_t pol_stream = ptx::l2_policy_evict_first();
         const uint64_t pol_q = ptx::l2_policy_evict_last();
-        TileWalker w;
+        TileWalker w, wp;
         w.init(p.prefix, p.U, g0, g1);
+        wp.init(p.prefix, p.U, g0, g1);
+        if (!wp.done()) wp.next();   // the look-ahead walker runs one tile ahead
         Tile cur{}, prev{};
         bool have_prev = false;
         int e = 0, uc = 0;
         bool ok = g0 < g1;
-        // lane 0 waits/arms barriers; lanes 0..1 each issue one box of an entry
-        auto issue_entry = [&](int rows0, int rows1, bool has0, bool has1, int col0, int col1, uint32_t tx_total) -> bool {
-            const int slot = e % kRing;
-            bool good = true;
-            if (lane == 0) good = wait_bar(bar(BAR_RING_EMPTY + slot), ((e / kRing) & 1) ^ 1, abort_flag, p.status);
-            good = __shfl_sync(0xffffffffu, good, 0);
-            if (!good) return false;
-            if (lane == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_RING_FULL + slot), tx_total);
-            __syncwarp();
-            const uint32_t dst = sbase + kOffRing + slot * kEntry;
-            const uint32_t full = leader_bar(BAR_RING_FULL + slot);
-            if (lane == 0 && has0) ptx::tma_load_2d_pair(dst, &p.tm_pool, col0, rows0, full, pol_stream);
-            if (lane == 1 && has1) ptx::tma_load_2d_pair(dst + kBox, &p.tm_pool, col1, rows1, full, pol_stream);
-            ++e;
-            return true;
-        };
+        int ent_row[kMaxStep][2], ent_col[kMaxStep][2];
+        unsigned ent_has[kMaxStep];   // bit0/1: box present; bit2: V entry (last use of the lines)
+        uint32_t ent_tx[kMaxStep];
         auto page_row = [&](const Tile& t, int pg) -> int {
             // cache row of page pg (0..3) of tile t; invalid entries are flagged and clamped
             const int b = p.unit_meta[t.u].w;
@@ -279,10 +274,21 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         };
         while (ok && (!w.done() || have_prev)) {
             const bool has_cur = !w.done();
+            int n = 0;
             if (has_cur) {
                 cur = w.next();
+                if (!wp.done()) {
+                    // Pull the next tile's pages (this CTA's S pages 2r, 2r+1; the
+                    // peer's P.V operand reads hit the same lines) into L2 a step
+                    // ahead, so the ring's loads below are L2 hits with short latency.
+                    const Tile nt = wp.next();
+                    const int pg = 2 * static_cast<int>(rank) + (lane & 1);
+                    if (lane < 2 && pg < nt.np)
+                        ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(page_row(nt, pg)) * kRow,
+                                              kPage * kRow * 2);
+                }
                 if (cur.first) {
-                    // new unit segment: load Q (this CTA's 64 heads)
+                    // new unit segment: load Q (this CTA's 64 heads) from 9 lanes
                     bool good = true;
                     if (lane == 0) good = wait_bar(bar(BAR_Q_EMPTY), (uc & 1) ^ 1, abort_flag, p.status);
                     good = __shfl_sync(0xffffffffu, good, 0);
@@ -300,20 +306,53 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 const bool h0 = 2 * static_cast<int>(rank) < cur.np, h1 = 2 * static_cast<int>(rank) + 1 < cur.np;
                 const int r0 = h0 ? page_row(cur, 2 * rank) : 0;
                 const int r1 = h1 ? page_row(cur, 2 * rank + 1) : 0;
-                const uint32_t tx = static_cast<uint32_t>(cur.np) * kBox;   // both CTAs together
-                for (int c = 0; c < 9 && ok; ++c)
-                    ok = issue_entry(r0, r1, h0, h1, 64 * c, 64 * c, tx);
-                if (!ok) break;
+                for (int c = 0; c < 9; ++c, ++n) {
+                    ent_row[n][0] = r0;
+                    ent_row[n][1] = r1;
+                    ent_col[n][0] = ent_col[n][1] = 64 * c;
+                    ent_has[n] = (h0 ? 1u : 0u) | (h1 ? 2u : 0u);
+                    ent_tx[n] = static_cast<uint32_t>(cur.np) * kBox;    // both CTAs together
+                }
             }
             if (have_prev) {
                 // V(prev): per page, per P.V instruction h: 2 latent chunks, all 64 keys
-                for (int pg = 0; pg < prev.np && ok; ++pg) {
+                for (int pg = 0; pg < prev.np; ++pg) {
                     const int r = page_row(prev, pg);
-                    for (int h = 0; h < 2 && ok; ++h)
-                        ok = issue_entry(r, r, true, true, 64 * owned_chunk(rank, h, 0), 64 * owned_chunk(rank, h, 1),
-                                         2 * kEntry);
+                    for (int h = 0; h < 2; ++h, ++n) {
+                        ent_row[n][0] = ent_row[n][1] = r;
+                        ent_col[n][0] = 64 * owned_chunk(rank, h, 0);
+                        ent_col[n][1] = 64 * owned_chunk(rank, h, 1);
+                        ent_has[n] = 7u;
+                        ent_tx[n] = 2 * kEntry;
+                    }
                 }
-                if (!ok) break;
+            }
+            for (int k = 0; k < n && ok; k += kBatch) {
+                const int nb = min(kBatch, n - k);
+                bool good = true;
+                if (lane == 0) {
+                    for (int j = 0; j < nb && good; ++j) {
+                        const int ee = e + j;
+                        good = wait_bar(bar(BAR_RING_EMPTY + ee % kRing), ((ee / kRing) & 1) ^ 1, abort_flag, p.status);
+                        if (good && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_RING_FULL + ee % kRing), ent_tx[k + j]);
+                    }
+                }
+                good = __shfl_sync(0xffffffffu, good, 0);
+                if (!good) { ok = false; break; }
+                const int j = lane >> 1, half = lane & 1;
+                if (j < nb && (ent_has[k + j] >> half & 1u)) {
+                    const int ee = e + j;
+                    const uint32_t dst = sbase + kOffRing + (ee % kRing) * kEntry + half * kBox;
+                    // S loads keep normal L2 priority: the peer CTA reads the same lines
+                    // again for its P.V operand one step later; V loads are their last use
+                    if (ent_has[k + j] & 4u)
+                        ptx::tma_load_2d_pair(dst, &p.tm_pool, ent_col[k + j][half], ent_row[k + j][half],
+                                              leader_bar(BAR_RING_FULL + ee % kRing), pol_stream);
+                    else
+                        ptx::tma_load_2d_pair_normal(dst, &p.tm_pool, ent_col[k + j][half], ent_row[k + j][half],
+                                                     leader_bar(BAR_RING_FULL + ee % kRing));
+                }
+                e += nb;
             }
             have_prev = has_cur;
             prev = cur;
@@ -788,6 +827,7 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int /*max_split
         !make_map_2d(&k.tm_qa, P.q_abs, kDc, q_rows, kDc * 2, 64, 64) ||
         !make_map_2d(&k.tm_qr, P.q_r, kDr, q_rows, kDr * 2, 64, 64))
         return cudaErrorInvalidValue;
+    k.pool = P.pool;
     k.block_table = P.block_table;
     k.prefix = reinterpret_cast<const int32_t*>(base + w.prefix);
     k.unit_meta = reinterpret_cast<const int4*>(base + w.meta);

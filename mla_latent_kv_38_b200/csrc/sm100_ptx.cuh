@@ -101,6 +101,23 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap,
         : "memory");
 }
 
+// Same without an L2 eviction hint (normal priority).
+__device__ __forceinline__ void tma_load_2d_pair_normal(uint32_t dst, const void* tmap, int x, int y,
+                                                        uint32_t mbar_cluster_addr) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(mbar_cluster_addr), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Bring `bytes` (multiple of 16) of contiguous global memory into L2; no
+// completion tracking, no shared memory involved.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* gaddr, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gaddr)), "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
