@@ -45,20 +45,22 @@
 namespace mla {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;   // 8 warps: S loads, S MMAs, 4 x softmax, P.V MMAs, V loads
 constexpr int kClusters = 74;                     // 148 SMs / 2
 constexpr int kDc = 512, kDr = 64, kRow = 576;    // row = c^KV || k^R
 constexpr int kPage = 64;                         // cache rows per page (TMA box height)
 constexpr int kTilePages = 4;                     // a tile = 4 pages = 256 keys (MMA N)
-constexpr int kRing = 7;                          // 16 KB entries in the load ring
+constexpr int kSRing = 4;                         // 16 KB entries, S operand stream
+constexpr int kVRing = 3;                         // 16 KB entries, P.V operand stream
 
 constexpr uint32_t kBox = 8192;                   // one page x 64 columns (128 B rows)
 constexpr uint32_t kEntry = 2 * kBox;             // ring entry: 2 boxes
 constexpr uint32_t kQBytes = 9 * kBox;            // 64 heads x 576 columns
 constexpr uint32_t kPBytes = 4 * kBox;            // 64 heads x 256 keys (4 blocks of 64 keys)
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffRing = kOffQ + kQBytes;
-constexpr uint32_t kOffP = kOffRing + kRing * kEntry;
+constexpr uint32_t kOffSRing = kOffQ + kQBytes;
+constexpr uint32_t kOffVRing = kOffSRing + kSRing * kEntry;
+constexpr uint32_t kOffP = kOffVRing + kVRing * kEntry;
 constexpr uint32_t kOffXmax = kOffP + kPBytes;    // 2 x 128 floats
 constexpr uint32_t kOffXsum = kOffXmax + 1024;    // 128 floats
 constexpr uint32_t kOffBar = kOffXsum + 512;
@@ -69,16 +71,19 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 enum {
     BAR_Q_FULL = 0,
     BAR_Q_EMPTY = 1,
-    BAR_RING_FULL = 2,                       // + slot (leader: both CTAs' bytes)
-    BAR_RING_EMPTY = BAR_RING_FULL + kRing,  // + slot (each CTA, MMA commit)
-    BAR_S_FULL = BAR_RING_EMPTY + kRing,     // + S buffer
+    BAR_SR_FULL = 2,                         // + slot (leader: both CTAs' bytes)
+    BAR_SR_EMPTY = BAR_SR_FULL + kSRing,     // + slot (each CTA, MMA commit)
+    BAR_VR_FULL = BAR_SR_EMPTY + kSRing,
+    BAR_VR_EMPTY = BAR_VR_FULL + kVRing,
+    BAR_S_FULL = BAR_VR_EMPTY + kVRing,      // + S buffer
     BAR_S_FREE = BAR_S_FULL + 2,             // + S buffer (leader, 8 warps)
     BAR_P_FULL = BAR_S_FREE + 2,             // leader, 8 warps
     BAR_P_FREE = BAR_P_FULL + 1,             // each CTA, MMA commit
     BAR_TAIL_READY = BAR_P_FREE + 1,         // each CTA, MMA thread arrives remotely
     BAR_TAIL_DONE = BAR_TAIL_READY + 1,      // leader, 8 warps
-    BAR_DRAIN = BAR_TAIL_DONE + 1,
-    NUM_BARS = BAR_DRAIN + 1
+    BAR_DRAIN = BAR_TAIL_DONE + 1,           // S issuer's own drain on abort
+    BAR_DRAIN_PV = BAR_DRAIN + 1,            // P.V issuer's
+    NUM_BARS = BAR_DRAIN_PV + 1
 };
 static_assert(NUM_BARS <= 32, "barrier area");
 
@@ -199,9 +204,13 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     if (threadIdx.x == 0) {
         ptx::mbar_init(bar(BAR_Q_FULL), 1);
         ptx::mbar_init(bar(BAR_Q_EMPTY), 1);
-        for (int s = 0; s < kRing; ++s) {
-            ptx::mbar_init(bar(BAR_RING_FULL + s), 1);
-            ptx::mbar_init(bar(BAR_RING_EMPTY + s), 1);
+        for (int s = 0; s < kSRing; ++s) {
+            ptx::mbar_init(bar(BAR_SR_FULL + s), 1);
+            ptx::mbar_init(bar(BAR_SR_EMPTY + s), 1);
+        }
+        for (int s = 0; s < kVRing; ++s) {
+            ptx::mbar_init(bar(BAR_VR_FULL + s), 1);
+            ptx::mbar_init(bar(BAR_VR_EMPTY + s), 1);
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(bar(BAR_S_FULL + b), 1);
@@ -212,6 +221,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         ptx::mbar_init(bar(BAR_TAIL_READY), 1);
         ptx::mbar_init(bar(BAR_TAIL_DONE), 8);
         ptx::mbar_init(bar(BAR_DRAIN), 1);
+        ptx::mbar_init(bar(BAR_DRAIN_PV), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -237,213 +247,196 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     const int g0 = cluster < Ce ? static_cast<int>((static_cast<long long>(cluster) * total) / Ce) : 0;
     const int g1 = cluster < Ce ? static_cast<int>((static_cast<long long>(cluster + 1) * total) / Ce) : 0;
 
-    // Ring order, shared by the producer and the MMA issuer:
-    //   S(0), S(1), V(0), S(2), V(1), ..., S(n-1), V(n-2), V(n-1)
-    // S(i): 9 entries (column chunk c of this CTA's pages 2r, 2r+1 of tile i);
-    // V(i): 2 entries per page (latent chunks owned for P.V instruction h).
+    // Two load streams, each consumed in order by one MMA issuer:
+    //   S ring: S(i) = 9 entries (column chunk c of this CTA's pages 2r, 2r+1)
+    //   V ring: V(i) = 2 entries per page (latent chunks owned for P.V h = 0, 1)
+    auto page_row = [&](const Tile& t, int pg) -> int {
+        // cache row of page pg (0..3) of tile t; invalid entries are flagged and clamped
+        const int b = p.unit_meta[t.u].w;
+        int blk = p.block_table[static_cast<size_t>(b) * p.max_blocks + t.page0 + pg];
+        if (blk < 0 || blk >= p.num_blocks) {
+            raise_status(p.status, MLA_STATUS_BAD_BLOCK);
+            blk = 0;
+        }
+        return blk * kPage;
+    };
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        // Each step's entries (S(cur): 9, V(prev): 2 per page) are listed first,
-        // then issued up to kBatch at a time: lane 0 waits for their slots and
-        // arms the barriers, lanes 2j and 2j+1 issue the two boxes of entry j.
-        constexpr int kBatch = 4;
-        constexpr int kMaxStep = 9 + 2 * kTilePages;
-        const uint64_t pol_stream = ptx::l2_policy_evict_first();
+        // ------------------------------------------------------------ S stream (and Q)
+        // Lanes 0 and 1 each wait for the entry's slot and issue one box (lane 0
+        // of the leader CTA arms the full barrier with both CTAs' bytes).
         const uint64_t pol_q = ptx::l2_policy_evict_last();
         TileWalker w, wp;
         w.init(p.prefix, p.U, g0, g1);
         wp.init(p.prefix, p.U, g0, g1);
         if (!wp.done()) wp.next();   // the look-ahead walker runs one tile ahead
-        Tile cur{}, prev{};
-        bool have_prev = false;
         int e = 0, uc = 0;
         bool ok = g0 < g1;
-        int ent_row[kMaxStep][2], ent_col[kMaxStep][2];
-        unsigned ent_has[kMaxStep];   // bit0/1: box present; bit2: V entry (last use of the lines)
-        uint32_t ent_tx[kMaxStep];
-        auto page_row = [&](const Tile& t, int pg) -> int {
-            // cache row of page pg (0..3) of tile t; invalid entries are flagged and clamped
-            const int b = p.unit_meta[t.u].w;
-            int blk = p.block_table[static_cast<size_t>(b) * p.max_blocks + t.page0 + pg];
-            if (blk < 0 || blk >= p.num_blocks) {
-                raise_status(p.status, MLA_STATUS_BAD_BLOCK);
-                blk = 0;
+        while (ok && !w.done()) {
+            const Tile cur = w.next();
+            if (!wp.done()) {
+                // Pull the next tile's pages (this CTA's S pages 2r, 2r+1; the peer's
+                // P.V operand reads hit the same lines) into L2 a tile ahead.
+                const Tile nt = wp.next();
+                const int pg = 2 * static_cast<int>(rank) + (lane & 1);
+                if (lane < 2 && pg < nt.np)
+                    ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(page_row(nt, pg)) * kRow, kPage * kRow * 2);
             }
-            return blk * kPage;
-        };
-        while (ok && (!w.done() || have_prev)) {
-            const bool has_cur = !w.done();
-            int n = 0;
-            if (has_cur) {
-                cur = w.next();
-                if (!wp.done()) {
-                    // Pull the next tile's pages (this CTA's S pages 2r, 2r+1; the
-                    // peer's P.V operand reads hit the same lines) into L2 a step
-                    // ahead, so the ring's loads below are L2 hits with short latency.
-                    const Tile nt = wp.next();
-                    const int pg = 2 * static_cast<int>(rank) + (lane & 1);
-                    if (lane < 2 && pg < nt.np)
-                        ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(page_row(nt, pg)) * kRow,
-                                              kPage * kRow * 2);
-                }
-                if (cur.first) {
-                    // new unit segment: load Q (this CTA's 64 heads) from 9 lanes
-                    bool good = true;
-                    if (lane == 0) good = wait_bar(bar(BAR_Q_EMPTY), (uc & 1) ^ 1, abort_flag, p.status);
-                    good = __shfl_sync(0xffffffffu, good, 0);
-                    if (!good) { ok = false; break; }
-                    const int bt = cur.u / p.n_hb, hb = cur.u - bt * p.n_hb;
-                    const int qrow = bt * p.n_h + hb * 128 + 64 * static_cast<int>(rank);
-                    if (lane == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_Q_FULL), 2 * kQBytes);
-                    __syncwarp();
-                    const uint32_t qf = leader_bar(BAR_Q_FULL);
-                    if (lane < 8) ptx::tma_load_2d_pair(sbase + kOffQ + lane * kBox, &p.tm_qa, 64 * lane, qrow, qf, pol_q);
-                    if (lane == 8) ptx::tma_load_2d_pair(sbase + kOffQ + 8 * kBox, &p.tm_qr, 0, qrow, qf, pol_q);
-                    ++uc;
-                }
-                // S(cur): 9 column chunks of pages 2r, 2r+1
-                const bool h0 = 2 * static_cast<int>(rank) < cur.np, h1 = 2 * static_cast<int>(rank) + 1 < cur.np;
-                const int r0 = h0 ? page_row(cur, 2 * rank) : 0;
-                const int r1 = h1 ? page_row(cur, 2 * rank + 1) : 0;
-                for (int c = 0; c < 9; ++c, ++n) {
-                    ent_row[n][0] = r0;
-                    ent_row[n][1] = r1;
-                    ent_col[n][0] = ent_col[n][1] = 64 * c;
-                    ent_has[n] = (h0 ? 1u : 0u) | (h1 ? 2u : 0u);
-                    ent_tx[n] = static_cast<uint32_t>(cur.np) * kBox;    // both CTAs together
-                }
-            }
-            if (have_prev) {
-                // V(prev): per page, per P.V instruction h: 2 latent chunks, all 64 keys
-                for (int pg = 0; pg < prev.np; ++pg) {
-                    const int r = page_row(prev, pg);
-                    for (int h = 0; h < 2; ++h, ++n) {
-                        ent_row[n][0] = ent_row[n][1] = r;
-                        ent_col[n][0] = 64 * owned_chunk(rank, h, 0);
-                        ent_col[n][1] = 64 * owned_chunk(rank, h, 1);
-                        ent_has[n] = 7u;
-                        ent_tx[n] = 2 * kEntry;
-                    }
-                }
-            }
-            for (int k = 0; k < n && ok; k += kBatch) {
-                const int nb = min(kBatch, n - k);
+            if (cur.first) {
+                // new unit segment: load Q (this CTA's 64 heads) from 9 lanes
                 bool good = true;
-                if (lane == 0) {
-                    for (int j = 0; j < nb && good; ++j) {
-                        const int ee = e + j;
-                        good = wait_bar(bar(BAR_RING_EMPTY + ee % kRing), ((ee / kRing) & 1) ^ 1, abort_flag, p.status);
-                        if (good && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_RING_FULL + ee % kRing), ent_tx[k + j]);
-                    }
-                }
+                if (lane == 0) good = wait_bar(bar(BAR_Q_EMPTY), (uc & 1) ^ 1, abort_flag, p.status);
                 good = __shfl_sync(0xffffffffu, good, 0);
                 if (!good) { ok = false; break; }
-                const int j = lane >> 1, half = lane & 1;
-                if (j < nb && (ent_has[k + j] >> half & 1u)) {
-                    const int ee = e + j;
-                    const uint32_t dst = sbase + kOffRing + (ee % kRing) * kEntry + half * kBox;
-                    // S loads keep normal L2 priority: the peer CTA reads the same lines
-                    // again for its P.V operand one step later; V loads are their last use
-                    if (ent_has[k + j] & 4u)
-                        ptx::tma_load_2d_pair(dst, &p.tm_pool, ent_col[k + j][half], ent_row[k + j][half],
-                                              leader_bar(BAR_RING_FULL + ee % kRing), pol_stream);
-                    else
-                        ptx::tma_load_2d_pair_normal(dst, &p.tm_pool, ent_col[k + j][half], ent_row[k + j][half],
-                                                     leader_bar(BAR_RING_FULL + ee % kRing));
-                }
-                e += nb;
+                const int bt = cur.u / p.n_hb, hb = cur.u - bt * p.n_hb;
+                const int qrow = bt * p.n_h + hb * 128 + 64 * static_cast<int>(rank);
+                if (lane == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_Q_FULL), 2 * kQBytes);
+                __syncwarp();
+                const uint32_t qf = leader_bar(BAR_Q_FULL);
+                if (lane < 8) ptx::tma_load_2d_pair(sbase + kOffQ + lane * kBox, &p.tm_qa, 64 * lane, qrow, qf, pol_q);
+                if (lane == 8) ptx::tma_load_2d_pair(sbase + kOffQ + 8 * kBox, &p.tm_qr, 0, qrow, qf, pol_q);
+                ++uc;
             }
-            have_prev = has_cur;
-            prev = cur;
+            // S(cur): 9 column chunks of pages 2r, 2r+1
+            const int my_pg = 2 * static_cast<int>(rank) + (lane & 1);
+            const bool has = lane < 2 && my_pg < cur.np;
+            const int row = has ? page_row(cur, my_pg) : 0;
+            const uint32_t tx = static_cast<uint32_t>(cur.np) * kBox;    // both CTAs together
+            for (int c = 0; c < 9; ++c, ++e) {
+                const int slot = e % kSRing;
+                bool good = true;
+                if (lane < 2) {
+                    good = wait_bar(bar(BAR_SR_EMPTY + slot), ((e / kSRing) & 1) ^ 1, abort_flag, p.status);
+                    if (good && lane == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_SR_FULL + slot), tx);
+                    if (good && has)
+                        ptx::tma_load_2d_pair_normal(sbase + kOffSRing + slot * kEntry + (lane & 1) * kBox, &p.tm_pool,
+                                                     64 * c, row, leader_bar(BAR_SR_FULL + slot));
+                }
+                if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
+            }
+        }
+    } else if (warp == 7) {
+        // ------------------------------------------------------------ V stream
+        const uint64_t pol_v = ptx::l2_policy_evict_first();   // last use of these lines
+        TileWalker w;
+        w.init(p.prefix, p.U, g0, g1);
+        int e = 0;
+        bool ok = g0 < g1;
+        while (ok && !w.done()) {
+            const Tile cur = w.next();
+            for (int pg = 0; pg < cur.np && ok; ++pg) {
+                const int row = page_row(cur, pg);
+                for (int h = 0; h < 2; ++h, ++e) {
+                    const int slot = e % kVRing;
+                    bool good = true;
+                    if (lane < 2) {
+                        good = wait_bar(bar(BAR_VR_EMPTY + slot), ((e / kVRing) & 1) ^ 1, abort_flag, p.status);
+                        if (good && lane == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_VR_FULL + slot), 2 * kEntry);
+                        if (good)
+                            ptx::tma_load_2d_pair(sbase + kOffVRing + slot * kEntry + lane * kBox, &p.tm_pool,
+                                                  64 * owned_chunk(rank, h, lane), row, leader_bar(BAR_VR_FULL + slot),
+                                                  pol_v);
+                    }
+                    if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
+                }
+            }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ S = Q K^T issuer
+        // S(i) occupies entries 9 i .. 9 i + 8 of the S ring.
         if (rank == 0 && lane == 0 && g0 < g1) {
             TileWalker w;
             w.init(p.prefix, p.U, g0, g1);
-            Tile cur{}, prev{};
-            bool have_prev = false;
-            int e = 0, i = 0, uc = 0, tails = 0;
+            int i = 0, uc = 0;
             bool ok = true;
-            auto wait_entry = [&](int idx) -> bool {
-                return wait_bar(bar(BAR_RING_FULL + idx % kRing), (idx / kRing) & 1, abort_flag, p.status);
-            };
-            while (ok && (!w.done() || have_prev)) {
-                const bool has_cur = !w.done();
-                if (has_cur) {
-                    cur = w.next();
-                    const int sb = i & 1;
-                    if (cur.first && !(ok = wait_bar(bar(BAR_Q_FULL), uc & 1, abort_flag, p.status))) break;
-                    if (!(ok = wait_bar(bar(BAR_S_FREE + sb), ((i >> 1) & 1) ^ 1, abort_flag, p.status))) break;
-                    const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffQ, 16, 1024);
-                    for (int c = 0; c < 9; ++c) {
-                        if (!(ok = wait_entry(e))) break;
-                        ptx::tc_fence_after();
-                        const uint64_t b0 = ptx::smem_desc_sw128(sbase + kOffRing + (e % kRing) * kEntry, 16, 1024);
-#pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4) {
-                            const uint64_t a = a0 + static_cast<uint64_t>((c * kBox + 32 * k4) >> 4);
-                            const uint64_t bd = b0 + static_cast<uint64_t>((32 * k4) >> 4);
-                            ptx::mma_pair_ss(tmem_base + kTmemS + 128 * sb, a, bd, kIdescS, (c | k4) ? 1u : 0u);
-                        }
-                        ptx::mma_commit_pair(bar(BAR_RING_EMPTY + e % kRing), 0x3);
-                        ++e;
-                    }
-                    if (!ok) break;
-                    ptx::mma_commit_pair(bar(BAR_S_FULL + sb), 0x3);
-                    if (cur.last) {
-                        ptx::mma_commit_pair(bar(BAR_Q_EMPTY), 0x3);
-                        ++uc;
-                    }
-                    ++i;
-                }
-                if (have_prev) {
-                    // P.V of the previous tile, once its P is written
-                    const int ip = i - 1 - (has_cur ? 1 : 0);
-                    if (!(ok = wait_bar(bar(BAR_P_FULL), ip & 1, abort_flag, p.status))) break;
-                    const int4 meta = p.unit_meta[prev.u];
-                    const bool tail = prev.unit_end && (meta.x % kPage) != 0;
+            const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffQ, 16, 1024);
+            while (ok && !w.done()) {
+                const Tile cur = w.next();
+                const int e0 = 9 * i;
+                const int sb = i & 1;
+                if (cur.first && !(ok = wait_bar(bar(BAR_Q_FULL), uc & 1, abort_flag, p.status))) break;
+                if (!(ok = wait_bar(bar(BAR_S_FREE + sb), ((i >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+                for (int c = 0; c < 9; ++c) {
+                    const int e = e0 + c;
+                    if (!(ok = wait_bar(bar(BAR_SR_FULL + e % kSRing), (e / kSRing) & 1, abort_flag, p.status))) break;
                     ptx::tc_fence_after();
-                    const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffP, 16, 1024);
-                    for (int pg = 0; pg < prev.np && ok; ++pg) {
-                        if (tail && pg == prev.np - 1) {
-                            // the unit's last page holds rows past the end: once its two
-                            // V entries have landed, the softmax warps of both CTAs zero
-                            // those rows (entries are consumed in ring order, so the
-                            // earlier pages' slots are already free for these loads)
-                            if (!(ok = wait_entry(e) && wait_entry(e + 1))) break;
-                            ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 0));
-                            ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 1));
-                            if (!(ok = wait_bar(bar(BAR_TAIL_DONE), tails & 1, abort_flag, p.status))) break;
-                            ++tails;
-                        }
-                        for (int h = 0; h < 2; ++h) {
-                            if (!(ok = wait_entry(e))) break;
-                            ptx::tc_fence_after();
-                            const uint64_t b0 = ptx::smem_desc_sw128(sbase + kOffRing + (e % kRing) * kEntry, kBox, 1024);
+                    const uint64_t b0 = ptx::smem_desc_sw128(sbase + kOffSRing + (e % kSRing) * kEntry, 16, 1024);
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk) {
-                                const uint64_t a = a0 + static_cast<uint64_t>((pg * kBox + 32 * kk) >> 4);
-                                const uint64_t bd = b0 + static_cast<uint64_t>((2048 * kk) >> 4);
-                                ptx::mma_pair_ss(tmem_base + kTmemO + 128 * h, a, bd, kIdescPV,
-                                                 (prev.first && pg == 0 && kk == 0) ? 0u : 1u);
-                            }
-                            ptx::mma_commit_pair(bar(BAR_RING_EMPTY + e % kRing), 0x3);
-                            ++e;
-                        }
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const uint64_t a = a0 + static_cast<uint64_t>((c * kBox + 32 * k4) >> 4);
+                        const uint64_t bd = b0 + static_cast<uint64_t>((32 * k4) >> 4);
+                        ptx::mma_pair_ss(tmem_base + kTmemS + 128 * sb, a, bd, kIdescS, (c | k4) ? 1u : 0u);
                     }
-                    if (!ok) break;
-                    ptx::mma_commit_pair(bar(BAR_P_FREE), 0x3);
+                    ptx::mma_commit_pair(bar(BAR_SR_EMPTY + e % kSRing), 0x3);
                 }
-                have_prev = has_cur;
-                prev = cur;
+                if (!ok) break;
+                ptx::mma_commit_pair(bar(BAR_S_FULL + sb), 0x3);
+                if (cur.last) {
+                    ptx::mma_commit_pair(bar(BAR_Q_EMPTY), 0x3);
+                    ++uc;
+                }
+                ++i;
             }
             if (!ok) {
-                // let every issued MMA finish before the teardown frees anything
+                // let every MMA this thread issued finish before the teardown frees anything
                 ptx::mma_commit_pair(bar(BAR_DRAIN), 0x1);
                 const uint64_t t0 = ptx::global_timer_ns();
                 while (!ptx::mbar_try_wait(bar(BAR_DRAIN), 0) && ptx::global_timer_ns() - t0 < kTimeoutNs) {
+                }
+            }
+        }
+    } else if (warp == 6) {
+        // ------------------------------------------------------------ O += P V issuer
+        // V(i) occupies the next 2 np entries of the V ring.
+        if (rank == 0 && lane == 0 && g0 < g1) {
+            TileWalker w;
+            w.init(p.prefix, p.U, g0, g1);
+            int i = 0, tails = 0, e = 0;
+            bool ok = true;
+            const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffP, 16, 1024);
+            while (ok && !w.done()) {
+                const Tile t = w.next();
+                const int kv_len = p.unit_meta[t.u].x;   // read before the wait hides its latency
+                if (!(ok = wait_bar(bar(BAR_P_FULL), i & 1, abort_flag, p.status))) break;
+                const bool tail = t.unit_end && (kv_len % kPage) != 0;
+                ptx::tc_fence_after();
+                for (int pg = 0; pg < t.np && ok; ++pg) {
+                    if (tail && pg == t.np - 1) {
+                        // the unit's last page holds rows past the end: once its two
+                        // V entries have landed, the softmax warps of both CTAs zero
+                        // those rows (entries are consumed in ring order, so the
+                        // earlier pages' slots are already free for these loads)
+                        if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status) &&
+                                   wait_bar(bar(BAR_VR_FULL + (e + 1) % kVRing), ((e + 1) / kVRing) & 1, abort_flag,
+                                            p.status)))
+                            break;
+                        ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 0));
+                        ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 1));
+                        if (!(ok = wait_bar(bar(BAR_TAIL_DONE), tails & 1, abort_flag, p.status))) break;
+                        ++tails;
+                    }
+                    for (int h = 0; h < 2; ++h, ++e) {
+                        if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status))) break;
+                        ptx::tc_fence_after();
+                        const uint64_t b0 = ptx::smem_desc_sw128(sbase + kOffVRing + (e % kVRing) * kEntry, kBox, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t a = a0 + static_cast<uint64_t>((pg * kBox + 32 * kk) >> 4);
+                            const uint64_t bd = b0 + static_cast<uint64_t>((2048 * kk) >> 4);
+                            ptx::mma_pair_ss(tmem_base + kTmemO + 128 * h, a, bd, kIdescPV,
+                                             (t.first && pg == 0 && kk == 0) ? 0u : 1u);
+                        }
+                        ptx::mma_commit_pair(bar(BAR_VR_EMPTY + e % kVRing), 0x3);
+                    }
+                }
+                if (!ok) break;
+                ptx::mma_commit_pair(bar(BAR_P_FREE), 0x3);
+                ++i;
+            }
+            if (!ok) {
+                ptx::mma_commit_pair(bar(BAR_DRAIN_PV), 0x1);
+                const uint64_t t0 = ptx::global_timer_ns();
+                while (!ptx::mbar_try_wait(bar(BAR_DRAIN_PV), 0) && ptx::global_timer_ns() - t0 < kTimeoutNs) {
                 }
             }
         }
@@ -464,7 +457,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         float m_used = -INFINITY, l_part = 0.f;
         while (ok && !w.done()) {
             const Tile t = w.next();
-            const bool is_cluster_last = w.done();
             const int4 meta = p.unit_meta[t.u];
             // keys of this tile that belong to this segment
             const int key_end = min(meta.x, kPage * (t.page0 + t.np));
@@ -485,7 +477,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             ptx::tmem_wait_ld();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_S_FREE + sb));
+            if (lane == 0) ptx::mbar_arrive_cluster_relaxed(leader_bar(BAR_S_FREE + sb));
 
             const int key0 = kPage * t.page0 + (hi ? 128 : 0);
             float mx = -INFINITY;
@@ -549,8 +541,8 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_P_FULL));
 
-            // ring position of this tile's V entries (same order as the producer)
-            const int v_start = 9 * (i + (is_cluster_last ? 1 : 2)) + v_before;
+            // V ring position of this tile's entries
+            const int v_start = v_before;
             v_before += 2 * t.np;
             if (t.unit_end && (meta.x % kPage) != 0) {
                 // zero rows past the end in this CTA's two V entries of the last page
@@ -566,7 +558,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                     const int half = rem / (bad * 8);
                     const int rem2 = rem - half * bad * 8;
                     const int row = valid + (rem2 >> 3), ch = rem2 & 7;
-                    uint4* dst = reinterpret_cast<uint4*>(smem + kOffRing + ((et + ent) % kRing) * kEntry +
+                    uint4* dst = reinterpret_cast<uint4*>(smem + kOffVRing + ((et + ent) % kVRing) * kEntry +
                                                           half * kBox + row * 128) + ch;
                     *dst = make_uint4(0, 0, 0, 0);
                 }
