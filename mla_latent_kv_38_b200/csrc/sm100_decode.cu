@@ -50,8 +50,8 @@ constexpr int kClusters = 74;                     // 148 SMs / 2
 constexpr int kDc = 512, kDr = 64, kRow = 576;    // row = c^KV || k^R
 constexpr int kPage = 64;                         // cache rows per page (TMA box height)
 constexpr int kTilePages = 4;                     // a tile = 4 pages = 256 keys (MMA N)
-constexpr int kSRing = 4;                         // 16 KB entries, S operand stream
-constexpr int kVRing = 3;                         // 16 KB entries, P.V operand stream
+constexpr int kSRing = 3;                         // 16 KB entries, S operand stream
+constexpr int kVRing = 4;                         // 16 KB entries, P.V operand stream
 
 constexpr uint32_t kBox = 8192;                   // one page x 64 columns (128 B rows)
 constexpr uint32_t kEntry = 2 * kBox;             // ring entry: 2 boxes
@@ -99,12 +99,14 @@ constexpr float kRescaleThreshold = 8.0f;         // log2 units
 
 struct Sm100Params {
     CUtensorMap tm_pool;      // pool as [rows][576], box 64 cols x 64 rows
+    CUtensorMap tm_pool_v;    // pool as [chunk][rows][64], box 64 cols x 64 rows x 2 chunks
     CUtensorMap tm_qa;        // q_abs as [n_tok*n_h][512], box 64 x 64
     CUtensorMap tm_qr;        // q_r   as [n_tok*n_h][64],  box 64 x 64
     const uint16_t* pool;     // for L2 prefetches of whole pages
     const int32_t* block_table;
     const int32_t* prefix;    // (U + 1) exclusive prefix of pages per unit
     const int4* unit_meta;    // (U) {kv_len, first cluster, parts, batch index}
+    const int4* cluster_info; // (C) {first page, end page, first unit, -}
     uint16_t* out_latent;
     float* out_lse;
     float* part_o;            // (C + U) slots x 128 rows x 512
@@ -155,12 +157,12 @@ struct Tile {
 struct TileWalker {
     const int32_t* prefix;
     int g, g0, g1, u;
-    __device__ void init(const int32_t* pf, int U, int g0_, int g1_) {
+    __device__ void init(const int32_t* pf, int u0, int g0_, int g1_) {
         prefix = pf;
         g = g0_;
         g0 = g0_;
         g1 = g1_;
-        u = g0_ < g1_ ? find_unit(pf, U, g0_) : 0;
+        u = u0;
         while (g < g1 && prefix[u + 1] <= g) ++u;
     }
     __device__ bool done() const { return g >= g1; }
@@ -240,12 +242,10 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    // this cluster's contiguous range of global pages; with fewer pages than
-    // clusters only the first `total` clusters work, so no range is empty
-    const int total = p.prefix[p.U];
-    const int Ce = min(p.C, total);
-    const int g0 = cluster < Ce ? static_cast<int>((static_cast<long long>(cluster) * total) / Ce) : 0;
-    const int g1 = cluster < Ce ? static_cast<int>((static_cast<long long>(cluster + 1) * total) / Ce) : 0;
+    // this cluster's contiguous range of global pages [g0, g1) and the unit of
+    // page g0, precomputed by the schedule kernel (empty range: no work)
+    const int4 cinfo = p.cluster_info[cluster];
+    const int g0 = cinfo.x, g1 = cinfo.y, u0 = cinfo.z;
 
     // Two load streams, each consumed in order by one MMA issuer:
     //   S ring: S(i) = 9 entries (column chunk c of this CTA's pages 2r, 2r+1)
@@ -267,8 +267,8 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // of the leader CTA arms the full barrier with both CTAs' bytes).
         const uint64_t pol_q = ptx::l2_policy_evict_last();
         TileWalker w, wp;
-        w.init(p.prefix, p.U, g0, g1);
-        wp.init(p.prefix, p.U, g0, g1);
+        w.init(p.prefix, u0, g0, g1);
+        wp.init(p.prefix, u0, g0, g1);
         if (!wp.done()) wp.next();   // the look-ahead walker runs one tile ahead
         int e = 0, uc = 0;
         bool ok = g0 < g1;
@@ -319,7 +319,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // ------------------------------------------------------------ V stream
         const uint64_t pol_v = ptx::l2_policy_evict_first();   // last use of these lines
         TileWalker w;
-        w.init(p.prefix, p.U, g0, g1);
+        w.init(p.prefix, u0, g0, g1);
         int e = 0;
         bool ok = g0 < g1;
         while (ok && !w.done()) {
@@ -329,13 +329,13 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 for (int h = 0; h < 2; ++h, ++e) {
                     const int slot = e % kVRing;
                     bool good = true;
-                    if (lane < 2) {
+                    if (lane == 0) {
                         good = wait_bar(bar(BAR_VR_EMPTY + slot), ((e / kVRing) & 1) ^ 1, abort_flag, p.status);
-                        if (good && lane == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_VR_FULL + slot), 2 * kEntry);
+                        if (good && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_VR_FULL + slot), 2 * kEntry);
+                        // both latent chunks of the page in one box: [chunk][row][64 columns]
                         if (good)
-                            ptx::tma_load_2d_pair(sbase + kOffVRing + slot * kEntry + lane * kBox, &p.tm_pool,
-                                                  64 * owned_chunk(rank, h, lane), row, leader_bar(BAR_VR_FULL + slot),
-                                                  pol_v);
+                            ptx::tma_load_3d_pair(sbase + kOffVRing + slot * kEntry, &p.tm_pool_v, 0, row,
+                                                  owned_chunk(rank, h, 0), leader_bar(BAR_VR_FULL + slot), pol_v);
                     }
                     if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
                 }
@@ -346,7 +346,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // S(i) occupies entries 9 i .. 9 i + 8 of the S ring.
         if (rank == 0 && lane == 0 && g0 < g1) {
             TileWalker w;
-            w.init(p.prefix, p.U, g0, g1);
+            w.init(p.prefix, u0, g0, g1);
             int i = 0, uc = 0;
             bool ok = true;
             const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffQ, 16, 1024);
@@ -356,10 +356,10 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 const int sb = i & 1;
                 if (cur.first && !(ok = wait_bar(bar(BAR_Q_FULL), uc & 1, abort_flag, p.status))) break;
                 if (!(ok = wait_bar(bar(BAR_S_FREE + sb), ((i >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+                ptx::tc_fence_after();   // the softmax's reads of this S buffer are done
                 for (int c = 0; c < 9; ++c) {
                     const int e = e0 + c;
                     if (!(ok = wait_bar(bar(BAR_SR_FULL + e % kSRing), (e / kSRing) & 1, abort_flag, p.status))) break;
-                    ptx::tc_fence_after();
                     const uint64_t b0 = ptx::smem_desc_sw128(sbase + kOffSRing + (e % kSRing) * kEntry, 16, 1024);
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
@@ -390,7 +390,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // V(i) occupies the next 2 np entries of the V ring.
         if (rank == 0 && lane == 0 && g0 < g1) {
             TileWalker w;
-            w.init(p.prefix, p.U, g0, g1);
+            w.init(p.prefix, u0, g0, g1);
             int i = 0, tails = 0, e = 0;
             bool ok = true;
             const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffP, 16, 1024);
@@ -417,7 +417,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                     }
                     for (int h = 0; h < 2; ++h, ++e) {
                         if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status))) break;
-                        ptx::tc_fence_after();
                         const uint64_t b0 = ptx::smem_desc_sw128(sbase + kOffVRing + (e % kVRing) * kEntry, kBox, 1024);
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
@@ -450,7 +449,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         float* xmax = reinterpret_cast<float*>(smem + kOffXmax);
         float* xsum = reinterpret_cast<float*>(smem + kOffXsum);
         TileWalker w;
-        w.init(p.prefix, p.U, g0, g1);
+        w.init(p.prefix, u0, g0, g1);
         int i = 0, tails = 0;
         int v_before = 0;      // V ring entries of tiles before i
         bool ok = true;
@@ -642,7 +641,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
 __global__ void __launch_bounds__(1024)
 mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, int n_hb,
                           int max_blocks, int C, int32_t* __restrict__ prefix,
-                          int4* __restrict__ unit_meta, int32_t* status) {
+                          int4* __restrict__ unit_meta, int4* __restrict__ cluster_info, int32_t* status) {
     __shared__ int warp_tot[32];
     __shared__ int carry;
     const int U = B * T_q * n_hb;
@@ -704,6 +703,22 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, 
             unit_meta[u].y = c0;
             unit_meta[u].z = c1 - c0 + 1;
         }
+    }
+    // per cluster: page range and the unit holding its first page
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += 1024) {
+        int4 ci = make_int4(0, 0, 0, 0);
+        if (c < Ce) {
+            const int a = static_cast<int>((static_cast<long long>(c) * T) / Ce);
+            const int e = static_cast<int>((static_cast<long long>(c + 1) * T) / Ce);
+            int lo = 0, hi = U - 1;   // last unit with prefix <= a
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (prefix[mid] <= a) lo = mid; else hi = mid - 1;
+            }
+            ci = make_int4(a, e, lo, 0);
+        }
+        cluster_info[c] = ci;
     }
 }
 
@@ -779,17 +794,32 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The pool viewed as [chunk (9)][row][64 columns]: one box loads several
+// 64-column chunks of the same rows into consecutive 8 KB blocks.
+bool make_map_chunks(CUtensorMap* m, const void* base, uint64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[3] = {64, rows, 9};
+    const cuuint64_t strides[2] = {kRow * 2, 128};
+    const cuuint32_t box[3] = {64, 64, 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 size_t r256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct Sm100Ws {
-    size_t prefix, meta, part_lse, part_o, total;
+    size_t prefix, meta, cinfo, part_lse, part_o, total;
 };
 
 Sm100Ws sm100_ws(int U) {
     Sm100Ws w;
     w.prefix = 0;
     w.meta = w.prefix + r256(static_cast<size_t>(U + 1) * 4);
-    w.part_lse = w.meta + r256(static_cast<size_t>(U) * 16);
+    w.cinfo = w.meta + r256(static_cast<size_t>(U) * 16);
+    w.part_lse = w.cinfo + r256(static_cast<size_t>(kClusters) * 16);
     w.part_o = w.part_lse + r256(static_cast<size_t>(kClusters + U) * 128 * 4);
     w.total = w.part_o + r256(static_cast<size_t>(kClusters + U) * 128 * kDc * 4);
     return w;
@@ -816,6 +846,7 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int /*max_split
     const uint64_t pool_rows = static_cast<uint64_t>(P.num_blocks) * P.block_size;
     const uint64_t q_rows = static_cast<uint64_t>(P.n_tok) * P.n_h;
     if (!make_map_2d(&k.tm_pool, P.pool, kRow, pool_rows, kRow * 2, 64, 64) ||
+        !make_map_chunks(&k.tm_pool_v, P.pool, pool_rows) ||
         !make_map_2d(&k.tm_qa, P.q_abs, kDc, q_rows, kDc * 2, 64, 64) ||
         !make_map_2d(&k.tm_qr, P.q_r, kDr, q_rows, kDr * 2, 64, 64))
         return cudaErrorInvalidValue;
@@ -823,6 +854,7 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int /*max_split
     k.block_table = P.block_table;
     k.prefix = reinterpret_cast<const int32_t*>(base + w.prefix);
     k.unit_meta = reinterpret_cast<const int4*>(base + w.meta);
+    k.cluster_info = reinterpret_cast<const int4*>(base + w.cinfo);
     k.out_latent = P.out_latent;
     k.out_lse = P.out_lse;
     k.part_o = reinterpret_cast<float*>(base + w.part_o);
@@ -839,7 +871,8 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int /*max_split
 
     mla_sm100_schedule_kernel<<<1, 1024, 0, stream>>>(P.seq_lens, P.B, P.T_q, n_hb, P.max_blocks, kClusters,
                                                       reinterpret_cast<int32_t*>(base + w.prefix),
-                                                      reinterpret_cast<int4*>(base + w.meta), P.status);
+                                                      reinterpret_cast<int4*>(base + w.meta),
+                                                      reinterpret_cast<int4*>(base + w.cinfo), P.status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(mla_decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

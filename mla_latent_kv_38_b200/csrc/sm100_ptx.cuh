@@ -106,6 +106,16 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap,
         : "memory");
 }
 
+// 3D tiled load (same conventions as the 2D form).
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void* tmap, int x, int y, int z,
+                                                 uint32_t mbar_cluster_addr, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(mbar_cluster_addr), "r"(x), "r"(y), "r"(z), "l"(policy)
+        : "memory");
+}
+
 // Same without an L2 eviction hint (normal priority).
 __device__ __forceinline__ void tma_load_2d_pair_normal(uint32_t dst, const void* tmap, int x, int y,
                                                         uint32_t mbar_cluster_addr) {
