@@ -249,7 +249,7 @@ def run_ours(args):
         raise RuntimeError(f"device status {st} after warm-up")
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
     sampler = ClockSampler(local)
     barrier()
     torch.cuda.synchronize(dev)
@@ -260,6 +260,7 @@ def run_ours(args):
             s = dc.spec
             ev[k][0].record(stream)
             M.mla_absorb_q(dc.cfg, dc.q_c, dc.w_uk, dc.q_abs, s.n_tok)
+            ev[k][4].record(stream)
             M.mla_rope_append(dc.cfg, dc.q_r, dc.k_r_new, dc.c_kv_new, dc.positions, dc.rope_table,
                               dc.max_pos, dc.block_table, s.max_blocks, dc.pool, s.num_blocks, s.B,
                               s.T_q, dc.status)
@@ -272,6 +273,12 @@ def run_ours(args):
     barrier()
     step_ms = sum(e[0].elapsed_time(e[3]) for e in ev)
     decode_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    phases_us = {
+        "absorb_q": 1e3 * sum(e[0].elapsed_time(e[4]) for e in ev) / K,
+        "rope_append": 1e3 * sum(e[4].elapsed_time(e[1]) for e in ev) / K,
+        "decode": 1e3 * decode_ms,
+        "up_v": 1e3 * sum(e[2].elapsed_time(e[3]) for e in ev) / K,
+    }
     step_ms = max_over_ranks(step_ms)
     tokens_per_step = spec.n_tok
     value = world * tokens_per_step * K / (step_ms / 1e3)
@@ -342,6 +349,7 @@ def run_ours(args):
                    "context": [int(spec.seq_lens.min()), int(spec.seq_lens.max())],
                    "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write)",
                    "parallelism": f"replicas x{world}"},
+        "phases_us": phases_us,
         "decode_hbm_tbs": hbm_gbs / 1e3, "decode_tflops": tflops,
         "decode_tflops_frac_sustained": tflops / peaks.get("bf16_tflops_sustained", 1e9),
         "roofline": roof,

@@ -61,9 +61,13 @@ typedef struct {
     int d_r;
     int block_size;
     float scale;
-    int impl; /* mla_decode kernel: 0 = best for the shape, 1 = portable
-                 SIMT kernel (any supported shape), 2 = tcgen05 kernel
-                 (d_c = 512, d_r = 64, n_h a multiple of 64 only) */
+    int impl; /* kernel family: 0 = best for the shape, 1 = portable CUDA-core
+                 kernels (any supported shape), 2 = tcgen05 tensor-core kernels,
+                 MLA_ERR_CONFIG where they do not tile the shape:
+                   mla_decode   d_c = 512, d_r = 64, n_h a multiple of 128
+                   mla_absorb_q d_h a multiple of 64, d_c a multiple of 128
+                   mla_up_v     d_h a multiple of 128
+                 (mla_rope_append has one kernel for every shape) */
 } mla_config_t;
 
 enum {

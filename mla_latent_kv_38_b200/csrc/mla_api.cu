@@ -7,6 +7,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100_decode.h"
+#include "sm100_proj.h"
 
 namespace {
 
@@ -110,8 +111,14 @@ int mla_absorb_q(const mla_config_t* cfg, const mla_bf16* q_c, const mla_bf16* w
     if (!q_c || !w_uk || !q_abs) return MLA_ERR_NULL;
     if (!aligned16(q_c) || !aligned16(w_uk) || !aligned16(q_abs)) return MLA_ERR_ALIGN;
     if (n_tok < 1 || n_tok > 65536) return MLA_ERR_SIZE;
-    return cuda_rc(mla::launch_absorb_q_simt(q_c, w_uk, q_abs, n_tok, cfg->n_h, cfg->d_h, cfg->d_c,
-                                             static_cast<cudaStream_t>(stream)));
+    const bool sm100_shape = mla::sm100_absorb_supports(cfg->d_h, cfg->d_c);
+    if (cfg->impl == 2 && !sm100_shape) return MLA_ERR_CONFIG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cfg->impl == 2 || (cfg->impl == 0 && sm100_shape)) {
+        if (mla_check_device() != MLA_OK) return MLA_ERR_UNSUPPORTED;
+        return cuda_rc(mla::launch_absorb_q_sm100(q_c, w_uk, q_abs, n_tok, cfg->n_h, cfg->d_h, cfg->d_c, st));
+    }
+    return cuda_rc(mla::launch_absorb_q_simt(q_c, w_uk, q_abs, n_tok, cfg->n_h, cfg->d_h, cfg->d_c, st));
 }
 
 int mla_rope_append(const mla_config_t* cfg, mla_bf16* q_r, const mla_bf16* k_r,
@@ -212,8 +219,14 @@ int mla_up_v(const mla_config_t* cfg, const mla_bf16* latent, const mla_bf16* w_
     if (!latent || !w_uv || !out) return MLA_ERR_NULL;
     if (!aligned16(latent) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_ALIGN;
     if (n_tok < 1 || n_tok > 65536) return MLA_ERR_SIZE;
-    return cuda_rc(mla::launch_up_v_simt(latent, w_uv, out, n_tok, cfg->n_h, cfg->d_h, cfg->d_c,
-                                         static_cast<cudaStream_t>(stream)));
+    const bool sm100_shape = mla::sm100_up_v_supports(cfg->d_h, cfg->d_c);
+    if (cfg->impl == 2 && !sm100_shape) return MLA_ERR_CONFIG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cfg->impl == 2 || (cfg->impl == 0 && sm100_shape)) {
+        if (mla_check_device() != MLA_OK) return MLA_ERR_UNSUPPORTED;
+        return cuda_rc(mla::launch_up_v_sm100(latent, w_uv, out, n_tok, cfg->n_h, cfg->d_h, cfg->d_c, st));
+    }
+    return cuda_rc(mla::launch_up_v_simt(latent, w_uv, out, n_tok, cfg->n_h, cfg->d_h, cfg->d_c, st));
 }
 
 int mla_clear_status(int32_t* dev_status, void* stream) {

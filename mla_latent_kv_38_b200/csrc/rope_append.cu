@@ -8,7 +8,7 @@
 // absolute positions past_len .. T_total-1, and the cache is the latent
 // concatenated with the rotated key.
 //
-// One warp per token.  The latent row is a 16-byte vector copy (bit exact);
+// The latent row is a 16-byte vector copy (bit exact);
 // RoPE is float32 multiply / add with explicit round-to-nearest intrinsics so
 // that no fused multiply-add changes the bits, then bf16 round to nearest even.
 
@@ -26,14 +26,53 @@ __device__ __forceinline__ void rope_pair(uint16_t x1b, uint16_t x2b, float c, f
     *y2 = f2bf(b);
 }
 
+// Blocks [0, q_blocks) rotate the queries: one thread per (token, head, four
+// consecutive pairs m .. m+3), with 8-byte loads of both halves of the head's
+// RoPE part and 16-byte loads of the cos / sin rows.  The remaining blocks do
+// the cache append, one warp per token.
 __global__ void __launch_bounds__(256)
 rope_append_kernel(uint16_t* __restrict__ q_r, const uint16_t* __restrict__ k_r,
                    const uint16_t* __restrict__ c_kv, const int32_t* __restrict__ positions,
                    const float* __restrict__ table, int max_pos,
                    const int32_t* __restrict__ block_table, int max_blocks,
                    uint16_t* __restrict__ pool, int num_blocks, int n_tok, int T_q,
-                   int n_h, int d_c, int d_r, int block_size, int32_t* status) {
-    const int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+                   int n_h, int d_c, int d_r, int block_size, int q_blocks, int32_t* status) {
+    const int h = d_r >> 1;
+    if (static_cast<int>(blockIdx.x) < q_blocks) {
+        // ---- query RoPE, in place
+        const int quads = h >> 2;
+        const long g = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+        if (g >= static_cast<long>(n_tok) * n_h * quads) return;
+        const int m = static_cast<int>(g % quads) * 4;
+        const long ni = g / quads;                      // token * n_h + head
+        const int n = static_cast<int>(ni / n_h);
+        const int p = positions[n];
+        if (p < 0 || p >= max_pos || p / block_size >= max_blocks) return;   // flagged by the append
+        uint16_t* q = q_r + ni * d_r;
+        const float4 c = *reinterpret_cast<const float4*>(table + static_cast<size_t>(p) * d_r + m);
+        const float4 sn = *reinterpret_cast<const float4*>(table + static_cast<size_t>(p) * d_r + h + m);
+        const uint2 x1 = *reinterpret_cast<const uint2*>(q + m);
+        const uint2 x2 = *reinterpret_cast<const uint2*>(q + h + m);
+        const float cc[4] = {c.x, c.y, c.z, c.w}, ss[4] = {sn.x, sn.y, sn.z, sn.w};
+        const uint32_t a_in[2] = {x1.x, x1.y}, b_in[2] = {x2.x, x2.y};
+        uint32_t a_out[2], b_out[2];
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            uint16_t y1[2], y2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                rope_pair(static_cast<uint16_t>(a_in[w] >> (16 * e)), static_cast<uint16_t>(b_in[w] >> (16 * e)),
+                          cc[2 * w + e], ss[2 * w + e], &y1[e], &y2[e]);
+            a_out[w] = y1[0] | (static_cast<uint32_t>(y1[1]) << 16);
+            b_out[w] = y2[0] | (static_cast<uint32_t>(y2[1]) << 16);
+        }
+        *reinterpret_cast<uint2*>(q + m) = make_uint2(a_out[0], a_out[1]);
+        *reinterpret_cast<uint2*>(q + h + m) = make_uint2(b_out[0], b_out[1]);
+        return;
+    }
+
+    // ---- cache append, one warp per token
+    const int n = (blockIdx.x - q_blocks) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (n >= n_tok) return;
     const int b = n / T_q;
@@ -42,19 +81,7 @@ rope_append_kernel(uint16_t* __restrict__ q_r, const uint16_t* __restrict__ k_r,
         if (lane == 0) raise_status(status, MLA_STATUS_BAD_POSITION);
         return;
     }
-    const int h = d_r >> 1;
     const float* cs = table + static_cast<size_t>(p) * d_r;
-
-    // query RoPE, every head, in place
-    if (q_r != nullptr) {
-        uint16_t* q = q_r + static_cast<size_t>(n) * n_h * d_r;
-        for (int e = lane; e < n_h * h; e += 32) {
-            const int i = e / h, m = e - i * h;
-            uint16_t* qi = q + i * d_r;
-            rope_pair(qi[m], qi[m + h], cs[m], cs[h + m], &qi[m], &qi[m + h]);
-        }
-    }
-
     const int blk = block_table[static_cast<size_t>(b) * max_blocks + p / block_size];
     if (blk < 0 || blk >= num_blocks) {
         if (lane == 0) raise_status(status, MLA_STATUS_BAD_BLOCK);
@@ -80,12 +107,14 @@ cudaError_t launch_rope_append(uint16_t* q_r, const uint16_t* k_r, const uint16_
                                const int32_t* block_table, int max_blocks, uint16_t* pool,
                                int num_blocks, int n_tok, int T_q, int n_h, int d_c, int d_r,
                                int block_size, int32_t* status, cudaStream_t stream) {
-    const int warps = 8;
-    const int grid = (n_tok + warps - 1) / warps;
-    rope_append_kernel<<<grid, warps * 32, 0, stream>>>(q_r, k_r, c_kv, positions, table, max_pos,
-                                                        block_table, max_blocks, pool, num_blocks,
-                                                        n_tok, T_q, n_h, d_c, d_r, block_size,
-                                                        status);
+    const int threads = 256, warps = threads / 32;
+    const long q_threads = q_r != nullptr ? static_cast<long>(n_tok) * n_h * (d_r / 8) : 0;
+    const long q_blocks = (q_threads + threads - 1) / threads;
+    const long a_blocks = (n_tok + warps - 1) / warps;
+    if (q_blocks + a_blocks > 0x7fffffffL) return cudaErrorInvalidValue;
+    rope_append_kernel<<<static_cast<unsigned>(q_blocks + a_blocks), threads, 0, stream>>>(
+        q_r, k_r, c_kv, positions, table, max_pos, block_table, max_blocks, pool, num_blocks, n_tok, T_q, n_h, d_c,
+        d_r, block_size, static_cast<int>(q_blocks), status);
     return cudaGetLastError();
 }
 

@@ -1,0 +1,243 @@
+// Per-head projections around the absorbed decode on the tcgen05 tensor cores.
+//
+//   absorb_q: q_abs[n,i,:] = W^UK_i^T q^C[n,i,:]   ("MLA(Multi-head Latent
+//             Attention): DeepSeek-V2 논문정리", "Key에 대한 수식 전개")
+//   up_v:     o[n,i,:]     = W^UV_i latent[n,i,:]  (same page, "Value에 대한
+//             수식 전개")
+//
+// Both are, per head i, a product D = A . B^T with the head's weight slice as
+// A (M = 128 output features per CTA) and the tokens' activations as B
+// (N = tokens, K = the contracted feature):
+//
+//   absorb_q: A = W^UK_i^T  (M = latent column c, K = d_h), stored [k][c], so A
+//             is read MN-major; B = q^C[:, i, :] (K-major).
+//   up_v:     A = W^UV_i    (M = head feature k, K = d_c), stored [k][c], so A
+//             is K-major;  B = latent[:, i, :]  (K-major).
+//
+// With the few tokens of a decode step (N = 32 for 32 sequences) the weights
+// dominate the bytes (2 x 16 MiB at the DeepSeek-V2 shape) and both calls are
+// bound by HBM: each CTA loads its weight tile once with TMA, keeps it in
+// shared memory and runs every token tile of its head against it.  One thread
+// issues the MMAs (cta_group::1, M = 128, N = token tile <= 256) into tensor
+// memory; four warps read the fp32 accumulator back (one TMEM lane per thread,
+// i.e. one output feature per thread) and store it as bf16.
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "sm100_proj.h"
+#include "sm100_ptx.cuh"
+#include "tensor_map.h"
+
+namespace mla {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kM = 128;                       // output features per CTA
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr size_t kSmemLimit = 200 * 1024;     // A + B tiles per CTA
+constexpr size_t kSmemPerSm = 233472;         // shared memory of one SM (228 KB)
+
+struct ProjParams {
+    CUtensorMap tm_a;   // weights, [n_h * d_h][d_c], 64-column boxes
+    CUtensorMap tm_b;   // activations, [n_tok][n_h * K], boxes of 64 x nt
+    uint16_t* out;      // [n_tok][n_h][m_total]
+    int n_tok, n_h, d_h, d_c;
+    int K;              // contracted length: d_h (absorb_q) or d_c (up_v)
+    int m_total;        // output features per head: d_c (absorb_q) or d_h (up_v)
+    int nt;             // token tile (multiple of 16, <= 256)
+    uint32_t idesc;
+    uint32_t tmem_cols;
+};
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::global_timer_ns();
+    while (!ptx::mbar_try_wait(bar, parity))
+        if (ptx::global_timer_ns() - t0 > kTimeoutNs) return false;
+    return true;
+}
+
+// grid (m_total / 128, n_h); 128 threads.  kAbsorb selects the A layout.
+template <bool kAbsorb>
+__global__ void __launch_bounds__(kThreads, 1) mla_proj_sm100_kernel(const __grid_constant__ ProjParams p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                           ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = ptx::smem_u32(smem);
+    const int K = p.K, nt = p.nt;
+    const uint32_t a_bytes = static_cast<uint32_t>(kM) * K * 2;
+    const uint32_t b_box = static_cast<uint32_t>(nt) * 128;      // 64 columns x nt rows
+    const int kchunks = K / 64;
+    const uint32_t sA = sbase, sB = sbase + a_bytes;
+    const uint32_t bars = sB + kchunks * b_box;                  // full A, full B, MMA done
+    const uint32_t barA = bars, barB = bars + 8, barD = bars + 16;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bars - sbase) + 32);
+    __shared__ int s_ok;
+
+    const int warp = threadIdx.x >> 5;
+    const int head = blockIdx.y;
+    const int m0 = blockIdx.x * kM;
+    const int n_tiles = (p.n_tok + nt - 1) / nt;
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(barA, 1);
+        ptx::mbar_init(barB, 1);
+        ptx::mbar_init(barD, 1);
+        ptx::fence_mbar_init();
+        ptx::prefetch_tmap(&p.tm_a);
+        ptx::prefetch_tmap(&p.tm_b);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc1(ptx::smem_u32(tmem_slot), p.tmem_cols);
+        ptx::tmem_relinquish1();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto load_b = [&](int t) {
+        ptx::mbar_arrive_expect_tx(barB, kchunks * b_box);
+        for (int kc = 0; kc < kchunks; ++kc)
+            ptx::tma_load_2d(sB + kc * b_box, &p.tm_b, head * K + 64 * kc, t * nt, barB);
+    };
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_arrive_expect_tx(barA, a_bytes);
+        if (kAbsorb) {
+            // two boxes of 64 latent columns x d_h rows: [mh][k][64 c]
+            for (int mh = 0; mh < 2; ++mh)
+                ptx::tma_load_2d(sA + mh * (K * 128), &p.tm_a, m0 + 64 * mh, head * p.d_h, barA);
+        } else {
+            // d_c / 64 boxes of 64 latent columns x 128 rows: [kc][k][64 c]
+            for (int kc = 0; kc < kchunks; ++kc)
+                ptx::tma_load_2d(sA + kc * (kM * 128), &p.tm_a, 64 * kc, head * p.d_h + m0, barA);
+        }
+        load_b(0);
+    }
+
+    const int row = m0 + threadIdx.x;   // this thread's output feature (TMEM lane)
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    for (int t = 0; t < n_tiles; ++t) {
+        if (threadIdx.x == 0) {
+            bool ok = (t > 0 || wait_bounded(barA, 0)) && wait_bounded(barB, t & 1);
+            if (ok) {
+                ptx::tc_fence_after();
+                for (int s = 0; s < K / 16; ++s) {
+                    uint64_t a, b;
+                    if (kAbsorb) {
+                        // MN-major: 8-row (k) atoms 1 KB apart, the two 64-column halves K*128 B apart
+                        a = ptx::smem_desc_sw128(sA + s * 2048, K * 128, 1024);
+                    } else {
+                        a = ptx::smem_desc_sw128(sA + (s >> 2) * (kM * 128) + (s & 3) * 32, 16, 1024);
+                    }
+                    b = ptx::smem_desc_sw128(sB + (s >> 2) * b_box + (s & 3) * 32, 16, 1024);
+                    ptx::mma1_ss(tmem, a, b, p.idesc, s > 0 ? 1u : 0u);
+                }
+                ptx::mma1_commit(barD);
+                ok = wait_bounded(barD, t & 1);
+                // the MMAs have read B: fetch the next token tile during the epilogue
+                if (ok && t + 1 < n_tiles) load_b(t + 1);
+            }
+            s_ok = ok;
+        }
+        __syncthreads();
+        if (!s_ok) break;
+        ptx::tc_fence_after();
+        const int n0 = t * nt;
+        const int nvalid = min(nt, p.n_tok - n0);
+        uint16_t* dst = p.out + (static_cast<size_t>(n0) * p.n_h + head) * p.m_total + row;
+        const size_t step = static_cast<size_t>(p.n_h) * p.m_total;
+        for (int j0 = 0; j0 < nvalid; j0 += 16) {
+            uint32_t r[16];
+            ptx::tmem_ld16(t_lane + j0, r);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (j0 + j < nvalid) dst[static_cast<size_t>(j0 + j) * step] = f2bf(__uint_as_float(r[j]));
+        }
+        ptx::tc_fence_before();
+        __syncthreads();
+    }
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc1(tmem, p.tmem_cols);
+}
+
+uint32_t tmem_cols_for(int nt) {
+    uint32_t c = 32;
+    while (c < static_cast<uint32_t>(nt)) c <<= 1;
+    return c;
+}
+
+int token_tile(int n_tok, int K) {
+    const size_t a_bytes = static_cast<size_t>(kM) * K * 2;
+    int cap = static_cast<int>((kSmemLimit - a_bytes) / (static_cast<size_t>(K) * 2));
+    cap = cap / 16 * 16;
+    if (cap > 256) cap = 256;
+    const int want = (n_tok + 15) / 16 * 16;
+    return want < cap ? want : cap;
+}
+
+template <bool kAbsorb>
+cudaError_t launch_proj(ProjParams& p, cudaStream_t stream) {
+    size_t smem = static_cast<size_t>(kM) * p.K * 2 + static_cast<size_t>(p.K) * 2 * p.nt + 1024 + 64;
+    p.tmem_cols = tmem_cols_for(p.nt);
+    // no more CTAs per SM than the 512 tensor-memory columns hold, so that no
+    // allocation has to wait for another CTA to finish
+    const size_t max_ctas = 512 / p.tmem_cols;
+    const size_t min_smem = kSmemPerSm / (max_ctas + 1) - 1024 + 16;
+    if (max_ctas < 16 && smem < min_smem) smem = min_smem;
+    cudaError_t e = cudaFuncSetAttribute(mla_proj_sm100_kernel<kAbsorb>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    p.idesc = ptx::idesc_bf16_f32(kM, p.nt, kAbsorb ? 1 : 0, 0);
+    dim3 grid(p.m_total / kM, p.n_h);
+    mla_proj_sm100_kernel<kAbsorb><<<grid, kThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool sm100_absorb_supports(int d_h, int d_c) { return d_h % 64 == 0 && d_h <= 256 && d_c % kM == 0; }
+
+bool sm100_up_v_supports(int d_h, int d_c) { return d_h % kM == 0 && d_c % 64 == 0 && d_c <= 512; }
+
+cudaError_t launch_absorb_q_sm100(const uint16_t* q_c, const uint16_t* w_uk, uint16_t* q_abs, int n_tok, int n_h,
+                                  int d_h, int d_c, cudaStream_t stream) {
+    ProjParams p;
+    p.n_tok = n_tok;
+    p.n_h = n_h;
+    p.d_h = d_h;
+    p.d_c = d_c;
+    p.K = d_h;
+    p.m_total = d_c;
+    p.nt = token_tile(n_tok, d_h);
+    p.out = q_abs;
+    const uint64_t hk = static_cast<uint64_t>(n_h) * d_h;
+    if (!make_map_2d(&p.tm_a, w_uk, d_c, hk, static_cast<uint64_t>(d_c) * 2, 64, d_h) ||
+        !make_map_2d(&p.tm_b, q_c, hk, n_tok, hk * 2, 64, p.nt))
+        return cudaErrorInvalidValue;
+    return launch_proj<true>(p, stream);
+}
+
+cudaError_t launch_up_v_sm100(const uint16_t* latent, const uint16_t* w_uv, uint16_t* out, int n_tok, int n_h,
+                              int d_h, int d_c, cudaStream_t stream) {
+    ProjParams p;
+    p.n_tok = n_tok;
+    p.n_h = n_h;
+    p.d_h = d_h;
+    p.d_c = d_c;
+    p.K = d_c;
+    p.m_total = d_h;
+    p.nt = token_tile(n_tok, d_c);
+    p.out = out;
+    const uint64_t hk = static_cast<uint64_t>(n_h) * d_c;
+    if (!make_map_2d(&p.tm_a, w_uv, d_c, static_cast<uint64_t>(n_h) * d_h, static_cast<uint64_t>(d_c) * 2, 64,
+                     kM) ||
+        !make_map_2d(&p.tm_b, latent, hk, n_tok, hk * 2, 64, p.nt))
+        return cudaErrorInvalidValue;
+    return launch_proj<false>(p, stream);
+}
+
+}  // namespace mla

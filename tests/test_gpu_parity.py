@@ -130,25 +130,84 @@ def test_split_count_invariance(M, splits, impl):
     check_sequences(dc, range(spec.B))
 
 
-def test_absorb_q_parity(M):
-    spec = CaseSpec(**V2, seq_lens=np.array([64] * 5, np.int32), T_q=3, seed=7)
-    dc = _dc(spec, fill_history=False)
-    M.mla_absorb_q(dc.cfg, dc.q_c, dc.w_uk, dc.q_abs, spec.n_tok)
-    torch.cuda.synchronize()
-    want = O.absorb_q(O.bf16_to_f64(spec.q_c()), O.bf16_to_f64(spec.w_uk()))
-    assert_close(_f64(dc.q_abs), want, "q_abs")
+# Head shapes for the projections: the DeepSeek-V2 shape, and shapes that take
+# the other tiling branches (d_h = 64 or 192 for absorb_q's contraction, two
+# 128-feature tiles for up_v) or fall back to the CUDA-core kernels.
+PROJ_SHAPES = {
+    "v2": dict(n_h=128, d_c=512, d_h=128),
+    "small": dict(n_h=12, d_c=128, d_h=64),
+    "wide": dict(n_h=6, d_c=256, d_h=192),
+    "tall": dict(n_h=5, d_c=192, d_h=256),
+}
+# token counts: one token, below one 16-row MMA step, the V2 decode batch, and
+# more than one token tile with a ragged last tile
+PROJ_TOKENS = [1, 15, 32, 300]
+_proj_inputs = {}
 
 
-def test_up_v_parity(M):
-    from mla_latent_kv_38_b200 import synth
-    spec = CaseSpec(**V2, seq_lens=np.array([64] * 9, np.int32), seed=8)
-    dc = _dc(spec, fill_history=False)
-    lat_bits = synth.normal_bf16(8, 99, (spec.n_tok, spec.n_h, spec.d_c), std=0.05)
-    lat = torch.from_numpy(lat_bits.view(np.int16)).cuda().view(torch.bfloat16)
-    M.mla_up_v(dc.cfg, lat, dc.w_uv, dc.out, spec.n_tok)
+def _proj_case(shape, n_tok):
+    key = (shape, n_tok)
+    if key not in _proj_inputs:
+        from mla_latent_kv_38_b200 import synth
+        d = PROJ_SHAPES[shape]
+        n_h, d_c, d_h = d["n_h"], d["d_c"], d["d_h"]
+        seed = 11 + n_tok
+        q_c = synth.normal_bf16(seed, 1, (n_tok, n_h, d_h))
+        lat = synth.normal_bf16(seed, 2, (n_tok, n_h, d_c), std=0.05)
+        w_uk = synth.normal_bf16(seed, 3, (n_h, d_h, d_c), std=synth.weight_std(d_c))
+        w_uv = synth.normal_bf16(seed, 4, (n_h, d_h, d_c), std=synth.weight_std(d_c))
+        want_q = O.absorb_q(O.bf16_to_f64(q_c), O.bf16_to_f64(w_uk))
+        want_o = O.up_v(O.bf16_to_f64(lat), O.bf16_to_f64(w_uv))
+        _proj_inputs[key] = (q_c, lat, w_uk, w_uv, want_q, want_o)
+    return _proj_inputs[key]
+
+
+def _dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("impl", [0, 1])
+@pytest.mark.parametrize("n_tok", PROJ_TOKENS)
+@pytest.mark.parametrize("shape", sorted(PROJ_SHAPES))
+def test_projection_parity(M, shape, n_tok, impl):
+    d = PROJ_SHAPES[shape]
+    q_c, lat, w_uk, w_uv, want_q, want_o = _proj_case(shape, n_tok)
+    cfg = M.MlaConfig(d["n_h"], d["d_c"], d["d_h"], 16, 64, 0.0, impl)
+    q_abs = torch.full((n_tok, d["n_h"], d["d_c"]), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = torch.full((n_tok, d["n_h"], d["d_h"]), float("nan"), dtype=torch.bfloat16, device="cuda")
+    M.mla_absorb_q(cfg, _dev(q_c), _dev(w_uk), q_abs, n_tok)
+    M.mla_up_v(cfg, _dev(lat), _dev(w_uv), out, n_tok)
     torch.cuda.synchronize()
-    want = O.up_v(O.bf16_to_f64(lat_bits), O.bf16_to_f64(spec.w_uv()))
-    assert_close(_f64(dc.out), want, "up_v")
+    assert_close(_f64(q_abs), want_q, f"q_abs {shape} n_tok={n_tok}")
+    assert_close(_f64(out), want_o, f"up_v {shape} n_tok={n_tok}")
+
+
+def test_projection_tcgen05_shapes(M):
+    """impl = 2 forces the tensor-core projections and rejects shapes they do
+    not tile; the shapes they do tile match the CUDA-core kernels' results."""
+    for shape, absorb_ok, up_v_ok in [("v2", True, True), ("small", True, False),
+                                      ("wide", True, False), ("tall", False, True)]:
+        d = PROJ_SHAPES[shape]
+        q_c, lat, w_uk, w_uv, want_q, want_o = _proj_case(shape, 32)
+        cfg = M.MlaConfig(d["n_h"], d["d_c"], d["d_h"], 16, 64, 0.0, M.IMPL_TCGEN05)
+        q_abs = torch.empty((32, d["n_h"], d["d_c"]), dtype=torch.bfloat16, device="cuda")
+        out = torch.empty((32, d["n_h"], d["d_h"]), dtype=torch.bfloat16, device="cuda")
+        if absorb_ok:
+            M.mla_absorb_q(cfg, _dev(q_c), _dev(w_uk), q_abs, 32)
+            torch.cuda.synchronize()
+            assert_close(_f64(q_abs), want_q, f"q_abs {shape} tcgen05")
+        else:
+            with pytest.raises(M.MlaError) as e:
+                M.mla_absorb_q(cfg, _dev(q_c), _dev(w_uk), q_abs, 32)
+            assert e.value.code == -2, shape
+        if up_v_ok:
+            M.mla_up_v(cfg, _dev(lat), _dev(w_uv), out, 32)
+            torch.cuda.synchronize()
+            assert_close(_f64(out), want_o, f"up_v {shape} tcgen05")
+        else:
+            with pytest.raises(M.MlaError) as e:
+                M.mla_up_v(cfg, _dev(lat), _dev(w_uv), out, 32)
+            assert e.value.code == -2, shape
 
 
 def test_device_checks_flag_bad_rows(M):
