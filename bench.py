@@ -63,6 +63,34 @@ def dist_env():
     return world, rank, local
 
 
+class Ranks:
+    """Barrier and max-over-ranks on the process group (pg None: one process).
+
+    Every rank calls the same methods in the same order; the reduction runs
+    on `device` (the rank's GPU under NCCL, the CPU under gloo)."""
+
+    def __init__(self, pg, device):
+        self.pg, self.device = pg, device
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if self.pg is None:
+            return float(x)
+        import torch
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+
+def aggregate_rate(world: int, units_per_step_per_rank: int, steps: int, max_ms: float) -> float:
+    """Whole-job units per second: every rank processes its own copy of the
+    workload, and the job takes as long as its slowest rank."""
+    return world * units_per_step_per_rank * steps / (max_ms / 1e3)
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region (NVML polling thread)
 # ---------------------------------------------------------------------------
@@ -182,13 +210,16 @@ def run_reference(args):
 # our arm
 # ---------------------------------------------------------------------------
 
+DECODE_SOURCES = ("common.cuh", "sm100_decode.cu", "sm100_decode.h", "sm100_ptx.cuh", "tensor_map.h")
+
+
 def decode_source_hash():
+    """Hash of the sources the tcgen05 decode kernels are built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mla_latent_kv_38_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.startswith(("decode", "sm100")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+    for f in DECODE_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 
@@ -228,16 +259,8 @@ def run_ours(args):
     launches_decode = M.mla_decode_launches(dc.cfg, spec.B, spec.T_q, args.max_splits)
     launches_per_step = 3 + launches_decode       # absorb_q, rope_append, up_v + decode
 
-    def barrier():
-        if pg is not None:
-            pg.barrier()
-
-    def max_over_ranks(x):
-        if pg is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks(pg, dev)
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     # warm-up
     for _ in range(max(args.warmup, 3)):
@@ -281,7 +304,7 @@ def run_ours(args):
     }
     step_ms = max_over_ranks(step_ms)
     tokens_per_step = spec.n_tok
-    value = world * tokens_per_step * K / (step_ms / 1e3)
+    value = aggregate_rate(world, tokens_per_step, K, step_ms)
 
     # end to end through the public API with host buffers
     h_in = [torch.from_numpy(a.view(np.int16)).pin_memory() for a in
@@ -305,7 +328,7 @@ def run_ours(args):
         e1.synchronize()
         e2e_ms += e0.elapsed_time(e1)
     e2e_ms = max_over_ranks(e2e_ms)
-    e2e_value = world * tokens_per_step * K / (e2e_ms / 1e3)
+    e2e_value = aggregate_rate(world, tokens_per_step, K, e2e_ms)
 
     peaks, peak_src = load_peaks()
     bytes_alg = spec.algorithmic_bytes()

@@ -33,7 +33,9 @@ merge of split partials, an emulation of the GPU's float32 RoPE arithmetic for
 the bit-exact append check, and the per-token cache-size formulas of the
 "Сколько получилось" table.
 
-Readings where the pages are silent or garbled are listed in the design doc.
+Where the pages are silent or disagree, the functions below say which reading
+they take (score scale, shared RoPE key, half-split pairing, query positions,
+weight standard deviations).
 """
 
 from __future__ import annotations
