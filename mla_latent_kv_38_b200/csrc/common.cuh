@@ -59,6 +59,36 @@ __device__ __forceinline__ void raise_status(int32_t* st, int bits) {
     if (st != nullptr) atomicOr(st, bits);
 }
 
+// ---- programmatic dependent launch --------------------------------------
+// Kernels launched with launch_pdl() may be scheduled while the previous
+// kernel of the stream is still running.  Each of them lets its own successor
+// start early (griddep_launch_dependents) and executes griddep_wait() -- which
+// returns once the previous kernel has completed and its writes are visible --
+// before it reads or writes any buffer that an earlier kernel may touch, and
+// always before it exits, so that completion stays ordered along the stream.
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Parameters of one decode launch (shared by the SIMT and tcgen05 kernels).
 struct DecodeParams {
     const uint16_t* q_abs;      // (n_tok, n_h, d_c)

@@ -37,6 +37,8 @@ rope_append_kernel(uint16_t* __restrict__ q_r, const uint16_t* __restrict__ k_r,
                    const int32_t* __restrict__ block_table, int max_blocks,
                    uint16_t* __restrict__ pool, int num_blocks, int n_tok, int T_q,
                    int n_h, int d_c, int d_r, int block_size, int q_blocks, int32_t* status) {
+    griddep_launch_dependents();
+    griddep_wait();   // q_r, the pool and the status word may be in use by earlier kernels
     const int h = d_r >> 1;
     if (static_cast<int>(blockIdx.x) < q_blocks) {
         // ---- query RoPE, in place
@@ -112,10 +114,9 @@ cudaError_t launch_rope_append(uint16_t* q_r, const uint16_t* k_r, const uint16_
     const long q_blocks = (q_threads + threads - 1) / threads;
     const long a_blocks = (n_tok + warps - 1) / warps;
     if (q_blocks + a_blocks > 0x7fffffffL) return cudaErrorInvalidValue;
-    rope_append_kernel<<<static_cast<unsigned>(q_blocks + a_blocks), threads, 0, stream>>>(
-        q_r, k_r, c_kv, positions, table, max_pos, block_table, max_blocks, pool, num_blocks, n_tok, T_q, n_h, d_c,
-        d_r, block_size, static_cast<int>(q_blocks), status);
-    return cudaGetLastError();
+    return launch_pdl(rope_append_kernel, dim3(static_cast<unsigned>(q_blocks + a_blocks)), dim3(threads), 0, stream,
+                      q_r, k_r, c_kv, positions, table, max_pos, block_table, max_blocks, pool, num_blocks, n_tok,
+                      T_q, n_h, d_c, d_r, block_size, static_cast<int>(q_blocks), status);
 }
 
 }  // namespace mla

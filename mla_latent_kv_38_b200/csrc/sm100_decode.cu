@@ -78,9 +78,9 @@ enum {
     BAR_VR_EMPTY = BAR_VR_FULL + kVRing,
     BAR_S_FULL = BAR_VR_EMPTY + kVRing,      // + S buffer
     BAR_S_FREE = BAR_S_FULL + 2,             // + S buffer (leader, 8 warps)
-    BAR_P_FULL = BAR_S_FREE + 2,             // leader, 8 warps
-    BAR_P_FREE = BAR_P_FULL + 1,             // each CTA, MMA commit
-    BAR_TAIL_READY = BAR_P_FREE + 1,         // each CTA, MMA thread arrives remotely
+    BAR_P_FULL = BAR_S_FREE + 2,             // + P half (leader, 2 warps x 2 CTAs)
+    BAR_P_FREE = BAR_P_FULL + 2,             // + P half (each CTA, MMA commit)
+    BAR_TAIL_READY = BAR_P_FREE + 2,         // each CTA, MMA thread arrives remotely
     BAR_TAIL_DONE = BAR_TAIL_READY + 1,      // leader, 8 warps
     BAR_DRAIN = BAR_TAIL_DONE + 1,           // S issuer's own drain on abort
     BAR_DRAIN_PV = BAR_DRAIN + 1,            // P.V issuer's
@@ -96,6 +96,7 @@ constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 256, 0, 0);
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 256, 0, 1);
 
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kSchedSmemUnits = 8192;             // units whose prefix the schedule keeps in shared memory
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
 
 struct Sm100Params {
@@ -196,6 +197,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     auto bar = [&](int i) { return sbase + kOffBar + 8u * static_cast<uint32_t>(i); };
     auto leader_bar = [&](int i) { return ptx::map_to_rank(bar(i), 0); };
 
+    griddep_launch_dependents();
     if (threadIdx.x == 0) {
         ptx::mbar_init(bar(BAR_Q_FULL), 1);
         ptx::mbar_init(bar(BAR_Q_EMPTY), 1);
@@ -211,8 +213,10 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             ptx::mbar_init(bar(BAR_S_FULL + b), 1);
             ptx::mbar_init(bar(BAR_S_FREE + b), 8);   // 4 softmax warps x 2 CTAs
         }
-        ptx::mbar_init(bar(BAR_P_FULL), 8);
-        ptx::mbar_init(bar(BAR_P_FREE), 1);
+        for (int hf = 0; hf < 2; ++hf) {
+            ptx::mbar_init(bar(BAR_P_FULL + hf), 4);
+            ptx::mbar_init(bar(BAR_P_FREE + hf), 1);
+        }
         ptx::mbar_init(bar(BAR_TAIL_READY), 1);
         ptx::mbar_init(bar(BAR_TAIL_DONE), 8);
         ptx::mbar_init(bar(BAR_DRAIN), 1);
@@ -234,6 +238,9 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     ptx::cluster_sync();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // everything below reads what the schedule kernel (and the kernels before
+    // it: q_abs, q^R, the appended cache rows) wrote
+    griddep_wait();
 
     // this cluster's contiguous range of global pages [g0, g1) and the unit of
     // page g0, precomputed by the schedule kernel (empty range: no work)
@@ -243,10 +250,15 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     // Two load streams, each consumed in order by one MMA issuer:
     //   S ring: S(i) = 9 entries (column chunk c of this CTA's pages 2r, 2r+1)
     //   V ring: V(i) = 2 entries per page (latent chunks owned for P.V h = 0, 1)
-    auto page_row = [&](const Tile& t, int pg) -> int {
-        // cache row of page pg (0..3) of tile t; invalid entries are flagged and clamped
-        const int b = p.unit_meta[t.u].w;
-        int blk = p.block_table[static_cast<size_t>(b) * p.max_blocks + t.page0 + pg];
+    // Block-table entries are plain global loads.  Each producer issues them a
+    // tile or two before it needs them, so that their latency overlaps the
+    // ring waits of the tiles in between; an entry is validated where it is
+    // used (out-of-range entries are flagged and read as block 0).
+    auto load_blk = [&](const Tile& t, int pg) -> int {
+        const int b = t.u / (p.n_hb * p.T_q);
+        return p.block_table[static_cast<size_t>(b) * p.max_blocks + t.page0 + pg];
+    };
+    auto blk_row = [&](int blk) -> int {
         if (blk < 0 || blk >= p.num_blocks) {
             raise_status(p.status, MLA_STATUS_BAD_BLOCK);
             blk = 0;
@@ -257,24 +269,34 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     if (warp == 0) {
         // ------------------------------------------------------------ S stream (and Q)
         // Lanes 0 and 1 each wait for the entry's slot and issue one box (lane 0
-        // of the leader CTA arms the full barrier with both CTAs' bytes).
+        // of the leader CTA arms the full barrier with both CTAs' bytes).  Lane
+        // l < 2 owns this CTA's page 2r + l of every tile: its block for tiles
+        // i, i+1, i+2 sits in b0, b1, b2 while tile i is issued, and tile i+2's
+        // pages are pulled into L2 (the peer's P.V reads hit the same lines).
         const uint64_t pol_q = ptx::l2_policy_evict_last();
-        TileWalker w, wp;
+        const int my_pg = 2 * static_cast<int>(rank) + (lane & 1);
+        TileWalker w, wa;
         w.init(p.prefix, u0, g0, g1);
-        wp.init(p.prefix, u0, g0, g1);
-        if (!wp.done()) wp.next();   // the look-ahead walker runs one tile ahead
+        wa.init(p.prefix, u0, g0, g1);
+        int b0 = 0, b1 = 0, b2 = 0;
+        bool h0 = false, h1 = false, h2 = false;
+        auto look = [&](int& b, bool& h) {
+            h = false;
+            if (!wa.done()) {
+                const Tile t = wa.next();
+                h = lane < 2 && my_pg < t.np;
+                if (h) b = load_blk(t, my_pg);
+            }
+        };
+        look(b0, h0);
+        look(b1, h1);
+        look(b2, h2);
+        if (h0) ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(blk_row(b0)) * kRow, kPage * kRow * 2);
+        if (h1) ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(blk_row(b1)) * kRow, kPage * kRow * 2);
         int e = 0, uc = 0;
         bool ok = g0 < g1;
         while (ok && !w.done()) {
             const Tile cur = w.next();
-            if (!wp.done()) {
-                // Pull the next tile's pages (this CTA's S pages 2r, 2r+1; the peer's
-                // P.V operand reads hit the same lines) into L2 a tile ahead.
-                const Tile nt = wp.next();
-                const int pg = 2 * static_cast<int>(rank) + (lane & 1);
-                if (lane < 2 && pg < nt.np)
-                    ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(page_row(nt, pg)) * kRow, kPage * kRow * 2);
-            }
             if (cur.first) {
                 // new unit segment: load Q (this CTA's 64 heads) from 9 lanes
                 bool good = true;
@@ -291,9 +313,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 ++uc;
             }
             // S(cur): 9 column chunks of pages 2r, 2r+1
-            const int my_pg = 2 * static_cast<int>(rank) + (lane & 1);
-            const bool has = lane < 2 && my_pg < cur.np;
-            const int row = has ? page_row(cur, my_pg) : 0;
+            const int row = h0 ? blk_row(b0) : 0;
             const uint32_t tx = static_cast<uint32_t>(cur.np) * kBox;    // both CTAs together
             for (int c = 0; c < 9; ++c, ++e) {
                 const int slot = e % kSRing;
@@ -301,24 +321,40 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 if (lane < 2) {
                     good = wait_bar(bar(BAR_SR_EMPTY + slot), ((e / kSRing) & 1) ^ 1, abort_flag, p.status);
                     if (good && lane == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_SR_FULL + slot), tx);
-                    if (good && has)
+                    if (good && h0)
                         ptx::tma_load_2d_pair_normal(sbase + kOffSRing + slot * kEntry + (lane & 1) * kBox, &p.tm_pool,
                                                      64 * c, row, leader_bar(BAR_SR_FULL + slot));
                 }
                 if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
             }
+            if (h2) ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(blk_row(b2)) * kRow, kPage * kRow * 2);
+            b0 = b1; h0 = h1;
+            b1 = b2; h1 = h2;
+            look(b2, h2);
         }
     } else if (warp == 7) {
         // ------------------------------------------------------------ V stream
+        // Lane pg < 4 holds the block of page pg of the current tile (v0) and of
+        // the next one (v1).
         const uint64_t pol_v = ptx::l2_policy_evict_first();   // last use of these lines
-        TileWalker w;
+        TileWalker w, wa;
         w.init(p.prefix, u0, g0, g1);
+        wa.init(p.prefix, u0, g0, g1);
+        int v0 = 0, v1 = 0;
+        auto look = [&](int& v) {
+            if (!wa.done()) {
+                const Tile t = wa.next();
+                if (lane < t.np) v = load_blk(t, lane);
+            }
+        };
+        look(v0);
+        look(v1);
         int e = 0;
         bool ok = g0 < g1;
         while (ok && !w.done()) {
             const Tile cur = w.next();
             for (int pg = 0; pg < cur.np && ok; ++pg) {
-                const int row = page_row(cur, pg);
+                const int row = blk_row(__shfl_sync(0xffffffffu, v0, pg));
                 for (int h = 0; h < 2; ++h, ++e) {
                     const int slot = e % kVRing;
                     bool good = true;
@@ -333,6 +369,8 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                     if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
                 }
             }
+            v0 = v1;
+            look(v1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ S = Q K^T issuer
@@ -390,10 +428,17 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             while (ok && !w.done()) {
                 const Tile t = w.next();
                 const int kv_len = p.unit_meta[t.u].x;   // read before the wait hides its latency
-                if (!(ok = wait_bar(bar(BAR_P_FULL), i & 1, abort_flag, p.status))) break;
                 const bool tail = t.unit_end && (kv_len % kPage) != 0;
-                ptx::tc_fence_after();
-                for (int pg = 0; pg < t.np && ok; ++pg) {
+                // P is written in two halves: keys [0,128) (pages 0, 1) by the softmax
+                // warps of TMEM lanes 0-63, keys [128,256) by those of lanes 64-127;
+                // each half is released as soon as its pages' MMAs complete.
+                for (int pg = 0; pg < 4 && ok; ++pg) {
+                    if (pg == 0 || pg == 2) {
+                        if (pg == 2) ptx::mma_commit_pair(bar(BAR_P_FREE + 0), 0x3);
+                        if (!(ok = wait_bar(bar(BAR_P_FULL + (pg >> 1)), i & 1, abort_flag, p.status))) break;
+                        ptx::tc_fence_after();
+                    }
+                    if (pg >= t.np) continue;
                     if (tail && pg == t.np - 1) {
                         // the unit's last page holds rows past the end: once its two
                         // V entries have landed, the softmax warps of both CTAs zero
@@ -422,7 +467,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                     }
                 }
                 if (!ok) break;
-                ptx::mma_commit_pair(bar(BAR_P_FREE), 0x3);
+                ptx::mma_commit_pair(bar(BAR_P_FREE + 1), 0x3);
                 ++i;
             }
             if (!ok) {
@@ -441,15 +486,19 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
         float* xmax = reinterpret_cast<float*>(smem + kOffXmax);
         float* xsum = reinterpret_cast<float*>(smem + kOffXsum);
-        TileWalker w;
+        TileWalker w, wa;      // wa runs one tile ahead: the next tile's unit data is loaded early
         w.init(p.prefix, u0, g0, g1);
+        wa.init(p.prefix, u0, g0, g1);
+        int4 meta_nxt = make_int4(0, 0, 0, 0);
+        if (!wa.done()) meta_nxt = p.unit_meta[wa.next().u];
         int i = 0, tails = 0;
         int v_before = 0;      // V ring entries of tiles before i
         bool ok = true;
         float m_used = -INFINITY, l_part = 0.f;
         while (ok && !w.done()) {
             const Tile t = w.next();
-            const int4 meta = p.unit_meta[t.u];
+            const int4 meta = meta_nxt;
+            if (!wa.done()) meta_nxt = p.unit_meta[wa.next().u];
             // keys of this tile that belong to this segment
             const int key_end = min(meta.x, kPage * (t.page0 + t.np));
             if (t.first) {
@@ -500,8 +549,12 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             }
             l_part = l_part * alpha + ps;
 
-            // P.V of the previous tile must be complete: P buffer free, O stable
-            ok = wait_bar(bar(BAR_P_FREE), (i & 1) ^ 1, abort_flag, p.status);
+            // This half of the P buffer must be free (the previous tile's P.V MMAs on
+            // it complete); a rescale of O needs the whole previous P.V complete.
+            const int hf = hi ? 1 : 0;
+            ok = wait_bar(bar(BAR_P_FREE + hf), (i & 1) ^ 1, abort_flag, p.status);
+            if (ok && !hi && __any_sync(0xffffffffu, resc))
+                ok = wait_bar(bar(BAR_P_FREE + 1), (i & 1) ^ 1, abort_flag, p.status);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             ptx::tc_fence_after();
             if (resc) {
@@ -531,7 +584,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_P_FULL));
+            if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_P_FULL + hf));
 
             // V ring position of this tile's entries
             const int v_start = v_before;
@@ -561,7 +614,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
 
             if (t.last) {
                 // ---- epilogue of this unit segment: wait for P.V of this tile
-                ok = wait_bar(bar(BAR_P_FREE), i & 1, abort_flag, p.status);
+                ok = wait_bar(bar(BAR_P_FREE + 1), i & 1, abort_flag, p.status);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 ptx::tc_fence_after();
                 xsum[l] = l_part;
@@ -637,7 +690,11 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, 
                           int4* __restrict__ unit_meta, int4* __restrict__ cluster_info, int32_t* status) {
     __shared__ int warp_tot[32];
     __shared__ int carry;
+    __shared__ int pre_s[kSchedSmemUnits + 1];   // the prefix again, for the searches below
+    griddep_launch_dependents();
+    griddep_wait();   // the workspace may still be read by an earlier decode call's kernels
     const int U = B * T_q * n_hb;
+    const bool in_smem = U <= kSchedSmemUnits;
     if (threadIdx.x == 0) carry = 0;
     __syncthreads();
     for (int base = 0; base < U; base += 1024) {
@@ -677,17 +734,24 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, 
         }
         __syncthreads();
         const int incl = v + (w > 0 ? warp_tot[w - 1] : 0) + carry;
-        if (u < U) prefix[u + 1] = incl;
-        if (u == 0) prefix[0] = 0;
+        if (u < U) {
+            prefix[u + 1] = incl;
+            if (in_smem) pre_s[u + 1] = incl;
+        }
+        if (u == 0) {
+            prefix[0] = 0;
+            if (in_smem) pre_s[0] = 0;
+        }
         __syncthreads();
         if (threadIdx.x == 1023) carry = incl;
         __syncthreads();
     }
     __syncthreads();
+    const int* pf = in_smem ? pre_s : prefix;
     const long long T = carry;
     const long long Ce = T < C ? T : C;   // clusters that get work (all non-empty ranges)
     for (int u = threadIdx.x; u < U; u += 1024) {
-        const int a = prefix[u], e = prefix[u + 1];
+        const int a = pf[u], e = pf[u + 1];
         if (e > a) {
             // cluster c covers tiles [floor(c T / Ce), floor((c+1) T / Ce)); tile g
             // lies in cluster floor(((g + 1) Ce - 1) / T)
@@ -707,7 +771,7 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, 
             int lo = 0, hi = U - 1;   // last unit with prefix <= a
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
-                if (prefix[mid] <= a) lo = mid; else hi = mid - 1;
+                if (pf[mid] <= a) lo = mid; else hi = mid - 1;
             }
             ci = make_int4(a, e, lo, 0);
         }
@@ -721,6 +785,8 @@ __global__ void __launch_bounds__(128)
 mla_sm100_merge_kernel(const int4* __restrict__ unit_meta, const float* __restrict__ part_o,
                        const float* __restrict__ part_lse, uint16_t* __restrict__ out_latent,
                        float* __restrict__ out_lse, int n_h, int n_hb) {
+    griddep_launch_dependents();
+    griddep_wait();
     const int row = blockIdx.x, u = blockIdx.y;
     const int4 meta = unit_meta[u];
     const int bt = u / n_hb, hb = u - bt * n_hb;
@@ -832,22 +898,20 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int /*max_split
     k.max_blocks = P.max_blocks;
     k.scale_log2 = P.scale_log2;
 
-    mla_sm100_schedule_kernel<<<1, 1024, 0, stream>>>(P.seq_lens, P.B, P.T_q, n_hb, P.max_blocks, kClusters,
-                                                      reinterpret_cast<int32_t*>(base + w.prefix),
-                                                      reinterpret_cast<int4*>(base + w.meta),
-                                                      reinterpret_cast<int4*>(base + w.cinfo), P.status);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(mla_sm100_schedule_kernel, dim3(1), dim3(1024), 0, stream, P.seq_lens, P.B, P.T_q,
+                               n_hb, P.max_blocks, static_cast<int>(kClusters),
+                               reinterpret_cast<int32_t*>(base + w.prefix), reinterpret_cast<int4*>(base + w.meta),
+                               reinterpret_cast<int4*>(base + w.cinfo), P.status);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(mla_decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes));
     if (e != cudaSuccess) return e;
-    mla_decode_sm100_kernel<<<2 * kClusters, kThreads, kSmemBytes, stream>>>(k);
-    e = cudaGetLastError();
+    e = launch_pdl(mla_decode_sm100_kernel, dim3(2 * kClusters), dim3(kThreads), kSmemBytes, stream, k);
     if (e != cudaSuccess) return e;
     dim3 mgrid(128, U);
-    mla_sm100_merge_kernel<<<mgrid, 128, 0, stream>>>(k.unit_meta, k.part_o, k.part_lse, P.out_latent, P.out_lse,
-                                                      P.n_h, n_hb);
-    return cudaGetLastError();
+    return launch_pdl(mla_sm100_merge_kernel, mgrid, dim3(128), 0, stream, k.unit_meta,
+                      static_cast<const float*>(k.part_o), static_cast<const float*>(k.part_lse), P.out_latent,
+                      P.out_lse, P.n_h, n_hb);
 }
 
 }  // namespace mla

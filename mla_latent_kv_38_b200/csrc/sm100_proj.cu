@@ -80,6 +80,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_proj_sm100_kernel(const __gri
     const int m0 = blockIdx.x * kM;
     const int n_tiles = (p.n_tok + nt - 1) / nt;
 
+    griddep_launch_dependents();
     if (threadIdx.x == 0) {
         ptx::mbar_init(barA, 1);
         ptx::mbar_init(barB, 1);
@@ -103,6 +104,8 @@ __global__ void __launch_bounds__(kThreads, 1) mla_proj_sm100_kernel(const __gri
             ptx::tma_load_2d(sB + kc * b_box, &p.tm_b, head * K + 64 * kc, t * nt, barB);
     };
 
+    // The weights are read-only inputs no kernel writes: fetch them while the
+    // previous kernel finishes, then wait for it before touching activations.
     if (threadIdx.x == 0) {
         ptx::mbar_arrive_expect_tx(barA, a_bytes);
         if (kAbsorb) {
@@ -114,8 +117,9 @@ __global__ void __launch_bounds__(kThreads, 1) mla_proj_sm100_kernel(const __gri
             for (int kc = 0; kc < kchunks; ++kc)
                 ptx::tma_load_2d(sA + kc * (kM * 128), &p.tm_a, 64 * kc, head * p.d_h + m0, barA);
         }
-        load_b(0);
     }
+    griddep_wait();
+    if (threadIdx.x == 0) load_b(0);
 
     const int row = m0 + threadIdx.x;   // this thread's output feature (TMEM lane)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
@@ -193,8 +197,7 @@ cudaError_t launch_proj(ProjParams& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     p.idesc = ptx::idesc_bf16_f32(kM, p.nt, kAbsorb ? 1 : 0, 0);
     dim3 grid(p.m_total / kM, p.n_h);
-    mla_proj_sm100_kernel<kAbsorb><<<grid, kThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(mla_proj_sm100_kernel<kAbsorb>, grid, dim3(kThreads), smem, stream, p);
 }
 
 }  // namespace
