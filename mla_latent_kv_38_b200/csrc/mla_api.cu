@@ -4,6 +4,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100_decode.h"
@@ -82,11 +84,17 @@ const char* mla_status_str(int code) {
 }
 
 int mla_check_device(void) {
+    // answer cached per device: 0 unknown, 1 sm_100, 2 other
+    static std::atomic<int> known[64];
     int dev = 0, major = 0, minor = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_UNSUPPORTED;
+    const int k = dev >= 0 && dev < 64 ? known[dev].load(std::memory_order_relaxed) : 0;
+    if (k != 0) return k == 1 ? MLA_OK : MLA_ERR_UNSUPPORTED;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MLA_ERR_UNSUPPORTED;
     if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return MLA_ERR_UNSUPPORTED;
-    return (major == 10 && minor == 0) ? MLA_OK : MLA_ERR_UNSUPPORTED;
+    const bool ok = major == 10 && minor == 0;
+    if (dev >= 0 && dev < 64) known[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
+    return ok ? MLA_OK : MLA_ERR_UNSUPPORTED;
 }
 
 int mla_rope_table(int d_r, double base, int max_pos, float* host_table) {

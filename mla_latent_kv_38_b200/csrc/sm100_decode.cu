@@ -52,16 +52,17 @@ constexpr int kDc = 512, kDr = 64, kRow = 576;    // row = c^KV || k^R
 constexpr int kPage = 64;                         // cache rows per page (TMA box height)
 constexpr int kTilePages = 4;                     // a tile = 4 pages = 256 keys (MMA N)
 constexpr int kSRing = 3;                         // 16 KB entries, S operand stream
-constexpr int kVRing = 4;                         // 16 KB entries, P.V operand stream
+constexpr int kVRing = 2;                         // 32 KB entries (one page), P.V operand stream
 
 constexpr uint32_t kBox = 8192;                   // one page x 64 columns (128 B rows)
-constexpr uint32_t kEntry = 2 * kBox;             // ring entry: 2 boxes
+constexpr uint32_t kEntry = 2 * kBox;             // S ring entry: 2 boxes
+constexpr uint32_t kVEntry = 4 * kBox;            // V ring entry: 4 latent chunks of one page
 constexpr uint32_t kQBytes = 9 * kBox;            // 64 heads x 576 columns
 constexpr uint32_t kPBytes = 4 * kBox;            // 64 heads x 256 keys (4 blocks of 64 keys)
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffSRing = kOffQ + kQBytes;
 constexpr uint32_t kOffVRing = kOffSRing + kSRing * kEntry;
-constexpr uint32_t kOffP = kOffVRing + kVRing * kEntry;
+constexpr uint32_t kOffP = kOffVRing + kVRing * kVEntry;
 constexpr uint32_t kOffXmax = kOffP + kPBytes;    // 2 x 128 floats
 constexpr uint32_t kOffXsum = kOffXmax + 1024;    // 128 floats
 constexpr uint32_t kOffBar = kOffXsum + 512;
@@ -101,7 +102,7 @@ constexpr float kRescaleThreshold = 8.0f;         // log2 units
 
 struct Sm100Params {
     CUtensorMap tm_pool;      // pool as [rows][576], box 64 cols x 64 rows
-    CUtensorMap tm_pool_v;    // pool as [chunk][rows][64], box 64 cols x 64 rows x 2 chunks
+    CUtensorMap tm_pool_v;    // pool as [chunk][rows][64], box 64 cols x 64 rows x 4 chunks
     CUtensorMap tm_qa;        // q_abs as [n_tok*n_h][512], box 64 x 64
     CUtensorMap tm_qr;        // q_r   as [n_tok*n_h][64],  box 64 x 64
     const uint16_t* pool;     // for L2 prefetches of whole pages
@@ -176,11 +177,10 @@ struct TileWalker {
     }
 };
 
-// latent column chunk (64 wide) that a CTA contributes to P.V instruction h:
-// N columns [0,128) come from CTA 0, [128,256) from CTA 1
-__device__ __forceinline__ int owned_chunk(uint32_t rank, int h, int i) {
-    return 4 * h + 2 * static_cast<int>(rank) + i;
-}
+// P.V operand split: CTA r supplies latent chunks 4r .. 4r+3 (columns
+// [256r, 256r+256)); instruction h (N = 256) takes chunks 4r+2h, 4r+2h+1 from
+// each CTA, so TMEM column 128h + j of lane half r holds latent column
+// 256r + 128h + j.
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
@@ -291,8 +291,8 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         look(b0, h0);
         look(b1, h1);
         look(b2, h2);
-        if (h0) ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(blk_row(b0)) * kRow, kPage * kRow * 2);
-        if (h1) ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(blk_row(b1)) * kRow, kPage * kRow * 2);
+        // (tile 0 is loaded at once; prefetching it too would only queue ahead of those loads)
+        bool first_tile = true;
         int e = 0, uc = 0;
         bool ok = g0 < g1;
         while (ok && !w.done()) {
@@ -327,7 +327,9 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 }
                 if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
             }
+            if (first_tile && h1) ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(blk_row(b1)) * kRow, kPage * kRow * 2);
             if (h2) ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(blk_row(b2)) * kRow, kPage * kRow * 2);
+            first_tile = false;
             b0 = b1; h0 = h1;
             b1 = b2; h1 = h2;
             look(b2, h2);
@@ -353,21 +355,19 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         bool ok = g0 < g1;
         while (ok && !w.done()) {
             const Tile cur = w.next();
-            for (int pg = 0; pg < cur.np && ok; ++pg) {
+            for (int pg = 0; pg < cur.np && ok; ++pg, ++e) {
                 const int row = blk_row(__shfl_sync(0xffffffffu, v0, pg));
-                for (int h = 0; h < 2; ++h, ++e) {
-                    const int slot = e % kVRing;
-                    bool good = true;
-                    if (lane == 0) {
-                        good = wait_bar(bar(BAR_VR_EMPTY + slot), ((e / kVRing) & 1) ^ 1, abort_flag, p.status);
-                        if (good && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_VR_FULL + slot), 2 * kEntry);
-                        // both latent chunks of the page in one box: [chunk][row][64 columns]
-                        if (good)
-                            ptx::tma_load_3d_pair(sbase + kOffVRing + slot * kEntry, &p.tm_pool_v, 0, row,
-                                                  owned_chunk(rank, h, 0), leader_bar(BAR_VR_FULL + slot), pol_v);
-                    }
-                    if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
+                const int slot = e % kVRing;
+                bool good = true;
+                if (lane == 0) {
+                    good = wait_bar(bar(BAR_VR_EMPTY + slot), ((e / kVRing) & 1) ^ 1, abort_flag, p.status);
+                    if (good && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_VR_FULL + slot), 2 * kVEntry);
+                    // this CTA's 4 latent chunks of the page in one box: [chunk][row][64 columns]
+                    if (good)
+                        ptx::tma_load_3d_pair(sbase + kOffVRing + slot * kVEntry, &p.tm_pool_v, 0, row,
+                                              4 * static_cast<int>(rank), leader_bar(BAR_VR_FULL + slot), pol_v);
                 }
+                if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
             }
             v0 = v1;
             look(v1);
@@ -440,22 +440,21 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                     }
                     if (pg >= t.np) continue;
                     if (tail && pg == t.np - 1) {
-                        // the unit's last page holds rows past the end: once its two
-                        // V entries have landed, the softmax warps of both CTAs zero
-                        // those rows (entries are consumed in ring order, so the
-                        // earlier pages' slots are already free for these loads)
-                        if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status) &&
-                                   wait_bar(bar(BAR_VR_FULL + (e + 1) % kVRing), ((e + 1) / kVRing) & 1, abort_flag,
-                                            p.status)))
+                        // the unit's last page holds rows past the end: once its V
+                        // entry has landed, the softmax warps of both CTAs zero those
+                        // rows (entries are consumed in ring order, so the earlier
+                        // pages' slots are already free for this load)
+                        if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status)))
                             break;
                         ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 0));
                         ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 1));
                         if (!(ok = wait_bar(bar(BAR_TAIL_DONE), tails & 1, abort_flag, p.status))) break;
                         ++tails;
                     }
-                    for (int h = 0; h < 2; ++h, ++e) {
-                        if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status))) break;
-                        const uint64_t b0 = ptx::smem_desc_sw128(sbase + kOffVRing + (e % kVRing) * kEntry, kBox, 1024);
+                    if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status))) break;
+                    for (int h = 0; h < 2; ++h) {
+                        const uint64_t b0 =
+                            ptx::smem_desc_sw128(sbase + kOffVRing + (e % kVRing) * kVEntry + h * 2 * kBox, kBox, 1024);
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint64_t a = a0 + static_cast<uint64_t>((pg * kBox + 32 * kk) >> 4);
@@ -463,8 +462,9 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                             ptx::mma_pair_ss(tmem_base + kTmemO + 128 * h, a, bd, kIdescPV,
                                              (t.first && pg == 0 && kk == 0) ? 0u : 1u);
                         }
-                        ptx::mma_commit_pair(bar(BAR_VR_EMPTY + e % kVRing), 0x3);
                     }
+                    ptx::mma_commit_pair(bar(BAR_VR_EMPTY + e % kVRing), 0x3);
+                    ++e;
                 }
                 if (!ok) break;
                 ptx::mma_commit_pair(bar(BAR_P_FREE + 1), 0x3);
@@ -588,24 +588,21 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
 
             // V ring position of this tile's entries
             const int v_start = v_before;
-            v_before += 2 * t.np;
+            v_before += t.np;
             if (t.unit_end && (meta.x % kPage) != 0) {
-                // zero rows past the end in this CTA's two V entries of the last page
+                // zero rows past the end in this CTA's V entry of the last page (4 chunks)
                 ok = wait_bar(bar(BAR_TAIL_READY), tails & 1, abort_flag, p.status);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 ++tails;
                 const int valid = meta.x - kPage * (t.page0 + t.np - 1);
                 const int bad = kPage - valid;
-                const int et = v_start + 2 * (t.np - 1);
-                for (int x = l; x < 2 * 2 * bad * 8; x += 128) {
-                    const int ent = x / (2 * bad * 8);
-                    const int rem = x - ent * 2 * bad * 8;
-                    const int half = rem / (bad * 8);
-                    const int rem2 = rem - half * bad * 8;
-                    const int row = valid + (rem2 >> 3), ch = rem2 & 7;
-                    uint4* dst = reinterpret_cast<uint4*>(smem + kOffVRing + ((et + ent) % kVRing) * kEntry +
-                                                          half * kBox + row * 128) + ch;
-                    *dst = make_uint4(0, 0, 0, 0);
+                const int et = v_start + (t.np - 1);
+                unsigned char* ent = smem + kOffVRing + (et % kVRing) * kVEntry;
+                for (int x = l; x < 4 * bad * 8; x += 128) {
+                    const int chunk = x / (bad * 8);
+                    const int rem = x - chunk * bad * 8;
+                    const int row = valid + (rem >> 3), ch = rem & 7;
+                    reinterpret_cast<uint4*>(ent + chunk * kBox + row * 128)[ch] = make_uint4(0, 0, 0, 0);
                 }
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
@@ -629,7 +626,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 const size_t slot = static_cast<size_t>(cluster) + t.u;
 #pragma unroll 1
                 for (int h = 0; h < 2; ++h) {
-                    const int col0 = 256 * h + (hi ? 128 : 0);
+                    const int col0 = 128 * h + (hi ? 256 : 0);
 #pragma unroll 1
                     for (int q = 0; q < 4; ++q) {
                         uint32_t o[32];
@@ -830,7 +827,7 @@ bool make_map_chunks(CUtensorMap* m, const void* base, uint64_t rows) {
     if (fn == nullptr) return false;
     const cuuint64_t dims[3] = {64, rows, 9};
     const cuuint64_t strides[2] = {kRow * 2, 128};
-    const cuuint32_t box[3] = {64, 64, 2};
+    const cuuint32_t box[3] = {64, 64, 4};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -903,8 +900,8 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int /*max_split
                                reinterpret_cast<int32_t*>(base + w.prefix), reinterpret_cast<int4*>(base + w.meta),
                                reinterpret_cast<int4*>(base + w.cinfo), P.status);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(mla_decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes));
+    static std::atomic<uint64_t> smem_set{0};
+    e = allow_smem_once(mla_decode_sm100_kernel, static_cast<int>(kSmemBytes), smem_set);
     if (e != cudaSuccess) return e;
     e = launch_pdl(mla_decode_sm100_kernel, dim3(2 * kClusters), dim3(kThreads), kSmemBytes, stream, k);
     if (e != cudaSuccess) return e;

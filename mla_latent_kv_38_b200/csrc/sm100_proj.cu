@@ -37,6 +37,7 @@ constexpr int kM = 128;                       // output features per CTA
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr size_t kSmemLimit = 200 * 1024;     // A + B tiles per CTA
 constexpr size_t kSmemPerSm = 233472;         // shared memory of one SM (228 KB)
+constexpr size_t kSmemAttr = kSmemLimit + 4096;   // dynamic shared-memory limit set on the kernel (>= every launch)
 
 struct ProjParams {
     CUtensorMap tm_a;   // weights, [n_h * d_h][d_c], 64-column boxes
@@ -192,8 +193,8 @@ cudaError_t launch_proj(ProjParams& p, cudaStream_t stream) {
     const size_t max_ctas = 512 / p.tmem_cols;
     const size_t min_smem = kSmemPerSm / (max_ctas + 1) - 1024 + 16;
     if (max_ctas < 16 && smem < min_smem) smem = min_smem;
-    cudaError_t e = cudaFuncSetAttribute(mla_proj_sm100_kernel<kAbsorb>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    static std::atomic<uint64_t> smem_set{0};
+    cudaError_t e = allow_smem_once(mla_proj_sm100_kernel<kAbsorb>, static_cast<int>(kSmemAttr), smem_set);
     if (e != cudaSuccess) return e;
     p.idesc = ptx::idesc_bf16_f32(kM, p.nt, kAbsorb ? 1 : 0, 0);
     dim3 grid(p.m_total / kM, p.n_h);
