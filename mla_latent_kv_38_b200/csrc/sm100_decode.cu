@@ -67,7 +67,9 @@ constexpr uint32_t kOffXmax = kOffP + kPBytes;    // 2 x 128 floats
 constexpr uint32_t kOffXsum = kOffXmax + 1024;    // 128 floats
 constexpr uint32_t kOffBar = kOffXsum + 512;
 constexpr uint32_t kOffMisc = kOffBar + 8 * 32;   // tmem base, abort flag
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
+constexpr int kPrefixCache = 1024;                // units of a cluster's range kept in shared memory
+constexpr uint32_t kOffPrefix = kOffMisc + 16;
+constexpr uint32_t kSmemBytes = kOffPrefix + 4 * kPrefixCache + 1024;   // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 enum {
@@ -109,7 +111,7 @@ struct Sm100Params {
     const int32_t* block_table;
     const int32_t* prefix;    // (U + 1) exclusive prefix of pages per unit
     const int4* unit_meta;    // (U) {kv_len, first cluster, parts, batch index}
-    const int4* cluster_info; // (C) {first page, end page, first unit, -}
+    const int4* cluster_info; // (C) {first page, end page, first unit, last unit}
     uint16_t* out_latent;
     float* out_lse;
     float* part_o;            // (C + U) slots x 128 rows x 512
@@ -149,21 +151,25 @@ struct Tile {
 };
 
 // Walks a cluster's pages [g0, g1) as tiles.
+// The prefix entry of unit u is pf[u - off] (pf: a shared-memory copy of the
+// cluster's range, or the global array with off = 0).
 struct TileWalker {
-    const int32_t* prefix;
-    int g, g0, g1, u;
-    __device__ void init(const int32_t* pf, int u0, int g0_, int g1_) {
-        prefix = pf;
+    const int32_t* pf;
+    int off, g, g0, g1, u;
+    __device__ int prefix(int v) const { return pf[v - off]; }
+    __device__ void init(const int32_t* pf_, int off_, int u0, int g0_, int g1_) {
+        pf = pf_;
+        off = off_;
         g = g0_;
         g0 = g0_;
         g1 = g1_;
         u = u0;
-        while (g < g1 && prefix[u + 1] <= g) ++u;
+        while (g < g1 && prefix(u + 1) <= g) ++u;
     }
     __device__ bool done() const { return g >= g1; }
     __device__ Tile next() {
         Tile t;
-        const int ubeg = prefix[u], uend = prefix[u + 1];
+        const int ubeg = prefix(u), uend = prefix(u + 1);
         t.u = u;
         t.page0 = g - ubeg;
         t.first = (g == g0) || (g == ubeg);
@@ -172,7 +178,7 @@ struct TileWalker {
         t.last = g + t.np == seg_end;
         t.unit_end = g + t.np == uend;
         g += t.np;
-        while (g < g1 && prefix[u + 1] <= g) ++u;
+        while (g < g1 && prefix(u + 1) <= g) ++u;
         return t;
     }
 };
@@ -246,6 +252,15 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     // page g0, precomputed by the schedule kernel (empty range: no work)
     const int4 cinfo = p.cluster_info[cluster];
     const int g0 = cinfo.x, g1 = cinfo.y, u0 = cinfo.z;
+    // the page prefix of units u0 .. cinfo.w (+1), read by every role's tile walker
+    const int n_pre = cinfo.w - u0 + 2;
+    int32_t* pre_s = reinterpret_cast<int32_t*>(smem + kOffPrefix);
+    const bool pre_in_smem = g0 < g1 && n_pre <= kPrefixCache;
+    if (pre_in_smem)
+        for (int k = threadIdx.x; k < n_pre; k += kThreads) pre_s[k] = p.prefix[u0 + k];
+    __syncthreads();
+    const int32_t* pf_base = pre_in_smem ? pre_s : p.prefix;
+    const int pf_off = pre_in_smem ? u0 : 0;
 
     // Two load streams, each consumed in order by one MMA issuer:
     //   S ring: S(i) = 9 entries (column chunk c of this CTA's pages 2r, 2r+1)
@@ -271,28 +286,29 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // Lanes 0 and 1 each wait for the entry's slot and issue one box (lane 0
         // of the leader CTA arms the full barrier with both CTAs' bytes).  Lane
         // l < 2 owns this CTA's page 2r + l of every tile: its block for tiles
-        // i, i+1, i+2 sits in b0, b1, b2 while tile i is issued, and tile i+2's
-        // pages are pulled into L2 (the peer's P.V reads hit the same lines).
+        // i, i+1, i+2 sits in b0, b1, b2 while tile i is issued.  (An L2
+        // prefetch of the pages ahead measured slower: the bulk prefetch holds
+        // this warp for about a microsecond per tile.)
         const uint64_t pol_q = ptx::l2_policy_evict_last();
         const int my_pg = 2 * static_cast<int>(rank) + (lane & 1);
         TileWalker w, wa;
-        w.init(p.prefix, u0, g0, g1);
-        wa.init(p.prefix, u0, g0, g1);
+        w.init(pf_base, pf_off, u0, g0, g1);
+        wa.init(pf_base, pf_off, u0, g0, g1);
         int b0 = 0, b1 = 0, b2 = 0;
         bool h0 = false, h1 = false, h2 = false;
+        // (the loads are unconditional, to a valid entry, so that nothing waits
+        // for them until their value is used a tile or two later)
         auto look = [&](int& b, bool& h) {
             h = false;
             if (!wa.done()) {
                 const Tile t = wa.next();
                 h = lane < 2 && my_pg < t.np;
-                if (h) b = load_blk(t, my_pg);
+                b = load_blk(t, min(my_pg, t.np - 1));
             }
         };
         look(b0, h0);
         look(b1, h1);
         look(b2, h2);
-        // (tile 0 is loaded at once; prefetching it too would only queue ahead of those loads)
-        bool first_tile = true;
         int e = 0, uc = 0;
         bool ok = g0 < g1;
         while (ok && !w.done()) {
@@ -327,9 +343,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 }
                 if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
             }
-            if (first_tile && h1) ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(blk_row(b1)) * kRow, kPage * kRow * 2);
-            if (h2) ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(blk_row(b2)) * kRow, kPage * kRow * 2);
-            first_tile = false;
             b0 = b1; h0 = h1;
             b1 = b2; h1 = h2;
             look(b2, h2);
@@ -340,13 +353,13 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // the next one (v1).
         const uint64_t pol_v = ptx::l2_policy_evict_first();   // last use of these lines
         TileWalker w, wa;
-        w.init(p.prefix, u0, g0, g1);
-        wa.init(p.prefix, u0, g0, g1);
+        w.init(pf_base, pf_off, u0, g0, g1);
+        wa.init(pf_base, pf_off, u0, g0, g1);
         int v0 = 0, v1 = 0;
         auto look = [&](int& v) {
             if (!wa.done()) {
                 const Tile t = wa.next();
-                if (lane < t.np) v = load_blk(t, lane);
+                v = load_blk(t, min(lane, t.np - 1));
             }
         };
         look(v0);
@@ -377,7 +390,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // S(i) occupies entries 9 i .. 9 i + 8 of the S ring.
         if (rank == 0 && lane == 0 && g0 < g1) {
             TileWalker w;
-            w.init(p.prefix, u0, g0, g1);
+            w.init(pf_base, pf_off, u0, g0, g1);
             int i = 0, uc = 0;
             bool ok = true;
             const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffQ, 16, 1024);
@@ -421,7 +434,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // V(i) occupies the next 2 np entries of the V ring.
         if (rank == 0 && lane == 0 && g0 < g1) {
             TileWalker w;
-            w.init(p.prefix, u0, g0, g1);
+            w.init(pf_base, pf_off, u0, g0, g1);
             int i = 0, tails = 0, e = 0;
             bool ok = true;
             const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffP, 16, 1024);
@@ -487,10 +500,10 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         float* xmax = reinterpret_cast<float*>(smem + kOffXmax);
         float* xsum = reinterpret_cast<float*>(smem + kOffXsum);
         TileWalker w, wa;      // wa runs one tile ahead: the next tile's unit data is loaded early
-        w.init(p.prefix, u0, g0, g1);
-        wa.init(p.prefix, u0, g0, g1);
-        int4 meta_nxt = make_int4(0, 0, 0, 0);
-        if (!wa.done()) meta_nxt = p.unit_meta[wa.next().u];
+        w.init(pf_base, pf_off, u0, g0, g1);
+        wa.init(pf_base, pf_off, u0, g0, g1);
+        const int u_first = g0 < g1 ? wa.next().u : 0;
+        int4 meta_nxt = p.unit_meta[u_first];
         int i = 0, tails = 0;
         int v_before = 0;      // V ring entries of tiles before i
         bool ok = true;
@@ -498,7 +511,9 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         while (ok && !w.done()) {
             const Tile t = w.next();
             const int4 meta = meta_nxt;
-            if (!wa.done()) meta_nxt = p.unit_meta[wa.next().u];
+            int u_nxt = t.u;
+            if (!wa.done()) u_nxt = wa.next().u;
+            meta_nxt = p.unit_meta[u_nxt];
             // keys of this tile that belong to this segment
             const int key_end = min(meta.x, kPage * (t.page0 + t.np));
             if (t.first) {
@@ -624,6 +639,13 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 const bool whole = meta.z == 1;
                 const size_t grow = static_cast<size_t>(bt) * p.n_h + hb * 128 + head_in_unit;
                 const size_t slot = static_cast<size_t>(cluster) + t.u;
+                // This warp's 32 rows (consecutive heads) x 32 columns go through a
+                // 4 KB shared-memory tile in the free P buffer (16-byte chunks
+                // swizzled by row), so that each global store instruction writes
+                // whole row segments instead of 32 scattered 16-byte pieces.
+                unsigned char* stage = smem + kOffP + wq * 4096;
+                const size_t grow0 = grow - lane;
+                const size_t prow0 = slot * 128 + head_in_unit - lane;
 #pragma unroll 1
                 for (int h = 0; h < 2; ++h) {
                     const int col0 = 128 * h + (hi ? 256 : 0);
@@ -634,22 +656,41 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                         ptx::tmem_wait_ld();
                         const int col = col0 + 32 * q;
                         if (whole) {
-                            uint4* dst = reinterpret_cast<uint4*>(p.out_latent + grow * kDc + col);
+                            // 32 bf16 = 64 B per row, 4 chunks at position k ^ ((row >> 1) & 3)
 #pragma unroll
-                            for (int v = 0; v < 4; ++v) {
+                            for (int k = 0; k < 4; ++k) {
                                 uint4 wv;
-                                wv.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-                                wv.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-                                wv.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-                                wv.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-                                dst[v] = wv;
+                                wv.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
+                                wv.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
+                                wv.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
+                                wv.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
+                                *reinterpret_cast<uint4*>(stage + lane * 64 + ((k ^ ((lane >> 1) & 3)) * 16)) = wv;
                             }
-                        } else {
-                            float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * 128 + head_in_unit) * kDc + col);
+                            __syncwarp();
 #pragma unroll
-                            for (int v = 0; v < 8; ++v)
-                                dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
-                                                     __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
+                            for (int j = 0; j < 4; ++j) {
+                                const int row = 8 * j + (lane >> 2), k = lane & 3;
+                                const uint4 wv =
+                                    *reinterpret_cast<const uint4*>(stage + row * 64 + ((k ^ ((row >> 1) & 3)) * 16));
+                                *reinterpret_cast<uint4*>(p.out_latent + (grow0 + row) * kDc + col + 8 * k) = wv;
+                            }
+                            __syncwarp();
+                        } else {
+                            // 32 floats = 128 B per row, 8 chunks at position k ^ (row & 7)
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                *reinterpret_cast<float4*>(stage + lane * 128 + ((k ^ (lane & 7)) * 16)) =
+                                    make_float4(__uint_as_float(o[4 * k]) * inv, __uint_as_float(o[4 * k + 1]) * inv,
+                                                __uint_as_float(o[4 * k + 2]) * inv, __uint_as_float(o[4 * k + 3]) * inv);
+                            __syncwarp();
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int row = 4 * j + (lane >> 3), k = lane & 7;
+                                const float4 v =
+                                    *reinterpret_cast<const float4*>(stage + row * 128 + ((k ^ (row & 7)) * 16));
+                                *reinterpret_cast<float4*>(p.part_o + (prow0 + row) * kDc + col + 4 * k) = v;
+                            }
+                            __syncwarp();
                         }
                     }
                 }
@@ -770,7 +811,12 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, 
                 const int mid = (lo + hi + 1) >> 1;
                 if (pf[mid] <= a) lo = mid; else hi = mid - 1;
             }
-            ci = make_int4(a, e, lo, 0);
+            int lo2 = lo, hi2 = U - 1;   // last unit with prefix <= e - 1 (holds the range's last page)
+            while (lo2 < hi2) {
+                const int mid = (lo2 + hi2 + 1) >> 1;
+                if (pf[mid] <= e - 1) lo2 = mid; else hi2 = mid - 1;
+            }
+            ci = make_int4(a, e, lo, lo2);
         }
         cluster_info[c] = ci;
     }
