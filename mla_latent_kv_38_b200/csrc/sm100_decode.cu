@@ -13,25 +13,34 @@
 //
 // Mapping onto B200:
 //  * A cluster of two CTAs (two SMs) issues cta_group::2 MMAs with M = 128: CTA
-//    r owns heads [64r, 64r+64).  In the paired 128-row layout each SM's tensor
-//    memory holds its 64 rows spread over all 128 lanes, so the 128 x 512 fp32
-//    accumulator O needs 256 columns per SM and S (N = 64 keys) 32 columns;
-//    one CTA alone could not hold O (512 columns) and S together.
-//  * Per 64-row cache block (one page) each CTA loads by TMA (128-byte swizzle)
-//    its 32 keys x 576 columns for S (the pair's B operand is split by keys)
-//    and all 64 keys of the latent columns it contributes to P.V (the B
-//    operand of P.V is split by latent columns): CTA 0 columns [0,128) and
-//    [256,384), CTA 1 columns [128,256) and [384,512).
-//  * Warp roles per CTA: warp 0 issues TMA, warp 1 allocates tensor memory
-//    and (CTA 0 only) issues the MMAs, warps 2-5 run the softmax and the
-//    epilogue, one thread per tensor-memory lane.  S is double buffered so the
-//    softmax of block j overlaps P.V of block j-1.  The running max is
-//    rescaled lazily (only when it grows by more than 2^8).
-//  * Work: the key blocks of all (sequence, token, head block) units are laid
-//    end to end and cut into equal contiguous ranges, one per cluster
-//    (persistent, 74 clusters on 148 SMs).  A unit covered by one cluster is
-//    written directly in bf16; otherwise each cluster writes an fp32 partial
-//    and its log-sum-exp, merged by a reduction kernel.
+//    r owns heads [64r, 64r+64).  In the paired layout each SM's tensor memory
+//    holds its 64 rows spread over all 128 lanes (lanes 0-63 take the first
+//    half of N, lanes 64-127 the second), so O (64 heads x 512, fp32) takes 256
+//    columns per SM and one S buffer (N = 256 keys) 128 columns; O and two S
+//    buffers fill the 512 columns.
+//  * A tile is 4 cache pages (256 keys).  S = [q_abs ; q^R] . K^T runs as 9 MMA
+//    groups of K = 64 columns, N = 256: the pair's B operand is split by keys,
+//    so each CTA loads its own 2 pages (128 keys x 576 columns).  O += P . V
+//    runs as 2 x N = 256 per 16 keys: the B operand is split by latent
+//    columns, so each CTA loads all 4 pages of its 256 latent columns (these
+//    second reads hit L2).
+//  * All operands arrive by TMA (128-byte swizzle) in two rings, each with one
+//    producer warp and one in-order MMA consumer: S entries of 24 KB (one
+//    column chunk of the CTA's 2 pages plus the same chunk of its 64 query
+//    rows, re-read from L2 each tile so that no 72 KB query buffer has to stay
+//    resident) and V entries of 32 KB (the CTA's 4 latent chunks of one page,
+//    one 3-D box).
+//  * Warp roles per CTA: warp 0 S producer, warp 1 tensor-memory allocation
+//    and (CTA 0) the S MMAs, warps 2-5 softmax and epilogue (one thread per
+//    tensor-memory lane), warp 6 (CTA 0) the P.V MMAs, warp 7 V producer.  S
+//    is double buffered; P is written to shared memory in two key halves, each
+//    released as soon as its MMAs complete, so the next tile's softmax overlaps
+//    P.V.  The running max is rescaled lazily (only when it grows by 2^8).
+//  * Work: the pages of all (sequence, token, head block) units are laid end
+//    to end and cut into equal contiguous ranges, one per cluster (persistent,
+//    74 clusters on 148 SMs).  A unit covered by one cluster is written
+//    directly in bf16; otherwise each cluster writes an fp32 partial and its
+//    log-sum-exp, merged by a reduction kernel.
 //  * Every mbarrier wait is bounded by the global timer: on expiry the kernel
 //    sets MLA_STATUS_TIMEOUT and unwinds instead of hanging.
 
@@ -51,31 +60,25 @@ constexpr int kClusters = 74;                     // 148 SMs / 2
 constexpr int kDc = 512, kDr = 64, kRow = 576;    // row = c^KV || k^R
 constexpr int kPage = 64;                         // cache rows per page (TMA box height)
 constexpr int kTilePages = 4;                     // a tile = 4 pages = 256 keys (MMA N)
-constexpr int kSRing = 3;                         // 16 KB entries, S operand stream
-constexpr int kVRing = 2;                         // 32 KB entries (one page), P.V operand stream
+constexpr int kSRing = 4;                         // 24 KB entries, S operand stream
+constexpr int kVRing = 3;                         // 32 KB entries (one page), P.V operand stream
 
 constexpr uint32_t kBox = 8192;                   // one page x 64 columns (128 B rows)
-constexpr uint32_t kEntry = 2 * kBox;             // S ring entry: 2 boxes
+constexpr uint32_t kSEntry = 3 * kBox;            // S ring entry: a column chunk of the CTA's 2 pages + of its 64 heads' query
 constexpr uint32_t kVEntry = 4 * kBox;            // V ring entry: 4 latent chunks of one page
-constexpr uint32_t kQBytes = 9 * kBox;            // 64 heads x 576 columns
 constexpr uint32_t kPBytes = 4 * kBox;            // 64 heads x 256 keys (4 blocks of 64 keys)
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffSRing = kOffQ + kQBytes;
-constexpr uint32_t kOffVRing = kOffSRing + kSRing * kEntry;
+constexpr uint32_t kOffSRing = 0;
+constexpr uint32_t kOffVRing = kOffSRing + kSRing * kSEntry;
 constexpr uint32_t kOffP = kOffVRing + kVRing * kVEntry;
 constexpr uint32_t kOffXmax = kOffP + kPBytes;    // 2 x 128 floats
 constexpr uint32_t kOffXsum = kOffXmax + 1024;    // 128 floats
 constexpr uint32_t kOffBar = kOffXsum + 512;
 constexpr uint32_t kOffMisc = kOffBar + 8 * 32;   // tmem base, abort flag
-constexpr int kPrefixCache = 1024;                // units of a cluster's range kept in shared memory
-constexpr uint32_t kOffPrefix = kOffMisc + 16;
-constexpr uint32_t kSmemBytes = kOffPrefix + 4 * kPrefixCache + 1024;   // + alignment slack
+constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 enum {
-    BAR_Q_FULL = 0,
-    BAR_Q_EMPTY = 1,
-    BAR_SR_FULL = 2,                         // + slot (leader: both CTAs' bytes)
+    BAR_SR_FULL = 0,                         // + slot (leader: both CTAs' bytes)
     BAR_SR_EMPTY = BAR_SR_FULL + kSRing,     // + slot (each CTA, MMA commit)
     BAR_VR_FULL = BAR_SR_EMPTY + kSRing,
     BAR_VR_EMPTY = BAR_VR_FULL + kVRing,
@@ -156,7 +159,7 @@ struct Tile {
 struct TileWalker {
     const int32_t* pf;
     int off, g, g0, g1, u;
-    __device__ int prefix(int v) const { return pf[v - off]; }
+    __device__ int prefix(int v) const { return __ldg(pf + (v - off)); }
     __device__ void init(const int32_t* pf_, int off_, int u0, int g0_, int g1_) {
         pf = pf_;
         off = off_;
@@ -205,8 +208,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
 
     griddep_launch_dependents();
     if (threadIdx.x == 0) {
-        ptx::mbar_init(bar(BAR_Q_FULL), 1);
-        ptx::mbar_init(bar(BAR_Q_EMPTY), 1);
         for (int s = 0; s < kSRing; ++s) {
             ptx::mbar_init(bar(BAR_SR_FULL + s), 1);
             ptx::mbar_init(bar(BAR_SR_EMPTY + s), 1);
@@ -252,15 +253,8 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     // page g0, precomputed by the schedule kernel (empty range: no work)
     const int4 cinfo = p.cluster_info[cluster];
     const int g0 = cinfo.x, g1 = cinfo.y, u0 = cinfo.z;
-    // the page prefix of units u0 .. cinfo.w (+1), read by every role's tile walker
-    const int n_pre = cinfo.w - u0 + 2;
-    int32_t* pre_s = reinterpret_cast<int32_t*>(smem + kOffPrefix);
-    const bool pre_in_smem = g0 < g1 && n_pre <= kPrefixCache;
-    if (pre_in_smem)
-        for (int k = threadIdx.x; k < n_pre; k += kThreads) pre_s[k] = p.prefix[u0 + k];
-    __syncthreads();
-    const int32_t* pf_base = pre_in_smem ? pre_s : p.prefix;
-    const int pf_off = pre_in_smem ? u0 : 0;
+    const int32_t* pf_base = p.prefix;
+    const int pf_off = 0;
 
     // Two load streams, each consumed in order by one MMA issuer:
     //   S ring: S(i) = 9 entries (column chunk c of this CTA's pages 2r, 2r+1)
@@ -271,7 +265,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     // used (out-of-range entries are flagged and read as block 0).
     auto load_blk = [&](const Tile& t, int pg) -> int {
         const int b = t.u / (p.n_hb * p.T_q);
-        return p.block_table[static_cast<size_t>(b) * p.max_blocks + t.page0 + pg];
+        return __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks + t.page0 + pg);
     };
     auto blk_row = [&](int blk) -> int {
         if (blk < 0 || blk >= p.num_blocks) {
@@ -282,14 +276,14 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     };
 
     if (warp == 0) {
-        // ------------------------------------------------------------ S stream (and Q)
-        // Lanes 0 and 1 each wait for the entry's slot and issue one box (lane 0
-        // of the leader CTA arms the full barrier with both CTAs' bytes).  Lane
-        // l < 2 owns this CTA's page 2r + l of every tile: its block for tiles
-        // i, i+1, i+2 sits in b0, b1, b2 while tile i is issued.  (An L2
-        // prefetch of the pages ahead measured slower: the bulk prefetch holds
-        // this warp for about a microsecond per tile.)
-        const uint64_t pol_q = ptx::l2_policy_evict_last();
+        // ------------------------------------------------------------ S stream
+        // Entry c of a tile holds column chunk c (64 columns) of this CTA's two
+        // pages (keys) and of its 64 heads' query rows: the query is re-read from
+        // L2 with every tile instead of staying resident, which leaves room for
+        // deeper rings.  Lanes 0 and 1 load the pages, lane 2 the query chunk;
+        // lane 0 of the leader CTA arms the full barrier with both CTAs' bytes.
+        // Lane l < 2 owns this CTA's page 2r + l of every tile: its block for
+        // tiles i, i+1, i+2 sits in b0, b1, b2 while tile i is issued.
         const int my_pg = 2 * static_cast<int>(rank) + (lane & 1);
         TileWalker w, wa;
         w.init(pf_base, pf_off, u0, g0, g1);
@@ -309,37 +303,29 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         look(b0, h0);
         look(b1, h1);
         look(b2, h2);
-        int e = 0, uc = 0;
+        int e = 0;
         bool ok = g0 < g1;
         while (ok && !w.done()) {
             const Tile cur = w.next();
-            if (cur.first) {
-                // new unit segment: load Q (this CTA's 64 heads) from 9 lanes
-                bool good = true;
-                if (lane == 0) good = wait_bar(bar(BAR_Q_EMPTY), (uc & 1) ^ 1, abort_flag, p.status);
-                good = __shfl_sync(0xffffffffu, good, 0);
-                if (!good) { ok = false; break; }
-                const int bt = cur.u / p.n_hb, hb = cur.u - bt * p.n_hb;
-                const int qrow = bt * p.n_h + hb * 128 + 64 * static_cast<int>(rank);
-                if (lane == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_Q_FULL), 2 * kQBytes);
-                __syncwarp();
-                const uint32_t qf = leader_bar(BAR_Q_FULL);
-                if (lane < 8) ptx::tma_load_2d_pair(sbase + kOffQ + lane * kBox, &p.tm_qa, 64 * lane, qrow, qf, pol_q);
-                if (lane == 8) ptx::tma_load_2d_pair(sbase + kOffQ + 8 * kBox, &p.tm_qr, 0, qrow, qf, pol_q);
-                ++uc;
-            }
-            // S(cur): 9 column chunks of pages 2r, 2r+1
+            const int bt = cur.u / p.n_hb, hb = cur.u - bt * p.n_hb;
+            const int qrow = bt * p.n_h + hb * 128 + 64 * static_cast<int>(rank);
             const int row = h0 ? blk_row(b0) : 0;
-            const uint32_t tx = static_cast<uint32_t>(cur.np) * kBox;    // both CTAs together
+            const uint32_t tx = static_cast<uint32_t>(cur.np + 2) * kBox;    // both CTAs' pages and query chunks
             for (int c = 0; c < 9; ++c, ++e) {
                 const int slot = e % kSRing;
+                const uint32_t dst = sbase + kOffSRing + slot * kSEntry;
                 bool good = true;
-                if (lane < 2) {
+                if (lane < 3) {
                     good = wait_bar(bar(BAR_SR_EMPTY + slot), ((e / kSRing) & 1) ^ 1, abort_flag, p.status);
                     if (good && lane == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_SR_FULL + slot), tx);
-                    if (good && h0)
-                        ptx::tma_load_2d_pair_normal(sbase + kOffSRing + slot * kEntry + (lane & 1) * kBox, &p.tm_pool,
-                                                     64 * c, row, leader_bar(BAR_SR_FULL + slot));
+                    // one TMA instruction for the three lanes' boxes
+                    const bool q_lane = lane == 2;
+                    const void* tm = q_lane ? (c < 8 ? static_cast<const void*>(&p.tm_qa) : &p.tm_qr) : &p.tm_pool;
+                    const int bx = q_lane ? (c < 8 ? 64 * c : 0) : 64 * c;
+                    const int by = q_lane ? qrow : row;
+                    if (good && (h0 || q_lane))
+                        ptx::tma_load_2d_pair_normal(dst + (q_lane ? 2 : (lane & 1)) * kBox, tm, bx, by,
+                                                     leader_bar(BAR_SR_FULL + slot));
                 }
                 if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
             }
@@ -387,27 +373,27 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ S = Q K^T issuer
-        // S(i) occupies entries 9 i .. 9 i + 8 of the S ring.
+        // S(i) occupies entries 9 i .. 9 i + 8 of the S ring (keys as B, query as A).
         if (rank == 0 && lane == 0 && g0 < g1) {
             TileWalker w;
             w.init(pf_base, pf_off, u0, g0, g1);
-            int i = 0, uc = 0;
+            int i = 0;
             bool ok = true;
-            const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffQ, 16, 1024);
             while (ok && !w.done()) {
-                const Tile cur = w.next();
+                w.next();
                 const int e0 = 9 * i;
                 const int sb = i & 1;
-                if (cur.first && !(ok = wait_bar(bar(BAR_Q_FULL), uc & 1, abort_flag, p.status))) break;
                 if (!(ok = wait_bar(bar(BAR_S_FREE + sb), ((i >> 1) & 1) ^ 1, abort_flag, p.status))) break;
                 ptx::tc_fence_after();   // the softmax's reads of this S buffer are done
                 for (int c = 0; c < 9; ++c) {
                     const int e = e0 + c;
                     if (!(ok = wait_bar(bar(BAR_SR_FULL + e % kSRing), (e / kSRing) & 1, abort_flag, p.status))) break;
-                    const uint64_t b0 = ptx::smem_desc_sw128(sbase + kOffSRing + (e % kSRing) * kEntry, 16, 1024);
+                    const uint32_t ent = sbase + kOffSRing + (e % kSRing) * kSEntry;
+                    const uint64_t b0 = ptx::smem_desc_sw128(ent, 16, 1024);
+                    const uint64_t a0 = ptx::smem_desc_sw128(ent + 2 * kBox, 16, 1024);
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
-                        const uint64_t a = a0 + static_cast<uint64_t>((c * kBox + 32 * k4) >> 4);
+                        const uint64_t a = a0 + static_cast<uint64_t>((32 * k4) >> 4);
                         const uint64_t bd = b0 + static_cast<uint64_t>((32 * k4) >> 4);
                         ptx::mma_pair_ss(tmem_base + kTmemS + 128 * sb, a, bd, kIdescS, (c | k4) ? 1u : 0u);
                     }
@@ -415,10 +401,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 }
                 if (!ok) break;
                 ptx::mma_commit_pair(bar(BAR_S_FULL + sb), 0x3);
-                if (cur.last) {
-                    ptx::mma_commit_pair(bar(BAR_Q_EMPTY), 0x3);
-                    ++uc;
-                }
                 ++i;
             }
             if (!ok) {
@@ -440,7 +422,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffP, 16, 1024);
             while (ok && !w.done()) {
                 const Tile t = w.next();
-                const int kv_len = p.unit_meta[t.u].x;   // read before the wait hides its latency
+                const int kv_len = __ldg(&p.unit_meta[t.u].x);   // read before the wait hides its latency
                 const bool tail = t.unit_end && (kv_len % kPage) != 0;
                 // P is written in two halves: keys [0,128) (pages 0, 1) by the softmax
                 // warps of TMEM lanes 0-63, keys [128,256) by those of lanes 64-127;
@@ -503,7 +485,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         w.init(pf_base, pf_off, u0, g0, g1);
         wa.init(pf_base, pf_off, u0, g0, g1);
         const int u_first = g0 < g1 ? wa.next().u : 0;
-        int4 meta_nxt = p.unit_meta[u_first];
+        int4 meta_nxt = __ldg(&p.unit_meta[u_first]);
         int i = 0, tails = 0;
         int v_before = 0;      // V ring entries of tiles before i
         bool ok = true;
@@ -513,7 +495,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             const int4 meta = meta_nxt;
             int u_nxt = t.u;
             if (!wa.done()) u_nxt = wa.next().u;
-            meta_nxt = p.unit_meta[u_nxt];
+            meta_nxt = __ldg(&p.unit_meta[u_nxt]);
             // keys of this tile that belong to this segment
             const int key_end = min(meta.x, kPage * (t.page0 + t.np));
             if (t.first) {
