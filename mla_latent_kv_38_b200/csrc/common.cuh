@@ -24,9 +24,10 @@ __device__ __forceinline__ uint16_t f2bf(float f) {
     return *reinterpret_cast<uint16_t*>(&h);
 }
 
-// two floats -> packed bf16x2 (lo in the low half)
+// two floats -> packed bf16x2 (lo in the low half), one paired conversion
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    return static_cast<uint32_t>(f2bf(lo)) | (static_cast<uint32_t>(f2bf(hi)) << 16);
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
 }
 
 __device__ __forceinline__ void unpack8(const uint4& v, float* f) {

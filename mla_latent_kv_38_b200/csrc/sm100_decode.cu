@@ -74,8 +74,12 @@ constexpr uint32_t kOffXmax = kOffP + kPBytes;    // 2 x 128 floats
 constexpr uint32_t kOffXsum = kOffXmax + 1024;    // 128 floats
 constexpr uint32_t kOffBar = kOffXsum + 512;
 constexpr uint32_t kOffMisc = kOffBar + 8 * 32;   // tmem base, abort flag
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+constexpr uint32_t kSmemUsed = kOffMisc + 16;
+// Dynamic shared memory: the buffers above from a 1024-byte aligned base; what
+// the alignment leaves over at the end holds a copy of the cluster's unit
+// prefix when it fits.
+constexpr uint32_t kSmemBytes = 232448;
+static_assert(kSmemUsed + 1024 <= kSmemBytes, "shared memory budget");
 
 enum {
     BAR_SR_FULL = 0,                         // + slot (leader: both CTAs' bytes)
@@ -145,7 +149,10 @@ __device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, volatil
 
 // One tile of a cluster's work: up to 4 consecutive pages of one unit.
 struct Tile {
-    int u;          // unit
+    int u;          // unit = (b T_q + t) n_hb + hb
+    int bt;         // query row b T_q + t of the unit
+    int hb;         // head block of the unit
+    int b;          // sequence of the unit
     int page0;      // first page, within the unit
     int np;         // pages in this tile (1..4)
     bool first;     // first tile of a unit segment (new Q, O starts from zero)
@@ -153,36 +160,58 @@ struct Tile {
     bool unit_end;  // the unit's last page is in this tile
 };
 
-// Walks a cluster's pages [g0, g1) as tiles.
-// The prefix entry of unit u is pf[u - off] (pf: a shared-memory copy of the
-// cluster's range, or the global array with off = 0).
+// Walks a cluster's pages [g0, g1) as tiles.  The prefix entry of unit v is
+// pf[v - off] (pf: a shared-memory copy of the cluster's range of the prefix,
+// or the global array with off = 0).  The unit's (query row, head block,
+// sequence) are kept up to date incrementally, without divisions.
 struct TileWalker {
     const int32_t* pf;
     int off, g, g0, g1, u;
-    __device__ int prefix(int v) const { return __ldg(pf + (v - off)); }
-    __device__ void init(const int32_t* pf_, int off_, int u0, int g0_, int g1_) {
+    int bt, hb, b, t, n_hb, T_q;
+    __device__ int prefix(int v) const { return pf[v - off]; }
+    __device__ void step_unit() {
+        ++u;
+        if (++hb == n_hb) {
+            hb = 0;
+            ++bt;
+            if (++t == T_q) {
+                t = 0;
+                ++b;
+            }
+        }
+    }
+    __device__ void init(const int32_t* pf_, int off_, int u0, int g0_, int g1_, int n_hb_, int T_q_) {
         pf = pf_;
         off = off_;
         g = g0_;
         g0 = g0_;
         g1 = g1_;
+        n_hb = n_hb_;
+        T_q = T_q_;
         u = u0;
-        while (g < g1 && prefix(u + 1) <= g) ++u;
+        bt = u0 / n_hb;
+        hb = u0 - bt * n_hb;
+        b = bt / T_q;
+        t = bt - b * T_q;
+        while (g < g1 && prefix(u + 1) <= g) step_unit();
     }
     __device__ bool done() const { return g >= g1; }
     __device__ Tile next() {
-        Tile t;
+        Tile r;
         const int ubeg = prefix(u), uend = prefix(u + 1);
-        t.u = u;
-        t.page0 = g - ubeg;
-        t.first = (g == g0) || (g == ubeg);
+        r.u = u;
+        r.bt = bt;
+        r.hb = hb;
+        r.b = b;
+        r.page0 = g - ubeg;
+        r.first = (g == g0) || (g == ubeg);
         const int seg_end = min(g1, uend);   // tiles start at the segment start
-        t.np = min(kTilePages, seg_end - g);
-        t.last = g + t.np == seg_end;
-        t.unit_end = g + t.np == uend;
-        g += t.np;
-        while (g < g1 && prefix(u + 1) <= g) ++u;
-        return t;
+        r.np = min(kTilePages, seg_end - g);
+        r.last = g + r.np == seg_end;
+        r.unit_end = g + r.np == uend;
+        g += r.np;
+        while (g < g1 && prefix(u + 1) <= g) step_unit();
+        return r;
     }
 };
 
@@ -253,8 +282,16 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     // page g0, precomputed by the schedule kernel (empty range: no work)
     const int4 cinfo = p.cluster_info[cluster];
     const int g0 = cinfo.x, g1 = cinfo.y, u0 = cinfo.z;
-    const int32_t* pf_base = p.prefix;
-    const int pf_off = 0;
+    const int n_pre = cinfo.w - u0 + 2;   // prefix entries of units u0 .. cinfo.w, + 1
+    int32_t* pre_s = reinterpret_cast<int32_t*>(smem + kSmemUsed);
+    const int pre_cap = static_cast<int>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + kSmemBytes - reinterpret_cast<uintptr_t>(pre_s)) / 4);
+    const bool pre_in_smem = g0 < g1 && n_pre <= pre_cap;
+    if (pre_in_smem)
+        for (int k = threadIdx.x; k < n_pre; k += kThreads) pre_s[k] = p.prefix[u0 + k];
+    __syncthreads();
+    const int32_t* pf_base = pre_in_smem ? pre_s : p.prefix;
+    const int pf_off = pre_in_smem ? u0 : 0;
 
     // Two load streams, each consumed in order by one MMA issuer:
     //   S ring: S(i) = 9 entries (column chunk c of this CTA's pages 2r, 2r+1)
@@ -264,8 +301,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     // ring waits of the tiles in between; an entry is validated where it is
     // used (out-of-range entries are flagged and read as block 0).
     auto load_blk = [&](const Tile& t, int pg) -> int {
-        const int b = t.u / (p.n_hb * p.T_q);
-        return __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks + t.page0 + pg);
+        return __ldg(p.block_table + static_cast<size_t>(t.b) * p.max_blocks + t.page0 + pg);
     };
     auto blk_row = [&](int blk) -> int {
         if (blk < 0 || blk >= p.num_blocks) {
@@ -286,8 +322,8 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // tiles i, i+1, i+2 sits in b0, b1, b2 while tile i is issued.
         const int my_pg = 2 * static_cast<int>(rank) + (lane & 1);
         TileWalker w, wa;
-        w.init(pf_base, pf_off, u0, g0, g1);
-        wa.init(pf_base, pf_off, u0, g0, g1);
+        w.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
+        wa.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
         int b0 = 0, b1 = 0, b2 = 0;
         bool h0 = false, h1 = false, h2 = false;
         // (the loads are unconditional, to a valid entry, so that nothing waits
@@ -307,8 +343,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         bool ok = g0 < g1;
         while (ok && !w.done()) {
             const Tile cur = w.next();
-            const int bt = cur.u / p.n_hb, hb = cur.u - bt * p.n_hb;
-            const int qrow = bt * p.n_h + hb * 128 + 64 * static_cast<int>(rank);
+            const int qrow = cur.bt * p.n_h + cur.hb * 128 + 64 * static_cast<int>(rank);
             const int row = h0 ? blk_row(b0) : 0;
             const uint32_t tx = static_cast<uint32_t>(cur.np + 2) * kBox;    // both CTAs' pages and query chunks
             for (int c = 0; c < 9; ++c, ++e) {
@@ -339,8 +374,8 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // the next one (v1).
         const uint64_t pol_v = ptx::l2_policy_evict_first();   // last use of these lines
         TileWalker w, wa;
-        w.init(pf_base, pf_off, u0, g0, g1);
-        wa.init(pf_base, pf_off, u0, g0, g1);
+        w.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
+        wa.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
         int v0 = 0, v1 = 0;
         auto look = [&](int& v) {
             if (!wa.done()) {
@@ -376,7 +411,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // S(i) occupies entries 9 i .. 9 i + 8 of the S ring (keys as B, query as A).
         if (rank == 0 && lane == 0 && g0 < g1) {
             TileWalker w;
-            w.init(pf_base, pf_off, u0, g0, g1);
+            w.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
             int i = 0;
             bool ok = true;
             while (ok && !w.done()) {
@@ -416,7 +451,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // V(i) occupies the next 2 np entries of the V ring.
         if (rank == 0 && lane == 0 && g0 < g1) {
             TileWalker w;
-            w.init(pf_base, pf_off, u0, g0, g1);
+            w.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
             int i = 0, tails = 0, e = 0;
             bool ok = true;
             const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffP, 16, 1024);
@@ -482,8 +517,8 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         float* xmax = reinterpret_cast<float*>(smem + kOffXmax);
         float* xsum = reinterpret_cast<float*>(smem + kOffXsum);
         TileWalker w, wa;      // wa runs one tile ahead: the next tile's unit data is loaded early
-        w.init(pf_base, pf_off, u0, g0, g1);
-        wa.init(pf_base, pf_off, u0, g0, g1);
+        w.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
+        wa.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
         const int u_first = g0 < g1 ? wa.next().u : 0;
         int4 meta_nxt = __ldg(&p.unit_meta[u_first]);
         int i = 0, tails = 0;
@@ -506,25 +541,23 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             ok = wait_bar(bar(BAR_S_FULL + sb), (i >> 1) & 1, abort_flag, p.status);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             ptx::tc_fence_after();
-            uint32_t r[128];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t (&rq)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q]);
-                ptx::tmem_ld32(t_lane + kTmemS + 128 * sb + 32 * q, rq);
-            }
-            ptx::tmem_wait_ld();
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive_cluster_relaxed(leader_bar(BAR_S_FREE + sb));
-
+            // This thread's 128 scores (row m, keys key0 ..) are read from tensor
+            // memory twice, 32 at a time: once for the row maximum, once for the
+            // weights, which keeps the register footprint small.
+            const uint32_t s_col = t_lane + kTmemS + 128 * sb;
             const int key0 = kPage * t.page0 + (hi ? 128 : 0);
+            const int nvalid = key_end - key0;   // scores of this thread that count (<= 0 .. >= 128)
             float mx = -INFINITY;
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t r[32];
+                ptx::tmem_ld32(s_col + 32 * q, r);
+                ptx::tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 128; ++q) {
-                const float v = (key0 + q < key_end) ? __uint_as_float(r[q]) * p.scale_log2 : -INFINITY;
-                r[q] = __float_as_uint(v);
-                mx = fmaxf(mx, v);
+                for (int j = 0; j < 32; ++j)
+                    if (32 * q + j < nvalid) mx = fmaxf(mx, __uint_as_float(r[j]));
             }
+            mx *= p.scale_log2;   // the scale is positive
             float* xb = xmax + (i & 1) * 128;
             xb[l] = mx;
             ptx::named_bar_sync(1, 128);
@@ -537,14 +570,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             }
             const float alpha = ex2(m_used - new_m);
             m_used = new_m;
-            float ps = 0.f;
-#pragma unroll
-            for (int q = 0; q < 128; q += 2) {
-                const float p0 = ex2(__uint_as_float(r[q]) - m_used), p1 = ex2(__uint_as_float(r[q + 1]) - m_used);
-                ps += p0 + p1;
-                r[q >> 1] = pack_bf16x2(p0, p1);
-            }
-            l_part = l_part * alpha + ps;
 
             // This half of the P buffer must be free (the previous tile's P.V MMAs on
             // it complete); a rescale of O needs the whole previous P.V complete.
@@ -566,18 +591,38 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 }
                 ptx::tmem_wait_st();
             }
-            // P row m, keys (hi ? 128 : 0) + [0, 128): blocks of 64 keys, K-major,
-            // 128-byte rows, 128-byte swizzle (chunk index XOR row & 7)
+            // P row m, keys key0 + [0, 128): blocks of 64 keys, K-major, 128-byte
+            // rows, 128-byte swizzle (16-byte chunk index XOR row & 7)
+            float ps = 0.f;
+            const float neg_m = -m_used;
+            unsigned char* Prow = smem + kOffP + (hi ? 2 : 0) * kBox + m * 128;
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t r[32];
+                ptx::tmem_ld32(s_col + 32 * q, r);
+                ptx::tmem_wait_ld();
+                uint32_t pk[16];
 #pragma unroll
-            for (int blk = 0; blk < 2; ++blk) {
-                unsigned char* Pb = smem + kOffP + ((hi ? 2 : 0) + blk) * kBox + m * 128;
+                for (int j = 0; j < 32; j += 2) {
+                    const float p0 = 32 * q + j < nvalid ? ex2(fmaf(__uint_as_float(r[j]), p.scale_log2, neg_m)) : 0.f;
+                    const float p1 =
+                        32 * q + j + 1 < nvalid ? ex2(fmaf(__uint_as_float(r[j + 1]), p.scale_log2, neg_m)) : 0.f;
+                    ps += p0 + p1;
+                    pk[j >> 1] = pack_bf16x2(p0, p1);
+                }
+                unsigned char* Pb = Prow + (q >> 1) * kBox;
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const int phys = ch ^ (m & 7);
-                    const int w0 = 32 * blk + 4 * ch;
-                    *reinterpret_cast<uint4*>(Pb + phys * 16) = make_uint4(r[w0], r[w0 + 1], r[w0 + 2], r[w0 + 3]);
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int ch = (q & 1) * 4 + c4;
+                    *reinterpret_cast<uint4*>(Pb + ((ch ^ (m & 7)) * 16)) =
+                        make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
                 }
             }
+            l_part = l_part * alpha + ps;
+            // both reads of the S buffer are done
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster_relaxed(leader_bar(BAR_S_FREE + sb));
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             __syncwarp();
@@ -616,7 +661,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 const float lsum = l_part + xsum[l ^ 64];
                 const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
                 const float lse = lsum > 0.f ? (m_used + __log2f(lsum)) * kLn2 : -INFINITY;
-                const int bt = t.u / p.n_hb, hb = t.u - bt * p.n_hb;
+                const int bt = t.bt, hb = t.hb;
                 const int head_in_unit = 64 * static_cast<int>(rank) + m;
                 const bool whole = meta.z == 1;
                 const size_t grow = static_cast<size_t>(bt) * p.n_h + hb * 128 + head_in_unit;
