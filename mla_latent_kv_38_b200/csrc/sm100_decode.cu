@@ -549,13 +549,14 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             const int nvalid = key_end - key0;   // scores of this thread that count (<= 0 .. >= 128)
             float mx = -INFINITY;
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-                uint32_t r[32];
-                ptx::tmem_ld32(s_col + 32 * q, r);
+            for (int q = 0; q < 4; q += 2) {
+                uint32_t r[2][32];
+                ptx::tmem_ld32(s_col + 32 * q, r[0]);
+                ptx::tmem_ld32(s_col + 32 * q + 32, r[1]);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (32 * q + j < nvalid) mx = fmaxf(mx, __uint_as_float(r[j]));
+                for (int j = 0; j < 64; ++j)
+                    if (32 * q + j < nvalid) mx = fmaxf(mx, __uint_as_float(r[j >> 5][j & 31]));
             }
             mx *= p.scale_log2;   // the scale is positive
             float* xb = xmax + (i & 1) * 128;
@@ -597,26 +598,25 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             const float neg_m = -m_used;
             unsigned char* Prow = smem + kOffP + (hi ? 2 : 0) * kBox + m * 128;
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-                uint32_t r[32];
-                ptx::tmem_ld32(s_col + 32 * q, r);
+            for (int q = 0; q < 4; q += 2) {   // 64 keys = one 64-key block of P
+                uint32_t r[2][32];
+                ptx::tmem_ld32(s_col + 32 * q, r[0]);
+                ptx::tmem_ld32(s_col + 32 * q + 32, r[1]);
                 ptx::tmem_wait_ld();
-                uint32_t pk[16];
+                uint32_t pk[32];
 #pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    const float p0 = 32 * q + j < nvalid ? ex2(fmaf(__uint_as_float(r[j]), p.scale_log2, neg_m)) : 0.f;
-                    const float p1 =
-                        32 * q + j + 1 < nvalid ? ex2(fmaf(__uint_as_float(r[j + 1]), p.scale_log2, neg_m)) : 0.f;
+                for (int j = 0; j < 64; j += 2) {
+                    const float s0 = __uint_as_float(r[j >> 5][j & 31]), s1 = __uint_as_float(r[j >> 5][(j & 31) + 1]);
+                    const float p0 = 32 * q + j < nvalid ? ex2(fmaf(s0, p.scale_log2, neg_m)) : 0.f;
+                    const float p1 = 32 * q + j + 1 < nvalid ? ex2(fmaf(s1, p.scale_log2, neg_m)) : 0.f;
                     ps += p0 + p1;
                     pk[j >> 1] = pack_bf16x2(p0, p1);
                 }
                 unsigned char* Pb = Prow + (q >> 1) * kBox;
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const int ch = (q & 1) * 4 + c4;
+                for (int ch = 0; ch < 8; ++ch)
                     *reinterpret_cast<uint4*>(Pb + ((ch ^ (m & 7)) * 16)) =
-                        make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
-                }
+                        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
             }
             l_part = l_part * alpha + ps;
             // both reads of the S buffer are done
