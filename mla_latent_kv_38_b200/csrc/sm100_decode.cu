@@ -106,6 +106,7 @@ constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 256, 0, 0);
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 256, 0, 1);
 
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr uint32_t kSuspendHintNs = 100000;      // a waiting thread sleeps up to 0.1 ms per try
 constexpr int kSchedSmemUnits = 8192;             // units whose prefix the schedule keeps in shared memory
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
 
@@ -133,9 +134,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, volatil
     if (ptx::mbar_try_wait(addr, parity)) return true;
     const uint64_t t0 = ptx::global_timer_ns();
     while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 64; ++i)
-            if (ptx::mbar_try_wait(addr, parity)) return true;
+        if (ptx::mbar_try_wait_suspend(addr, parity, kSuspendHintNs)) return true;
         if (*abort_flag) return false;
         if (ptx::global_timer_ns() - t0 > kTimeoutNs) {
             *abort_flag = 1;
@@ -547,7 +546,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             const uint32_t s_col = t_lane + kTmemS + 128 * sb;
             const int key0 = kPage * t.page0 + (hi ? 128 : 0);
             const int nvalid = key_end - key0;   // scores of this thread that count (<= 0 .. >= 128)
-            float mx = -INFINITY;
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // independent chains
 #pragma unroll 1
             for (int q = 0; q < 4; q += 2) {
                 uint32_t r[2][32];
@@ -556,8 +555,9 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 ptx::tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
-                    if (32 * q + j < nvalid) mx = fmaxf(mx, __uint_as_float(r[j >> 5][j & 31]));
+                    if (32 * q + j < nvalid) mx4[j & 3] = fmaxf(mx4[j & 3], __uint_as_float(r[j >> 5][j & 31]));
             }
+            float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             mx *= p.scale_log2;   // the scale is positive
             float* xb = xmax + (i & 1) * 128;
             xb[l] = mx;
@@ -594,7 +594,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             }
             // P row m, keys key0 + [0, 128): blocks of 64 keys, K-major, 128-byte
             // rows, 128-byte swizzle (16-byte chunk index XOR row & 7)
-            float ps = 0.f;
+            float ps2[2] = {0.f, 0.f};
             const float neg_m = -m_used;
             unsigned char* Prow = smem + kOffP + (hi ? 2 : 0) * kBox + m * 128;
 #pragma unroll 1
@@ -609,7 +609,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                     const float s0 = __uint_as_float(r[j >> 5][j & 31]), s1 = __uint_as_float(r[j >> 5][(j & 31) + 1]);
                     const float p0 = 32 * q + j < nvalid ? ex2(fmaf(s0, p.scale_log2, neg_m)) : 0.f;
                     const float p1 = 32 * q + j + 1 < nvalid ? ex2(fmaf(s1, p.scale_log2, neg_m)) : 0.f;
-                    ps += p0 + p1;
+                    ps2[(j >> 1) & 1] += p0 + p1;
                     pk[j >> 1] = pack_bf16x2(p0, p1);
                 }
                 unsigned char* Pb = Prow + (q >> 1) * kBox;
@@ -618,6 +618,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                     *reinterpret_cast<uint4*>(Pb + ((ch ^ (m & 7)) * 16)) =
                         make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
             }
+            const float ps = ps2[0] + ps2[1];
             l_part = l_part * alpha + ps;
             // both reads of the S buffer are done
             ptx::tc_fence_before();

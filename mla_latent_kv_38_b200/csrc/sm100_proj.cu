@@ -54,7 +54,7 @@ struct ProjParams {
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = ptx::global_timer_ns();
-    while (!ptx::mbar_try_wait(bar, parity))
+    while (!ptx::mbar_try_wait_suspend(bar, parity, 100000))
         if (ptx::global_timer_ns() - t0 > kTimeoutNs) return false;
     return true;
 }
@@ -99,28 +99,29 @@ __global__ void __launch_bounds__(kThreads, 1) mla_proj_sm100_kernel(const __gri
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    auto load_b = [&](int t) {
-        ptx::mbar_arrive_expect_tx(barB, kchunks * b_box);
-        for (int kc = 0; kc < kchunks; ++kc)
-            ptx::tma_load_2d(sB + kc * b_box, &p.tm_b, head * K + 64 * kc, t * nt, barB);
+    // Boxes are issued by the lanes of warp 0 in parallel (one box each).
+    const int lane = threadIdx.x & 31;
+    auto load_b = [&](int t) {   // warp 0
+        if (lane == 0) ptx::mbar_arrive_expect_tx(barB, kchunks * b_box);
+        __syncwarp();
+        if (lane < kchunks) ptx::tma_load_2d(sB + lane * b_box, &p.tm_b, head * K + 64 * lane, t * nt, barB);
     };
 
     // The weights are read-only inputs no kernel writes: fetch them while the
     // previous kernel finishes, then wait for it before touching activations.
-    if (threadIdx.x == 0) {
-        ptx::mbar_arrive_expect_tx(barA, a_bytes);
+    if (warp == 0) {
+        if (lane == 0) ptx::mbar_arrive_expect_tx(barA, a_bytes);
+        __syncwarp();
         if (kAbsorb) {
             // two boxes of 64 latent columns x d_h rows: [mh][k][64 c]
-            for (int mh = 0; mh < 2; ++mh)
-                ptx::tma_load_2d(sA + mh * (K * 128), &p.tm_a, m0 + 64 * mh, head * p.d_h, barA);
+            if (lane < 2) ptx::tma_load_2d(sA + lane * (K * 128), &p.tm_a, m0 + 64 * lane, head * p.d_h, barA);
         } else {
             // d_c / 64 boxes of 64 latent columns x 128 rows: [kc][k][64 c]
-            for (int kc = 0; kc < kchunks; ++kc)
-                ptx::tma_load_2d(sA + kc * (kM * 128), &p.tm_a, 64 * kc, head * p.d_h + m0, barA);
+            if (lane < kchunks) ptx::tma_load_2d(sA + lane * (kM * 128), &p.tm_a, 64 * lane, head * p.d_h + m0, barA);
         }
     }
     griddep_wait();
-    if (threadIdx.x == 0) load_b(0);
+    if (warp == 0) load_b(0);
 
     const int row = m0 + threadIdx.x;   // this thread's output feature (TMEM lane)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
@@ -142,13 +143,13 @@ __global__ void __launch_bounds__(kThreads, 1) mla_proj_sm100_kernel(const __gri
                 }
                 ptx::mma1_commit(barD);
                 ok = wait_bounded(barD, t & 1);
-                // the MMAs have read B: fetch the next token tile during the epilogue
-                if (ok && t + 1 < n_tiles) load_b(t + 1);
             }
             s_ok = ok;
         }
         __syncthreads();
         if (!s_ok) break;
+        // the MMAs have read B: fetch the next token tile during the epilogue
+        if (warp == 0 && t + 1 < n_tiles) load_b(t + 1);
         ptx::tc_fence_after();
         const int n0 = t * nt;
         const int nvalid = min(nt, p.n_tok - n0);

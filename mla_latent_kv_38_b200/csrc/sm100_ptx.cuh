@@ -67,6 +67,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
     return ok != 0;
 }
 
+// Same, but a thread whose phase has not completed is suspended for up to
+// `hint_ns` (woken early when the phase completes) instead of returning at
+// once, so that waiting warps leave the issue slots to working ones.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t addr, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // non-blocking probe (for polling several barriers from one thread)
 __device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t parity) {
     uint32_t ok;
