@@ -55,7 +55,7 @@
 namespace mla {
 namespace {
 
-constexpr int kThreads = 256;   // 8 warps: S loads, S MMAs, 4 x softmax, P.V MMAs, V loads
+constexpr int kThreads = 384;   // 12 warps: S loads, S MMAs, P.V MMAs, V loads, 8 x softmax
 constexpr int kClusters = 74;                     // 148 SMs / 2
 constexpr int kDc = 512, kDr = 64, kRow = 576;    // row = c^KV || k^R
 constexpr int kPage = 64;                         // cache rows per page (TMA box height)
@@ -70,9 +70,8 @@ constexpr uint32_t kPBytes = 4 * kBox;            // 64 heads x 256 keys (4 bloc
 constexpr uint32_t kOffSRing = 0;
 constexpr uint32_t kOffVRing = kOffSRing + kSRing * kSEntry;
 constexpr uint32_t kOffP = kOffVRing + kVRing * kVEntry;
-constexpr uint32_t kOffXmax = kOffP + kPBytes;    // 2 x 128 floats
-constexpr uint32_t kOffXsum = kOffXmax + 1024;    // 128 floats
-constexpr uint32_t kOffBar = kOffXsum + 512;
+constexpr uint32_t kOffXmax = kOffP + kPBytes;    // 4 x 64 floats: partial row maxima (or sums)
+constexpr uint32_t kOffBar = kOffXmax + 1024;
 constexpr uint32_t kOffMisc = kOffBar + 8 * 32;   // tmem base, abort flag
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
 // Dynamic shared memory: the buffers above from a 1024-byte aligned base; what
@@ -246,14 +245,14 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(bar(BAR_S_FULL + b), 1);
-            ptx::mbar_init(bar(BAR_S_FREE + b), 8);   // 4 softmax warps x 2 CTAs
+            ptx::mbar_init(bar(BAR_S_FREE + b), 16);   // 8 softmax warps x 2 CTAs
         }
         for (int hf = 0; hf < 2; ++hf) {
-            ptx::mbar_init(bar(BAR_P_FULL + hf), 4);
+            ptx::mbar_init(bar(BAR_P_FULL + hf), 8);   // 4 softmax warps x 2 CTAs
             ptx::mbar_init(bar(BAR_P_FREE + hf), 1);
         }
         ptx::mbar_init(bar(BAR_TAIL_READY), 1);
-        ptx::mbar_init(bar(BAR_TAIL_DONE), 8);
+        ptx::mbar_init(bar(BAR_TAIL_DONE), 16);
         ptx::mbar_init(bar(BAR_DRAIN), 1);
         ptx::mbar_init(bar(BAR_DRAIN_PV), 1);
         *abort_flag = 0;
@@ -367,7 +366,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             b1 = b2; h1 = h2;
             look(b2, h2);
         }
-    } else if (warp == 7) {
+    } else if (warp == 3) {
         // ------------------------------------------------------------ V stream
         // Lane pg < 4 holds the block of page pg of the current tile (v0) and of
         // the next one (v1).
@@ -445,7 +444,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 }
             }
         }
-    } else if (warp == 6) {
+    } else if (warp == 2) {
         // ------------------------------------------------------------ O += P V issuer
         // V(i) occupies the next 2 np entries of the V ring.
         if (rank == 0 && lane == 0 && g0 < g1) {
@@ -508,13 +507,19 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         }
     } else {
         // ------------------------------------------------------------ softmax + epilogue
+        // Eight warps, two per tensor-memory lane quadrant: a thread owns lane l
+        // (head row m, key half hi of the S tile, latent half hi of O) and
+        // column group cg (64 of the lane's 128 S columns, 128 of its 256 O
+        // columns), so four threads share a head row.
+        const int sw = warp - 4;                     // softmax warp 0..7
         const int wq = warp & 3;                     // tensor-memory lane quadrant
+        const int cg = sw >> 2;                      // column group
         const int l = wq * 32 + lane;                // lane = (row, half)
         const bool hi = l >= 64;
         const int m = l & 63;
+        const int st = sw * 32 + lane;               // 0 .. 255 over the softmax warps
         const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
-        float* xmax = reinterpret_cast<float*>(smem + kOffXmax);
-        float* xsum = reinterpret_cast<float*>(smem + kOffXsum);
+        float* xmax = reinterpret_cast<float*>(smem + kOffXmax);   // [cg][l]
         TileWalker w, wa;      // wa runs one tile ahead: the next tile's unit data is loaded early
         w.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
         wa.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
@@ -524,6 +529,10 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         int v_before = 0;      // V ring entries of tiles before i
         bool ok = true;
         float m_used = -INFINITY, l_part = 0.f;
+        // the four partial values of row m (both key halves, both column groups)
+        auto row_max4 = [&]() {
+            return fmaxf(fmaxf(xmax[m], xmax[64 + m]), fmaxf(xmax[128 + m], xmax[192 + m]));
+        };
         while (ok && !w.done()) {
             const Tile t = w.next();
             const int4 meta = meta_nxt;
@@ -540,29 +549,27 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             ok = wait_bar(bar(BAR_S_FULL + sb), (i >> 1) & 1, abort_flag, p.status);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             ptx::tc_fence_after();
-            // This thread's 128 scores (row m, keys key0 ..) are read from tensor
-            // memory twice, 32 at a time: once for the row maximum, once for the
-            // weights, which keeps the register footprint small.
-            const uint32_t s_col = t_lane + kTmemS + 128 * sb;
-            const int key0 = kPage * t.page0 + (hi ? 128 : 0);
-            const int nvalid = key_end - key0;   // scores of this thread that count (<= 0 .. >= 128)
+            // This thread's 64 scores (row m, keys key0 ..) are read from tensor
+            // memory twice: once for the row maximum, once for the weights.
+            const uint32_t s_col = t_lane + kTmemS + 128 * sb + 64 * cg;
+            const int key0 = kPage * t.page0 + (hi ? 128 : 0) + 64 * cg;
+            const int nvalid = key_end - key0;   // scores of this thread that count (<= 0 .. >= 64)
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // independent chains
-#pragma unroll 1
-            for (int q = 0; q < 4; q += 2) {
+            {
                 uint32_t r[2][32];
-                ptx::tmem_ld32(s_col + 32 * q, r[0]);
-                ptx::tmem_ld32(s_col + 32 * q + 32, r[1]);
+                ptx::tmem_ld32(s_col, r[0]);
+                ptx::tmem_ld32(s_col + 32, r[1]);
                 ptx::tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
-                    if (32 * q + j < nvalid) mx4[j & 3] = fmaxf(mx4[j & 3], __uint_as_float(r[j >> 5][j & 31]));
+                    if (j < nvalid) mx4[j & 3] = fmaxf(mx4[j & 3], __uint_as_float(r[j >> 5][j & 31]));
             }
             float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             mx *= p.scale_log2;   // the scale is positive
-            float* xb = xmax + (i & 1) * 128;
-            xb[l] = mx;
-            ptx::named_bar_sync(1, 128);
-            mx = fmaxf(mx, xb[l ^ 64]);
+            xmax[cg * 128 + l] = mx;
+            ptx::named_bar_sync(1, 256);
+            mx = row_max4();
+            ptx::named_bar_sync(2, 256);   // every read done before the buffer is written again
             float new_m = m_used;
             bool resc = false;
             if (mx > m_used + kRescaleThreshold) {
@@ -582,37 +589,35 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             ptx::tc_fence_after();
             if (resc) {
 #pragma unroll 1
-                for (int q = 0; q < 8; ++q) {
+                for (int q = 0; q < 4; ++q) {
                     uint32_t o[32];
-                    ptx::tmem_ld32(t_lane + kTmemO + 32 * q, o);
+                    ptx::tmem_ld32(t_lane + kTmemO + 128 * cg + 32 * q, o);
                     ptx::tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                    ptx::tmem_st32(t_lane + kTmemO + 32 * q, o);
+                    ptx::tmem_st32(t_lane + kTmemO + 128 * cg + 32 * q, o);
                 }
                 ptx::tmem_wait_st();
             }
-            // P row m, keys key0 + [0, 128): blocks of 64 keys, K-major, 128-byte
-            // rows, 128-byte swizzle (16-byte chunk index XOR row & 7)
+            // P row m, keys key0 + [0, 64) = one 64-key block (2 hi + cg) of P:
+            // K-major, 128-byte rows, 128-byte swizzle (16-byte chunk index XOR row & 7)
             float ps2[2] = {0.f, 0.f};
             const float neg_m = -m_used;
-            unsigned char* Prow = smem + kOffP + (hi ? 2 : 0) * kBox + m * 128;
-#pragma unroll 1
-            for (int q = 0; q < 4; q += 2) {   // 64 keys = one 64-key block of P
+            {
                 uint32_t r[2][32];
-                ptx::tmem_ld32(s_col + 32 * q, r[0]);
-                ptx::tmem_ld32(s_col + 32 * q + 32, r[1]);
+                ptx::tmem_ld32(s_col, r[0]);
+                ptx::tmem_ld32(s_col + 32, r[1]);
                 ptx::tmem_wait_ld();
                 uint32_t pk[32];
 #pragma unroll
                 for (int j = 0; j < 64; j += 2) {
                     const float s0 = __uint_as_float(r[j >> 5][j & 31]), s1 = __uint_as_float(r[j >> 5][(j & 31) + 1]);
-                    const float p0 = 32 * q + j < nvalid ? ex2(fmaf(s0, p.scale_log2, neg_m)) : 0.f;
-                    const float p1 = 32 * q + j + 1 < nvalid ? ex2(fmaf(s1, p.scale_log2, neg_m)) : 0.f;
+                    const float p0 = j < nvalid ? ex2(fmaf(s0, p.scale_log2, neg_m)) : 0.f;
+                    const float p1 = j + 1 < nvalid ? ex2(fmaf(s1, p.scale_log2, neg_m)) : 0.f;
                     ps2[(j >> 1) & 1] += p0 + p1;
                     pk[j >> 1] = pack_bf16x2(p0, p1);
                 }
-                unsigned char* Pb = Prow + (q >> 1) * kBox;
+                unsigned char* Pb = smem + kOffP + (2 * hf + cg) * kBox + m * 128;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch)
                     *reinterpret_cast<uint4*>(Pb + ((ch ^ (m & 7)) * 16)) =
@@ -641,7 +646,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 const int bad = kPage - valid;
                 const int et = v_start + (t.np - 1);
                 unsigned char* ent = smem + kOffVRing + (et % kVRing) * kVEntry;
-                for (int x = l; x < 4 * bad * 8; x += 128) {
+                for (int x = st; x < 4 * bad * 8; x += 256) {
                     const int chunk = x / (bad * 8);
                     const int rem = x - chunk * bad * 8;
                     const int row = valid + (rem >> 3), ch = rem & 7;
@@ -653,13 +658,15 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             }
 
             if (t.last) {
-                // ---- epilogue of this unit segment: wait for P.V of this tile
+                // ---- epilogue of this unit segment: wait for P.V of this tile (all
+                // warps' P of this tile is in, so every read of the maxima is done)
                 ok = wait_bar(bar(BAR_P_FREE + 1), i & 1, abort_flag, p.status);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 ptx::tc_fence_after();
-                xsum[l] = l_part;
-                ptx::named_bar_sync(1, 128);
-                const float lsum = l_part + xsum[l ^ 64];
+                xmax[cg * 128 + l] = l_part;   // partial row sums
+                ptx::named_bar_sync(1, 256);
+                const float lsum = xmax[m] + xmax[64 + m] + xmax[128 + m] + xmax[192 + m];
+                ptx::named_bar_sync(2, 256);
                 const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
                 const float lse = lsum > 0.f ? (m_used + __log2f(lsum)) * kLn2 : -INFINITY;
                 const int bt = t.bt, hb = t.hb;
@@ -671,58 +678,55 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 // 4 KB shared-memory tile in the free P buffer (16-byte chunks
                 // swizzled by row), so that each global store instruction writes
                 // whole row segments instead of 32 scattered 16-byte pieces.
-                unsigned char* stage = smem + kOffP + wq * 4096;
+                unsigned char* stage = smem + kOffP + sw * 4096;
                 const size_t grow0 = grow - lane;
                 const size_t prow0 = slot * 128 + head_in_unit - lane;
+                const int h = cg;   // this thread's 128 O columns
+                const int col0 = 128 * h + (hi ? 256 : 0);
 #pragma unroll 1
-                for (int h = 0; h < 2; ++h) {
-                    const int col0 = 128 * h + (hi ? 256 : 0);
-#pragma unroll 1
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t o[32];
-                        ptx::tmem_ld32(t_lane + kTmemO + 128 * h + 32 * q, o);
-                        ptx::tmem_wait_ld();
-                        const int col = col0 + 32 * q;
-                        if (whole) {
-                            // 32 bf16 = 64 B per row, 4 chunks at position k ^ ((row >> 1) & 3)
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t o[32];
+                    ptx::tmem_ld32(t_lane + kTmemO + 128 * h + 32 * q, o);
+                    ptx::tmem_wait_ld();
+                    const int col = col0 + 32 * q;
+                    if (whole) {
+                        // 32 bf16 = 64 B per row, 4 chunks at position k ^ ((row >> 1) & 3)
 #pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                uint4 wv;
-                                wv.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
-                                wv.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
-                                wv.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
-                                wv.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
-                                *reinterpret_cast<uint4*>(stage + lane * 64 + ((k ^ ((lane >> 1) & 3)) * 16)) = wv;
-                            }
-                            __syncwarp();
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const int row = 8 * j + (lane >> 2), k = lane & 3;
-                                const uint4 wv =
-                                    *reinterpret_cast<const uint4*>(stage + row * 64 + ((k ^ ((row >> 1) & 3)) * 16));
-                                *reinterpret_cast<uint4*>(p.out_latent + (grow0 + row) * kDc + col + 8 * k) = wv;
-                            }
-                            __syncwarp();
-                        } else {
-                            // 32 floats = 128 B per row, 8 chunks at position k ^ (row & 7)
-#pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                *reinterpret_cast<float4*>(stage + lane * 128 + ((k ^ (lane & 7)) * 16)) =
-                                    make_float4(__uint_as_float(o[4 * k]) * inv, __uint_as_float(o[4 * k + 1]) * inv,
-                                                __uint_as_float(o[4 * k + 2]) * inv, __uint_as_float(o[4 * k + 3]) * inv);
-                            __syncwarp();
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                const int row = 4 * j + (lane >> 3), k = lane & 7;
-                                const float4 v =
-                                    *reinterpret_cast<const float4*>(stage + row * 128 + ((k ^ (row & 7)) * 16));
-                                *reinterpret_cast<float4*>(p.part_o + (prow0 + row) * kDc + col + 4 * k) = v;
-                            }
-                            __syncwarp();
+                        for (int k = 0; k < 4; ++k) {
+                            uint4 wv;
+                            wv.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
+                            wv.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
+                            wv.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
+                            wv.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
+                            *reinterpret_cast<uint4*>(stage + lane * 64 + ((k ^ ((lane >> 1) & 3)) * 16)) = wv;
                         }
+                        __syncwarp();
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int row = 8 * j + (lane >> 2), k = lane & 3;
+                            const uint4 wv =
+                                *reinterpret_cast<const uint4*>(stage + row * 64 + ((k ^ ((row >> 1) & 3)) * 16));
+                            *reinterpret_cast<uint4*>(p.out_latent + (grow0 + row) * kDc + col + 8 * k) = wv;
+                        }
+                        __syncwarp();
+                    } else {
+                        // 32 floats = 128 B per row, 8 chunks at position k ^ (row & 7)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            *reinterpret_cast<float4*>(stage + lane * 128 + ((k ^ (lane & 7)) * 16)) =
+                                make_float4(__uint_as_float(o[4 * k]) * inv, __uint_as_float(o[4 * k + 1]) * inv,
+                                            __uint_as_float(o[4 * k + 2]) * inv, __uint_as_float(o[4 * k + 3]) * inv);
+                        __syncwarp();
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int row = 4 * j + (lane >> 3), k = lane & 7;
+                            const float4 v = *reinterpret_cast<const float4*>(stage + row * 128 + ((k ^ (row & 7)) * 16));
+                            *reinterpret_cast<float4*>(p.part_o + (prow0 + row) * kDc + col + 4 * k) = v;
+                        }
+                        __syncwarp();
                     }
                 }
-                if (!hi) {
+                if (!hi && cg == 0) {
                     if (whole) p.out_lse[grow] = lse;
                     else p.part_lse[slot * 128 + head_in_unit] = lse;
                 }
