@@ -124,12 +124,13 @@ class ClockSampler:
                 self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(0.001)
 
     def __enter__(self):
         if self.ok:
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
+            time.sleep(0.002)   # the first samples precede the timed work
         return self
 
     def __exit__(self, *a):
