@@ -29,6 +29,14 @@ MUTATIONS = {
     "merge_weights_linear": ("w = np.exp(lse_parts - m)", "w = (lse_parts - m + 1)"),
     "absorb_transposed": ("out[:, i, :] = q_c[:, i, :] @ w_uk[i]",
                           "out[:, i, :] = (q_c[:, i, :] @ w_uk[i])[:, ::-1]"),
+    "up_v_feature_order": ("out[:, i, :] = latent[:, i, :] @ w_uv[i].T",
+                           "out[:, i, :] = latent[:, i, :] @ w_uv[i][::-1].T"),
+    "lse_without_max": ("lse[:, hi] = (m + np.log(z))[:, 0]", "lse[:, hi] = np.log(z)[:, 0]"),
+    "rope_table_cos_sin_swapped": ("return np.concatenate([np.cos(theta), np.sin(theta)], axis=1).astype(np.float32)",
+                                   "return np.concatenate([np.sin(theta), np.cos(theta)], axis=1).astype(np.float32)"),
+    "rope_emulation_sign": ("a = (x1 * c) - (x2 * s)", "a = (x1 * c) + (x2 * s)"),
+    "gather_wrong_slot": ("return int(block_table[b, pos // block_size]), pos % block_size",
+                          "return int(block_table[b, pos // block_size]), (pos + 1) % block_size"),
 }
 
 

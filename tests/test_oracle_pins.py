@@ -308,6 +308,20 @@ def test_gather_through_permuted_block_table():
         rows = O.gather_rows(pool, table, b, 17, bs)
         assert np.array_equal(rows[:, 0], np.full(17, b))
         assert np.array_equal(rows[:, 1], np.arange(17))
+    # worked by hand: sequence 0 owns blocks 7 2 9 0 5, sequence 1 owns 1 8 3 6 4;
+    # token p sits in the table's block p // 4 at slot p % 4
+    assert O.cache_slot(table, 0, 0, bs) == (7, 0)
+    assert O.cache_slot(table, 0, 16, bs) == (5, 0)
+    assert O.cache_slot(table, 1, 5, bs) == (8, 1)
+    assert O.cache_slot(table, 1, 15, bs) == (6, 3)
+    # a pool written without the oracle's index helper gathers back in order
+    pool2 = np.full((nb, bs, 2), -1, dtype=np.int64)
+    for b in range(B):
+        for p in range(17):
+            pool2[table[b][p // bs], p % bs] = [b, p]
+    for b in range(B):
+        rows = O.gather_rows(pool2, table, b, 17, bs)
+        assert np.array_equal(rows[:, 1], np.arange(17)) and (rows[:, 0] == b).all()
 
 
 # --------------------------------------------------------------------------
