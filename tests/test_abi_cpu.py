@@ -92,3 +92,73 @@ def test_host_validation_without_device(M):
     assert raw("mla_decode", *args) == -2           # tcgen05 kernel needs the V2 shape
     assert raw("mla_rope_table", 64, ctypes.c_double(10000.0), 0, p) == -3
     assert raw("mla_clear_status", None, None) == -1
+
+
+def test_rope_append_host_validation(M):
+    raw = M.raw_call
+    cfg = _cfg(M)
+    p = ctypes.c_void_p(FAKE)
+
+    def call(c=cfg, q_r=p, k_r=p, c_kv=p, pos=p, table=p, max_pos=4096, bt=p, mbps=64,
+             pool=p, num_blocks=2048, B=32, T_q=1, status=None):
+        return raw("mla_rope_append", ctypes.byref(c), q_r, k_r, c_kv, pos, table, max_pos, bt, mbps,
+                   pool, num_blocks, B, T_q, status, None)
+
+    assert call(c=_cfg(M, block_size=16)) == -2
+    assert call(c=_cfg(M, d_r=72)) == -2
+    for name in ("k_r", "c_kv", "pos", "table", "bt", "pool"):
+        assert call(**{name: None}) == -1, name
+    odd16 = ctypes.c_void_p(FAKE + 8)               # 8-byte but not 16-byte aligned
+    odd4 = ctypes.c_void_p(FAKE + 2)
+    for name in ("q_r", "k_r", "c_kv", "pool"):
+        assert call(**{name: odd16}) == -7, name
+    for name in ("pos", "table", "bt", "status"):
+        assert call(**{name: odd4}) == -7, name
+    assert call(B=0) == -3 and call(T_q=0) == -3
+    assert call(B=1 << 13, T_q=1 << 12) == -3       # more than 2^24 tokens
+    assert call(max_pos=0) == -3 and call(mbps=0) == -3 and call(num_blocks=0) == -3
+
+
+def test_decode_launch_counts(M):
+    v2 = _cfg(M)
+    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 32, 1, 0) == 3   # schedule, decode, merge
+    # portable kernels: one launch without splits, decode + merge with them
+    simt = _cfg(M, impl=1)
+    assert M.raw_call("mla_decode_launches", ctypes.byref(simt), 32, 1, 1) == 1
+    assert M.raw_call("mla_decode_launches", ctypes.byref(simt), 32, 1, 4) == 2
+    # automatic choice: 32 rows x 16 head groups fill 8 x 148 slots with 3 splits
+    assert M.raw_call("mla_decode_launches", ctypes.byref(simt), 32, 1, 0) == 2
+    assert M.raw_call("mla_decode_launches", ctypes.byref(simt), 4096, 16, 0) == 1
+    tiny = _cfg(M, n_h=4, d_c=64, d_h=32, d_r=16)
+    assert M.raw_call("mla_decode_launches", ctypes.byref(tiny), 1, 1, 0) == 2
+    tiny_tc = _cfg(M, n_h=4, d_c=64, d_h=32, d_r=16, impl=2)
+    assert M.raw_call("mla_decode_launches", ctypes.byref(tiny_tc), 1, 1, 0) == -2
+    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 32, 17, 0) == -3
+    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 0, 1, 0) == -3
+    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 32, 1, -1) == -3
+    # the workspace query answers 0 for arguments the decode call would reject
+    assert M.mla_decode_workspace_bytes(v2, 0, 1, 0) == 0
+    assert M.mla_decode_workspace_bytes(_cfg(M, block_size=32), 32, 1, 0) == 0
+
+
+def test_noalloc_rejects_before_touching_a_device(M):
+    raw = M.raw_call
+    cfg = _cfg(M)
+    p = ctypes.c_void_p(FAKE)
+
+    def call(c=cfg, B=32, T_q=1, splits=2, status=None, **ptrs):
+        a = dict(q_abs=p, q_r=p, pool=p, bt=p, lens=p, out=p, lse=p)
+        a.update(ptrs)
+        return raw("mla_decode_noalloc", ctypes.byref(c), a["q_abs"], a["q_r"], a["pool"], 2048, a["bt"],
+                   64, a["lens"], B, T_q, splits, a["out"], a["lse"], status, None)
+
+    assert call(c=_cfg(M, block_size=32)) == -2
+    for name in ("q_abs", "q_r", "pool", "bt", "lens", "out", "lse"):
+        assert call(**{name: None}) == -1, name
+    assert call(q_abs=ctypes.c_void_p(FAKE + 8)) == -7
+    assert call(status=ctypes.c_void_p(FAKE + 2)) == -7
+    assert call(splits=0) == -3 and call(splits=257) == -3 and call(T_q=17) == -3
+    # 2 splits x 4096 rows x (512 + 1) fp32 is 32 KiB over the fixed 16 MiB array
+    assert 2 * 32 * 128 * (4 * 512 + 4) > 16 << 20
+    assert call(splits=2) == -3
+    assert call(B=8, splits=64) == -3
