@@ -78,7 +78,7 @@ enum {
     MLA_ERR_WORKSPACE = -4,   /* workspace too small or misaligned            */
     MLA_ERR_LAUNCH = -5,      /* a CUDA launch or runtime call failed         */
     MLA_ERR_UNSUPPORTED = -6, /* device is not sm_100 or feature unavailable  */
-    MLA_ERR_ALIGN = -7        /* a pointer breaks the 16-byte alignment rule  */
+    MLA_ERR_ALIGN = -7        /* a pointer breaks its alignment rule (below)  */
 };
 
 /* Device status word bits (see mla_read_status). */
@@ -91,7 +91,9 @@ enum {
 
 /* Constraints shared by every call: d_c, d_r and d_h multiples of 8,
  * 8 <= d_c <= 512, 8 <= d_r <= 64, 8 <= d_h <= 256, block_size = 64,
- * 1 <= n_h <= 1024.  Every tensor pointer 16-byte aligned. */
+ * 1 <= n_h <= 1024.  Pointers to bf16 tensors are 16-byte aligned; pointers
+ * to int32 and float32 arrays (positions, tables, lengths, lse, status) are
+ * 4-byte aligned; the mla_decode workspace is 256-byte aligned. */
 
 /* Human-readable name of a return code. */
 const char* mla_status_str(int code);
