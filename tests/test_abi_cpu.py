@@ -162,3 +162,37 @@ def test_noalloc_rejects_before_touching_a_device(M):
     assert 2 * 32 * 128 * (4 * 512 + 4) > 16 << 20
     assert call(splits=2) == -3
     assert call(B=8, splits=64) == -3
+
+
+@pytest.mark.parametrize("field,value,ok", [
+    ("n_h", 0, False), ("n_h", 1, True), ("n_h", 1024, True), ("n_h", 1025, False),
+    ("d_c", 0, False), ("d_c", 8, True), ("d_c", 12, False), ("d_c", 512, True), ("d_c", 520, False),
+    ("d_r", 0, False), ("d_r", 8, True), ("d_r", 12, False), ("d_r", 64, True), ("d_r", 72, False),
+    ("d_h", 0, False), ("d_h", 8, True), ("d_h", 12, False), ("d_h", 256, True), ("d_h", 264, False),
+    ("block_size", 32, False), ("block_size", 128, False),
+    ("impl", -1, False), ("impl", 3, False),
+    ("scale", float("nan"), False), ("scale", -1.0, True), ("scale", 0.125, True),
+])
+def test_config_limits(M, field, value, ok):
+    """The shape limits the header states, at their boundaries (the launch-count
+    query runs the same configuration check as every compute call)."""
+    cfg = _cfg(M, impl=1)
+    setattr(cfg, field, value)
+    rc = M.raw_call("mla_decode_launches", ctypes.byref(cfg), 4, 1, 0)
+    if ok:
+        assert rc in (1, 2), rc
+        assert M.mla_decode_workspace_bytes(cfg, 4, 1, 0) > 0
+    else:
+        assert rc == -2, rc
+        assert M.mla_decode_workspace_bytes(cfg, 4, 1, 0) == 0
+
+
+def test_rope_table_argument_checks(M):
+    buf = (ctypes.c_float * 64)()
+    assert M.raw_call("mla_rope_table", 16, ctypes.c_double(10000.0), 4, None) == -1
+    for d_r, base, max_pos in ((15, 10000.0, 4), (0, 10000.0, 4), (16, 0.0, 4), (16, -2.0, 4),
+                               (16, float("nan"), 4), (16, 10000.0, 0)):
+        assert M.raw_call("mla_rope_table", d_r, ctypes.c_double(base), max_pos, buf) == -3, (d_r, base, max_pos)
+    assert M.raw_call("mla_rope_table", 16, ctypes.c_double(10000.0), 4, buf) == 0
+    # position 0 is the identity rotation: cos = 1, sin = 0 for every pair
+    assert list(buf[:8]) == [1.0] * 8 and list(buf[8:16]) == [0.0] * 8
