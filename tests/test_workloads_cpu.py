@@ -1,4 +1,9 @@
-"""The benchmark's workloads and roofline arithmetic, checked on the CPU.
+"""The benchmark's workloads, roofline arithmetic and input generator, checked
+on the CPU.
+
+The generator is pinned to SplitMix64's published outputs, its bf16 rounding to
+round-to-nearest-even (ties included), and its torch form (used to fill the
+cache history on the device) to its numpy form (used by the oracle).
 
 The five workloads carry the shapes and lengths of the pages' DeepSeek-V2
 setting ("Техотчёт DeepSeek-V2 (2024): MLA и экономика инференса", "Сколько
@@ -83,3 +88,77 @@ def test_seeded_inputs_are_reproducible_and_keyed():
     whole = s.c_kv_rows(1, 0, 70)
     assert np.array_equal(whole[10:20], s.c_kv_rows(1, 10, 20))
     assert not np.array_equal(whole, s.c_kv_rows(0, 0, 70))
+
+
+def test_splitmix64_matches_its_published_outputs():
+    """SplitMix64 (Steele, Lea and Flood, OOPSLA 2014) from state 0 starts
+    0xe220a8397b1dcdaf, 0x6e789e6aa1b965f4, 0x06c45d188009454f,
+    0xf88bb8a8724c81ec; the counter form used here is output k of the stream
+    seeded with the tensor's key."""
+    gamma = 0x9E3779B97F4A7C15
+    mask = (1 << 64) - 1
+
+    def mix(z):
+        z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & mask
+        z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & mask
+        return z ^ (z >> 31)
+
+    def stream(state, n):
+        out = []
+        for _ in range(n):
+            state = (state + gamma) & mask
+            out.append(mix(state))
+        return out
+
+    assert stream(0, 4) == [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F, 0xF88BB8A8724C81EC]
+    for seed, tid in ((0, 1), (7, 5), (123456789, 8)):
+        key = int(synth._key(seed, tid))
+        got = synth.uniform_u64(seed, tid, np.arange(6, dtype=np.uint64))
+        assert [int(x) for x in got] == stream(key, 6)
+
+
+def test_bf16_rounding_is_nearest_even_in_one_step():
+    r = np.random.default_rng(5)
+    x = np.concatenate([r.standard_normal(20000) * 10.0 ** r.integers(-6, 6, 20000),
+                        # exact halfway points between neighbouring bf16 values: odd
+                        # 9-bit significands 257 .. 511 at a few scales, both signs
+                        np.outer(np.arange(257, 512, 2), 2.0 ** np.array([-20, -9, 0, 7])).ravel(),
+                        -np.outer(np.arange(257, 512, 2), 2.0 ** np.array([-3, 11])).ravel()])
+    bits = synth.to_bf16_bits(x)
+    got = synth.bf16_bits_to_f64(bits)
+    ties = [0]
+    for v, g in zip(x.tolist(), got.tolist()):
+        # neighbours of v with 8 significant bits, in exact float arithmetic
+        m, e = np.frexp(abs(v))                     # v = m 2^e, 0.5 <= m < 1
+        ulp = 2.0 ** (int(e) - 8)
+        lo = np.floor(abs(v) / ulp) * ulp
+        hi = lo + ulp
+        if abs(v) - lo < hi - abs(v):
+            want = lo
+        elif abs(v) - lo > hi - abs(v):
+            want = hi
+        else:                                       # tie: the even significand
+            ties[0] += 1
+            want = lo if int(lo / ulp) % 2 == 0 else hi
+        assert g == np.copysign(want, v), (v, g, want)
+    assert ties[0] == 128 * 6
+
+
+def test_torch_generator_matches_numpy_generator():
+    """The cache history is drawn with the torch form of the generator; the
+    oracle draws the same rows with the numpy form."""
+    torch = pytest.importorskip("torch")
+    for seed, tid, start, count in ((0, 1, 0, 50000), (3, 2, (5 << 20) * 64, 4096), (9, 4, 12345, 777)):
+        a = synth.normal_bf16(seed, tid, (count,), start=start)
+        b = synth.normal_bf16_torch(seed, tid, count, start=start, device="cpu", chunk=1 << 14)
+        b = b.view(torch.int16).numpy().view(np.uint16)
+        assert (a != b).sum() == 0
+
+
+def test_box_muller_normals_have_unit_moments():
+    z = synth.normal_f64(11, 3, 0, 200000)
+    n = z.size
+    assert abs(z.mean()) < 5 / np.sqrt(n)
+    assert abs(z.var() - 1.0) < 5 * np.sqrt(2.0 / n)
+    # a tail fraction: P(|z| > 2) = 0.0455
+    assert abs((np.abs(z) > 2).mean() - 0.0455) < 0.003
