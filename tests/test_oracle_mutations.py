@@ -61,3 +61,36 @@ def test_pins_catch_planted_mistake(name, monkeypatch):
         except Exception:
             failures += 1
     assert failures >= 1, f"no pin caught mutation {name}"
+
+
+# Slips in the per-sequence evaluation that the GPU tests compare against; the
+# brute force of whole workload cases must catch each.
+import tests.test_oracle_brute_force as brute  # noqa: E402
+
+EVAL_SRC = os.path.join(os.path.dirname(SRC), "evaluate.py")
+
+EVAL_MUTATIONS = {
+    "query_rows_of_next_token": ("sl = slice(b * T_q, (b + 1) * T_q)", "sl = slice(b * T_q + 1, (b + 1) * T_q + 1)"),
+    "weights_swapped": ("_CACHE[key] = (O.bf16_to_f64(spec.w_uk()), O.bf16_to_f64(spec.w_uv()))",
+                        "_CACHE[key] = (O.bf16_to_f64(spec.w_uv()), O.bf16_to_f64(spec.w_uk()))"),
+    "rope_query_part_dropped": ("_CACHE[key] = (O.bf16_to_f64(spec.q_c()), O.bf16_to_f64(spec.q_r()))",
+                                "_CACHE[key] = (O.bf16_to_f64(spec.q_c()), 0 * O.bf16_to_f64(spec.q_r()))"),
+    "history_of_other_sequence": ("c = O.bf16_to_f64(spec.c_kv_rows(b, 0, L))",
+                                  "c = O.bf16_to_f64(spec.c_kv_rows(b + 1, 0, L))"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EVAL_MUTATIONS))
+def test_brute_force_catches_planted_evaluation_mistake(name, monkeypatch):
+    old, new = EVAL_MUTATIONS[name]
+    src = open(EVAL_SRC).read()
+    assert src.count(old) == 1, old
+    mod = types.ModuleType("oracle.evaluate_mutant")
+    mod.__package__ = "oracle"
+    exec(compile(src.replace(old, new), "evaluate_mutant", "exec"), mod.__dict__)
+    monkeypatch.setattr(brute, "evaluate", mod)
+    spec = brute.CaseSpec(n_h=2, d_c=16, d_h=8, d_r=8, seq_lens=brute.np.array([5, 23], brute.np.int32),
+                          T_q=3, seed=4)
+    with pytest.raises(Exception):
+        brute._check(spec, 0)
+        brute._check(spec, 1)
