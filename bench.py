@@ -158,6 +158,7 @@ def oracle_sample_rate(spec, steps, warmup, heads_per_step=8, budget_s=None):
     from oracle.evaluate import reference
     b = 0
     heads_all = list(range(spec.n_h))
+    heads_per_step = min(heads_per_step, spec.n_h)
     done_heads, t_total, k = 0, 0.0, 0
     for i in range(warmup + steps):
         hs = [heads_all[(i * heads_per_step + j) % spec.n_h] for j in range(heads_per_step)]

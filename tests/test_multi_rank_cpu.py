@@ -95,3 +95,22 @@ def test_reference_arm_prints_once_under_two_ranks():
     assert d["cpu_baseline"]["value"] == d["value"] and d["cpu_baseline"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_single_process():
+    """`bench.py --impl reference` without torchrun: one JSON line with the
+    contract's keys, the oracle timed on the host's cores."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "2", "--warmup", "1",
+           "--workload", "tiny"]
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 1 and d["steps"] == 2 and d["warmup"] == 1
+    assert d["value"] > 0 and d["ms_per_step"] > 0 and d["unit"] == "tokens/s"
+    assert d["config"]["workload"].startswith("tiny") and d["dtype"] == "f64" and d["data"] == "synthetic"
+    # a sampled step evaluates all 4 heads of the one query token: one token per step
+    assert d["cpu_baseline"]["sample"].startswith("2 steps x 4 of 4 heads")
+    assert d["value"] == pytest.approx(1 / (d["ms_per_step"] / 1e3), rel=1e-6)
