@@ -145,7 +145,8 @@ int mla_rope_append(const mla_config_t* cfg, mla_bf16* q_r, const mla_bf16* k_r,
                     int32_t* dev_status, void* stream);
 
 /* Bytes of workspace mla_decode needs for these sizes (256-byte aligned
- * pointer required).  max_splits as for mla_decode. */
+ * pointer required).  max_splits as for mla_decode.  The size covers only the
+ * kernel family that cfg selects for this shape; 0 for invalid arguments. */
 size_t mla_decode_workspace_bytes(const mla_config_t* cfg, int B, int T_q, int max_splits);
 
 /* Absorbed MLA decode over the paged cache ([v3] eq. (10) with [notes]
@@ -159,9 +160,18 @@ size_t mla_decode_workspace_bytes(const mla_config_t* cfg, int B, int T_q, int m
  *   q_abs (B*T_q, n_h, d_c) bf16;  q_r (B*T_q, n_h, d_r) bf16 (already RoPE'd)
  *   pool, block_table as for mla_rope_append; seq_lens (B) int32, the cache
  *   length AFTER the step's append, 1 <= T_q <= seq_lens[b].
- *   max_splits: upper bound on key-range splits per query row (0 = choose).
- * The key ranges are split across thread blocks; fp32 partial results in the
- * workspace are merged by a log-sum-exp reduction kernel.  The workspace
+ *   max_splits: upper bound on the parts the key range of one query row is
+ *   split into (0 = the library chooses):
+ *     tcgen05 kernels: the pages of all (query row, block of 128 heads) units
+ *       are laid end to end and cut into 74 contiguous ranges, one per pair of
+ *       SMs.  0 cuts them into equal ranges (a unit may span several); s > 0
+ *       moves every cut to the next of the points that divide each unit's P
+ *       pages into min(s, P) near-equal pieces, so no unit lies in more than
+ *       s ranges (1 = no unit is split).  mla_decode_split_counts reports the
+ *       parts each unit got.
+ *     portable kernels: exactly max_splits parts (0: a count from B, T_q, n_h).
+ * Partial results (fp32 latent rows and log-sum-exp) of split rows go to the
+ * workspace and are merged by a log-sum-exp reduction kernel.  The workspace
  * starts with the device status word (mla_read_status).  T_q <= 16. */
 int mla_decode(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q_r,
                const mla_bf16* pool, int num_blocks, const int32_t* block_table,
@@ -172,6 +182,26 @@ int mla_decode(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q
 /* Number of kernel launches one mla_decode call with these arguments makes
  * (decode, optional scheduling and merge kernels); negative on bad arguments. */
 int mla_decode_launches(const mla_config_t* cfg, int B, int T_q, int max_splits);
+
+/* Diagnostic: after an mla_decode call with these arguments has completed on
+ * `stream`, copies to host_counts the number of parts (key-range splits) of
+ * each unit of work, read back from the workspace; synchronises `stream`.
+ * tcgen05 kernels: one count per (query row, block of 128 heads), unit
+ * u = (b * T_q + t) * (n_h / 128) + head block, n_counts = B * T_q * n_h / 128
+ * (0 for a row whose sequence length was invalid).  Portable kernels: the
+ * fixed split count, written to all n_counts entries. */
+int mla_decode_split_counts(const mla_config_t* cfg, int B, int T_q, int max_splits,
+                            const void* workspace, int32_t* host_counts, int n_counts,
+                            void* stream);
+
+/* Test hook for the bounded device waits (no page has a counterpart).  Arms the NEXT mla_decode call that runs the
+ * tcgen05 kernels: that call never issues one of its cache loads, so a
+ * barrier that nothing completes is waited on, and every wait of the call is
+ * bounded by wait_limit_ns (1 ns .. 2 s) instead of 2 s.  The call returns
+ * MLA_OK; the kernel unwinds, sets MLA_STATUS_TIMEOUT in the status word and
+ * releases its tensor memory, and its outputs are undefined.  Later calls run
+ * normally.  Not for production use. */
+int mla_test_arm_decode_timeout(uint64_t wait_limit_ns);
 
 /* mla_decode for callers that cannot allocate device memory: the pages have
  * no counterpart; this is a deployment variant of the same computation.
@@ -192,7 +222,9 @@ int mla_decode_launches(const mla_config_t* cfg, int B, int T_q, int max_splits)
  *               MLA_STATUS_* bits into (NULL: not reported).
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.  All calls share the one array, which
+ * first call before any stream capture.  A cudaDeviceReset invalidates the
+ * cached address: do not call this entry point on a device again after
+ * resetting it in the same process.  All calls share the one array, which
  * keeps the last call's contents (each call fully writes what it reads, so
  * nothing needs clearing); calls that overlap on the GPU, on different streams
  * or from different host threads, race on it and must be serialised by the

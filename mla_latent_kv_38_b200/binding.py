@@ -27,7 +27,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 EXPORTED = (
     "mla_status_str", "mla_check_device", "mla_rope_table", "mla_absorb_q",
     "mla_rope_append", "mla_decode_workspace_bytes", "mla_decode", "mla_decode_launches",
-    "mla_decode_noalloc", "mla_up_v",
+    "mla_decode_noalloc", "mla_decode_split_counts", "mla_test_arm_decode_timeout", "mla_up_v",
     "mla_clear_status", "mla_read_status",
 )
 
@@ -75,6 +75,8 @@ _lib.mla_decode.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, 
 _lib.mla_decode_launches.argtypes = [_cfgp, _i, _i, _i]
 _lib.mla_decode_noalloc.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp,
                                     _vp]
+_lib.mla_decode_split_counts.argtypes = [_cfgp, _i, _i, _i, _vp, _vp, _i, _vp]
+_lib.mla_test_arm_decode_timeout.argtypes = [ctypes.c_uint64]
 _lib.mla_up_v.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp]
 _lib.mla_clear_status.argtypes = [_vp, _vp]
 _lib.mla_read_status.argtypes = [_vp, _vp, _vp]
@@ -159,6 +161,22 @@ def mla_decode_noalloc(cfg: MlaConfig, q_abs, q_r, pool, num_blocks: int, block_
         ctypes.byref(cfg), _ptr(q_abs), _ptr(q_r), _ptr(pool), int(num_blocks), _ptr(block_table),
         int(max_blocks_per_seq), _ptr(seq_lens), int(B), int(T_q), int(splits), _ptr(out_latent),
         _ptr(out_lse), _ptr(dev_status), _stream(stream)))
+
+
+def mla_decode_split_counts(cfg: MlaConfig, B: int, T_q: int, max_splits: int, workspace, n_counts: int,
+                            stream=None):
+    """Parts per unit of work of the last completed mla_decode call (host int32 tensor)."""
+    out = torch.zeros(n_counts, dtype=torch.int32)
+    _check("mla_decode_split_counts", _lib.mla_decode_split_counts(
+        ctypes.byref(cfg), int(B), int(T_q), int(max_splits), _ptr(workspace), out.data_ptr(), int(n_counts),
+        _stream(stream)))
+    return out
+
+
+def mla_test_arm_decode_timeout(wait_limit_ns: int):
+    """Test hook: the next tensor-core mla_decode call withholds one load and
+    bounds its waits by wait_limit_ns (it then reports MLA_STATUS_TIMEOUT)."""
+    _check("mla_test_arm_decode_timeout", _lib.mla_test_arm_decode_timeout(int(wait_limit_ns)))
 
 
 def mla_up_v(cfg: MlaConfig, latent, w_uv, out, n_tok: int, stream=None):

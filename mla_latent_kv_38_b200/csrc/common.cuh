@@ -46,23 +46,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// 2^x on the FMA pipe, for x <= 64 (x is clamped below at -126): x = n + f with
-// n = round(x) (the 1.5 * 2^23 shift), 2^f for f in [-0.5, 0.5] from a cubic
-// fitted here by weighted least squares (max relative error 7.5e-5, far below
-// a bf16 ulp), and n added to the exponent field.  Used where the
-// special-function unit's exp2 throughput would be the bottleneck.
-__device__ __forceinline__ float exp2_fma(float x) {
-    x = fmaxf(x, -126.f);
-    const float t = x + 12582912.f;
-    const float n = t - 12582912.f;
-    const float f = x - n;
-    float p = fmaf(f, 0.05517132f, 0.24261054f);
-    p = fmaf(p, f, 0.69326097f);
-    p = fmaf(p, f, 0.99992812f);
-    const int e = __float_as_int(t) - 0x4B400000;
-    return __int_as_float(__float_as_int(p) + (e << 23));
-}
-
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

@@ -11,7 +11,10 @@
 // The host cannot use the array's name as a device address: in host code it
 // only names a host-side stand-in.  The device address is looked up once per
 // device with cudaGetSymbolAddress, with that device current, the first time
-// the entry point runs on it, and cached.
+// the entry point runs on it, and cached.  The cached address belongs to the
+// device's context of that moment: after a cudaDeviceReset the module is
+// loaded again and the array may sit elsewhere, so a process that resets a
+// device must not call this entry point on that device again.
 
 #include <math.h>
 
@@ -55,11 +58,8 @@ extern "C" int mla_decode_noalloc(const mla_config_t* cfg, const mla_bf16* q_abs
                                   int max_blocks_per_seq, const int32_t* seq_lens, int B, int T_q,
                                   int splits, mla_bf16* out_latent, float* out_lse,
                                   int32_t* dev_status, void* stream) {
-    if (cfg == nullptr) return MLA_ERR_NULL;
-    if (cfg->n_h < 1 || cfg->n_h > 1024 || cfg->d_c < 8 || cfg->d_c > 512 || cfg->d_c % 8 ||
-        cfg->d_r < 8 || cfg->d_r > 64 || cfg->d_r % 8 || cfg->d_h < 8 || cfg->d_h > 256 ||
-        cfg->d_h % 8 || cfg->block_size != 64 || !(cfg->scale == cfg->scale))
-        return MLA_ERR_CONFIG;
+    const int rc_cfg = mla::check_config(cfg);   // the same checks as every other entry point
+    if (rc_cfg != MLA_OK) return rc_cfg;
     if (!q_abs || !q_r || !pool || !block_table || !seq_lens || !out_latent || !out_lse)
         return MLA_ERR_NULL;
     if (!al16(q_abs) || !al16(q_r) || !al16(pool) || !al16(out_latent) || !al4(out_lse) ||
@@ -102,9 +102,7 @@ extern "C" int mla_decode_noalloc(const mla_config_t* cfg, const mla_bf16* q_abs
     P.T_q = T_q;
     P.n_tok = B * T_q;
     P.splits = splits;
-    const float scale = cfg->scale > 0.f ? cfg->scale
-                                         : static_cast<float>(1.0 / sqrt(static_cast<double>(cfg->d_h + cfg->d_r)));
-    P.scale_log2 = scale * mla::kLog2e;
+    P.scale_log2 = mla::effective_scale(cfg) * mla::kLog2e;
     return mla::launch_decode_simt(P, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MLA_OK
                                                                                           : MLA_ERR_LAUNCH;
 }

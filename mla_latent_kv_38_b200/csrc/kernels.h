@@ -5,7 +5,15 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "mla.h"
+
 namespace mla {
+
+// Host-side argument checks shared by every entry point: MLA_OK or the
+// MLA_ERR_* code for an unsupported configuration, and the score scale that
+// cfg->scale selects (1/sqrt(d_h + d_r) when it is <= 0).
+int check_config(const mla_config_t* cfg);
+float effective_scale(const mla_config_t* cfg);
 
 struct DecodeParams;
 

@@ -22,6 +22,49 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+int choose_splits(const mla_config_t* c, int B, int T_q, int max_splits) {
+    if (max_splits > 0) return max_splits < kMaxSplits ? max_splits : kMaxSplits;
+    const long work = static_cast<long>(B) * T_q * ((c->n_h + 7) / 8);
+    long s = (8L * kB200Sms + work - 1) / work;
+    if (s < 1) s = 1;
+    if (s > 64) s = 64;
+    return static_cast<int>(s);
+}
+
+bool uses_sm100(const mla_config_t* c) {
+    const bool shape = mla::sm100_supports(c->n_h, c->d_c, c->d_r);
+    return c->impl == 2 || (c->impl == 0 && shape);
+}
+
+// Workspace: the status word (256 bytes), then the region of the kernel family
+// that will run -- the portable kernel's split partials, or the tcgen05
+// kernels' schedule arrays and partial slots.
+struct WsLayout {
+    size_t part_o, part_lse, sm100, total;
+};
+
+WsLayout ws_layout(const mla_config_t* c, int B, int T_q, int max_splits) {
+    WsLayout w;
+    w.part_o = w.part_lse = w.sm100 = 256;
+    if (uses_sm100(c)) {
+        w.total = w.sm100 + round256(mla::sm100_workspace_bytes(c->n_h, c->d_c, B, T_q));
+        return w;
+    }
+    const int splits = choose_splits(c, B, T_q, max_splits);
+    const size_t rows = static_cast<size_t>(B) * T_q * c->n_h;
+    const size_t simt_o = splits > 1 ? round256(static_cast<size_t>(splits) * rows * c->d_c * 4) : 0;
+    const size_t simt_l = splits > 1 ? round256(static_cast<size_t>(splits) * rows * 4) : 0;
+    w.part_lse = w.part_o + simt_o;
+    w.total = w.part_lse + simt_l;
+    return w;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_LAUNCH; }
+
+}  // namespace
+
+namespace mla {
+
 int check_config(const mla_config_t* c) {
     if (c == nullptr) return MLA_ERR_NULL;
     if (c->n_h < 1 || c->n_h > 1024) return MLA_ERR_CONFIG;
@@ -38,34 +81,10 @@ float effective_scale(const mla_config_t* c) {
     return c->scale > 0.f ? c->scale : static_cast<float>(1.0 / sqrt(static_cast<double>(c->d_h + c->d_r)));
 }
 
-int choose_splits(const mla_config_t* c, int B, int T_q, int max_splits) {
-    if (max_splits > 0) return max_splits < kMaxSplits ? max_splits : kMaxSplits;
-    const long work = static_cast<long>(B) * T_q * ((c->n_h + 7) / 8);
-    long s = (8L * kB200Sms + work - 1) / work;
-    if (s < 1) s = 1;
-    if (s > 64) s = 64;
-    return static_cast<int>(s);
-}
+}  // namespace mla
 
-struct WsLayout {
-    size_t part_o, part_lse, sm100, total;
-};
-
-WsLayout ws_layout(const mla_config_t* c, int B, int T_q, int splits) {
-    WsLayout w;
-    const size_t rows = static_cast<size_t>(B) * T_q * c->n_h;
-    const size_t simt_o = splits > 1 ? round256(static_cast<size_t>(splits) * rows * c->d_c * 4) : 0;
-    const size_t simt_l = splits > 1 ? round256(static_cast<size_t>(splits) * rows * 4) : 0;
-    w.part_o = 256;
-    w.part_lse = w.part_o + simt_o;
-    w.sm100 = w.part_lse + simt_l;
-    w.total = w.sm100 + round256(mla::sm100_workspace_bytes(c->n_h, c->d_c, B, T_q));
-    return w;
-}
-
-int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_LAUNCH; }
-
-}  // namespace
+using mla::check_config;
+using mla::effective_scale;
 
 extern "C" {
 
@@ -152,7 +171,8 @@ int mla_rope_append(const mla_config_t* cfg, mla_bf16* q_r, const mla_bf16* k_r,
 
 size_t mla_decode_workspace_bytes(const mla_config_t* cfg, int B, int T_q, int max_splits) {
     if (check_config(cfg) || B < 1 || T_q < 1 || max_splits < 0) return 0;
-    return ws_layout(cfg, B, T_q, choose_splits(cfg, B, T_q, max_splits)).total;
+    if (cfg->impl == 2 && !mla::sm100_supports(cfg->n_h, cfg->d_c, cfg->d_r)) return 0;
+    return ws_layout(cfg, B, T_q, max_splits).total;
 }
 
 int mla_decode(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q_r,
@@ -170,8 +190,11 @@ int mla_decode(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q
     if (B < 1 || T_q < 1 || T_q > 16 || static_cast<long>(B) * T_q > 65535) return MLA_ERR_SIZE;
     if (num_blocks < 1 || max_blocks_per_seq < 1 || max_splits < 0) return MLA_ERR_SIZE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLA_ERR_WORKSPACE;
-    const int splits = choose_splits(cfg, B, T_q, max_splits);
-    const WsLayout w = ws_layout(cfg, B, T_q, splits);
+    const bool sm100_shape = mla::sm100_supports(cfg->n_h, cfg->d_c, cfg->d_r);
+    if (cfg->impl == 2 && !sm100_shape) return MLA_ERR_CONFIG;
+    const bool use_sm100 = uses_sm100(cfg);
+    const int splits = use_sm100 ? 0 : choose_splits(cfg, B, T_q, max_splits);
+    const WsLayout w = ws_layout(cfg, B, T_q, max_splits);
     if (ws_bytes < w.total) return MLA_ERR_WORKSPACE;
 
     char* ws = static_cast<char*>(workspace);
@@ -199,9 +222,6 @@ int mla_decode(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q
     P.scale_log2 = effective_scale(cfg) * mla::kLog2e;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    const bool sm100_shape = mla::sm100_supports(cfg->n_h, cfg->d_c, cfg->d_r);
-    if (cfg->impl == 2 && !sm100_shape) return MLA_ERR_CONFIG;
-    const bool use_sm100 = cfg->impl == 2 || (cfg->impl == 0 && sm100_shape);
     if (use_sm100) {
         if (mla_check_device() != MLA_OK) return MLA_ERR_UNSUPPORTED;
         return cuda_rc(mla::launch_decode_sm100(P, ws + w.sm100, max_splits, st));
@@ -216,8 +236,38 @@ int mla_decode_launches(const mla_config_t* cfg, int B, int T_q, int max_splits)
     const bool sm100_shape = mla::sm100_supports(cfg->n_h, cfg->d_c, cfg->d_r);
     if (cfg->impl == 2 && !sm100_shape) return MLA_ERR_CONFIG;
     if (cfg->impl == 2 || (cfg->impl == 0 && sm100_shape))
-        return mla::sm100_launches(B, T_q, max_splits);
+        return mla::sm100_launches(B, T_q, cfg->n_h);
     return choose_splits(cfg, B, T_q, max_splits) > 1 ? 2 : 1;
+}
+
+int mla_decode_split_counts(const mla_config_t* cfg, int B, int T_q, int max_splits, const void* workspace,
+                            int32_t* host_counts, int n_counts, void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!workspace || !host_counts) return MLA_ERR_NULL;
+    if (B < 1 || T_q < 1 || T_q > 16 || max_splits < 0) return MLA_ERR_SIZE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (!uses_sm100(cfg)) {
+        const int s = choose_splits(cfg, B, T_q, max_splits);
+        for (int i = 0; i < n_counts; ++i) host_counts[i] = s;
+        return cuda_rc(cudaStreamSynchronize(st));
+    }
+    if (!mla::sm100_supports(cfg->n_h, cfg->d_c, cfg->d_r)) return MLA_ERR_CONFIG;
+    const int U = B * T_q * (cfg->n_h / 128);
+    if (n_counts != U) return MLA_ERR_SIZE;
+    const WsLayout w = ws_layout(cfg, B, T_q, max_splits);
+    const char* meta = static_cast<const char*>(workspace) + w.sm100 + mla::sm100_unit_meta_offset(cfg->n_h, B, T_q);
+    // the .z field (parts) of each int4 {kv_len, first cluster, parts, sequence}
+    cudaError_t e = cudaMemcpy2DAsync(host_counts, sizeof(int32_t), meta + 2 * sizeof(int32_t), 4 * sizeof(int32_t),
+                                      sizeof(int32_t), static_cast<size_t>(U), cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return MLA_ERR_LAUNCH;
+    return cuda_rc(cudaStreamSynchronize(st));
+}
+
+int mla_test_arm_decode_timeout(uint64_t wait_limit_ns) {
+    if (wait_limit_ns == 0 || wait_limit_ns > 2000000000ull) return MLA_ERR_SIZE;
+    mla::sm100_arm_timeout_test(wait_limit_ns);
+    return MLA_OK;
 }
 
 int mla_up_v(const mla_config_t* cfg, const mla_bf16* latent, const mla_bf16* w_uv, mla_bf16* out,

@@ -24,23 +24,33 @@
 //    runs as 2 x N = 256 per 16 keys: the B operand is split by latent
 //    columns, so each CTA loads all 4 pages of its 256 latent columns (these
 //    second reads hit L2).
-//  * All operands arrive by TMA (128-byte swizzle) in two rings, each with one
-//    producer warp and one in-order MMA consumer: S entries of 24 KB (one
-//    column chunk of the CTA's 2 pages plus the same chunk of its 64 query
-//    rows, re-read from L2 each tile so that no 72 KB query buffer has to stay
-//    resident) and V entries of 32 KB (the CTA's 4 latent chunks of one page,
-//    one 3-D box).
-//  * Warp roles per CTA: warp 0 S producer, warp 1 tensor-memory allocation
-//    and (CTA 0) the S MMAs, warps 2-5 softmax and epilogue (one thread per
-//    tensor-memory lane), warp 6 (CTA 0) the P.V MMAs, warp 7 V producer.  S
-//    is double buffered; P is written to shared memory in two key halves, each
-//    released as soon as its MMAs complete, so the next tile's softmax overlaps
-//    P.V.  The running max is rescaled lazily (only when it grows by 2^8).
+//  * The query block of a unit (64 heads x 576 columns per CTA, 72 KB) stays
+//    in shared memory for the whole unit segment; a new segment reloads it one
+//    64-column chunk at a time, each chunk as soon as the last S MMA that read
+//    the old one has completed.  The cache arrives by TMA (128-byte swizzle) in
+//    two rings, each with one producer warp and one in-order MMA consumer:
+//    16 KB S entries (one 64-column chunk of the CTA's 2 pages) and 16 KB V
+//    entries (2 latent chunks of one page, one 3-D box).
+//  * An otherwise idle warp of the second CTA issues bulk L2 prefetches of the
+//    cluster's pages a fixed number of tiles ahead of the loads, so that HBM
+//    streams at full rate while the MMA / softmax pipeline fills, drains and
+//    crosses unit segments.
+//  * Warp roles per CTA: warp 0 S producer (query and key chunks), warp 1
+//    tensor-memory allocation and (CTA 0) the S MMAs, warp 2 (CTA 0) the P.V
+//    MMAs / (CTA 1) the L2 prefetcher, warp 3 V producer, warps 4-11 softmax
+//    and epilogue (two warps per tensor-memory lane quadrant).  S is double
+//    buffered; P is written to shared memory in two key halves, each released
+//    as soon as its MMAs complete.  The running max is rescaled lazily (only
+//    when it grows by 2^8).
 //  * Work: the pages of all (sequence, token, head block) units are laid end
-//    to end and cut into equal contiguous ranges, one per cluster (persistent,
-//    74 clusters on 148 SMs).  A unit covered by one cluster is written
-//    directly in bf16; otherwise each cluster writes an fp32 partial and its
-//    log-sum-exp, merged by a reduction kernel.
+//    to end and cut into contiguous ranges, one per cluster (persistent, 74
+//    clusters on 148 SMs).  Each CTA computes the cut from the sequence
+//    lengths itself (a block-wide scan), so no separate scheduling launch
+//    precedes the decode unless the unit count is very large.  A bound on the
+//    parts per unit moves each cut to the next allowed split point.  A unit
+//    covered by one cluster is written directly in bf16; otherwise each
+//    cluster writes an fp32 partial and its log-sum-exp, merged by a
+//    reduction kernel.
 //  * Every mbarrier wait is bounded by the global timer: on expiry the kernel
 //    sets MLA_STATUS_TIMEOUT and unwinds instead of hanging.
 
@@ -55,47 +65,59 @@
 namespace mla {
 namespace {
 
-constexpr int kThreads = 384;   // 12 warps: S loads, S MMAs, P.V MMAs, V loads, 8 x softmax
+constexpr int kThreads = 384;   // 12 warps: S loads, S MMAs, P.V MMAs / prefetch, V loads, 8 x softmax
 constexpr int kClusters = 74;                     // 148 SMs / 2
 constexpr int kDc = 512, kDr = 64, kRow = 576;    // row = c^KV || k^R
 constexpr int kPage = 64;                         // cache rows per page (TMA box height)
 constexpr int kTilePages = 4;                     // a tile = 4 pages = 256 keys (MMA N)
-constexpr int kSRing = 4;                         // 24 KB entries, S operand stream
-constexpr int kVRing = 3;                         // 32 KB entries (one page), P.V operand stream
+constexpr int kChunks = 9;                        // 64-column chunks of a row (8 latent + 1 RoPE)
+constexpr int kSRing = 4;                         // 16 KB entries, S operand stream
+constexpr int kVRing = 3;                         // 16 KB entries, P.V operand stream
+constexpr int kPrefetchAhead = 2;                 // tiles the L2 prefetcher runs ahead of the S loads
+constexpr uint32_t kPageBytes = kPage * kRow * 2; // 73,728
 
 constexpr uint32_t kBox = 8192;                   // one page x 64 columns (128 B rows)
-constexpr uint32_t kSEntry = 3 * kBox;            // S ring entry: a column chunk of the CTA's 2 pages + of its 64 heads' query
-constexpr uint32_t kVEntry = 4 * kBox;            // V ring entry: 4 latent chunks of one page
+constexpr uint32_t kSEntry = 2 * kBox;            // chunk c of the CTA's 2 pages
+constexpr uint32_t kVEntry = 2 * kBox;            // 2 latent chunks of one page
 constexpr uint32_t kPBytes = 4 * kBox;            // 64 heads x 256 keys (4 blocks of 64 keys)
-constexpr uint32_t kOffSRing = 0;
+constexpr uint32_t kOffQ = 0;                     // 9 chunks of the CTA's 64 query rows
+constexpr uint32_t kOffSRing = kOffQ + kChunks * kBox;
 constexpr uint32_t kOffVRing = kOffSRing + kSRing * kSEntry;
 constexpr uint32_t kOffP = kOffVRing + kVRing * kVEntry;
 constexpr uint32_t kOffXmax = kOffP + kPBytes;    // 4 x 64 floats: partial row maxima (or sums)
 constexpr uint32_t kOffBar = kOffXmax + 1024;
-constexpr uint32_t kOffMisc = kOffBar + 8 * 32;   // tmem base, abort flag
-constexpr uint32_t kSmemUsed = kOffMisc + 16;
-// Dynamic shared memory: the buffers above from a 1024-byte aligned base; what
-// the alignment leaves over at the end holds a copy of the cluster's unit
-// prefix when it fits.
+constexpr uint32_t kMaxBars = 40;
+constexpr uint32_t kOffMisc = kOffBar + 8 * kMaxBars;   // tmem base, abort flag, progress counter
+constexpr uint32_t kOffCuts = kOffMisc + 64;      // cluster boundaries (75 ints)
+constexpr uint32_t kOffSlice = kOffCuts + 320;    // key counts of the cluster's units
+// Dynamic shared memory: the buffers above from a 1024-byte aligned base.
 constexpr uint32_t kSmemBytes = 232448;
-static_assert(kSmemUsed + 1024 <= kSmemBytes, "shared memory budget");
+constexpr int kSliceCap = static_cast<int>((kSmemBytes - 1024 - kOffSlice) / 4);
+// Units up to which every CTA computes the schedule itself (the scan's scratch
+// is the ring area, and the cluster's prefix slice always fits in shared memory).
+constexpr int kInKernelUnits = 2048;
+static_assert(kOffSlice + 4 * (kInKernelUnits + 1) + 1024 <= kSmemBytes, "shared memory budget");
+static_assert(4 * (kInKernelUnits + 1 + kClusters + 1) <= static_cast<int>(kOffP - kOffSRing), "schedule scratch");
+static_assert(4 * (kClusters + 1) <= 320, "cut area");
+static_assert(kSRing <= kChunks, "query chunk reuse needs the S ring to be at most one tile deep");
 
 enum {
     BAR_SR_FULL = 0,                         // + slot (leader: both CTAs' bytes)
     BAR_SR_EMPTY = BAR_SR_FULL + kSRing,     // + slot (each CTA, MMA commit)
     BAR_VR_FULL = BAR_SR_EMPTY + kSRing,
     BAR_VR_EMPTY = BAR_VR_FULL + kVRing,
-    BAR_S_FULL = BAR_VR_EMPTY + kVRing,      // + S buffer
-    BAR_S_FREE = BAR_S_FULL + 2,             // + S buffer (leader, 8 warps)
-    BAR_P_FULL = BAR_S_FREE + 2,             // + P half (leader, 2 warps x 2 CTAs)
+    BAR_Q_FULL = BAR_VR_EMPTY + kVRing,      // + chunk (leader: both CTAs' query bytes)
+    BAR_S_FULL = BAR_Q_FULL + kChunks,       // + S buffer
+    BAR_S_FREE = BAR_S_FULL + 2,             // + S buffer (leader, 8 warps x 2 CTAs)
+    BAR_P_FULL = BAR_S_FREE + 2,             // + P half (leader, 4 warps x 2 CTAs)
     BAR_P_FREE = BAR_P_FULL + 2,             // + P half (each CTA, MMA commit)
     BAR_TAIL_READY = BAR_P_FREE + 2,         // each CTA, MMA thread arrives remotely
-    BAR_TAIL_DONE = BAR_TAIL_READY + 1,      // leader, 8 warps
+    BAR_TAIL_DONE = BAR_TAIL_READY + 1,      // leader, 8 warps x 2 CTAs
     BAR_DRAIN = BAR_TAIL_DONE + 1,           // S issuer's own drain on abort
     BAR_DRAIN_PV = BAR_DRAIN + 1,            // P.V issuer's
     NUM_BARS = BAR_DRAIN_PV + 1
 };
-static_assert(NUM_BARS <= 32, "barrier area");
+static_assert(NUM_BARS <= static_cast<int>(kMaxBars), "barrier area");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;                    // 2 x 128 columns (paired layout)
@@ -104,38 +126,42 @@ constexpr uint32_t kTmemS = 256;                  // 2 x 128 columns
 constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 256, 0, 0);
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 256, 0, 1);
 
-constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint32_t kSuspendHintNs = 100000;      // a waiting thread sleeps up to 0.1 ms per try
-constexpr int kSchedSmemUnits = 8192;             // units whose prefix the schedule keeps in shared memory
+constexpr int kSchedSmemUnits = 8192;             // units whose prefix the schedule kernel keeps in shared memory
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
 
 struct Sm100Params {
     CUtensorMap tm_pool;      // pool as [rows][576], box 64 cols x 64 rows
-    CUtensorMap tm_pool_v;    // pool as [chunk][rows][64], box 64 cols x 64 rows x 4 chunks
+    CUtensorMap tm_pool_v;    // pool as [chunk][rows][64], box 64 cols x 64 rows x 2 chunks
     CUtensorMap tm_qa;        // q_abs as [n_tok*n_h][512], box 64 x 64
     CUtensorMap tm_qr;        // q_r   as [n_tok*n_h][64],  box 64 x 64
-    const uint16_t* pool;     // for L2 prefetches of whole pages
+    const uint16_t* pool;     // for the L2 prefetches of whole pages
     const int32_t* block_table;
-    const int32_t* prefix;    // (U + 1) exclusive prefix of pages per unit
-    const int4* unit_meta;    // (U) {kv_len, first cluster, parts, batch index}
-    const int4* cluster_info; // (C) {first page, end page, first unit, last unit}
+    const int32_t* seq_lens;
+    int32_t* prefix;          // (U + 1) exclusive prefix of pages per unit (schedule kernel only)
+    int32_t* unit_kv;         // (U) keys per unit (schedule kernel only)
+    int4* unit_meta;          // (U) {kv_len, first cluster, parts, sequence}
+    const int4* cluster_info; // (C) {first page, end page, first unit, last unit} (schedule kernel only)
     uint16_t* out_latent;
     float* out_lse;
     float* part_o;            // (C + U) slots x 128 rows x 512
     float* part_lse;          // (C + U) slots x 128
     int32_t* status;
-    int n_h, n_hb, T_q, U, C, num_blocks, max_blocks;
+    int n_h, n_hb, B, T_q, U, num_blocks, max_blocks, max_splits;
+    int in_kernel_schedule;   // 1: each CTA computes the schedule; 0: the schedule kernel did
+    int withhold_load;        // test hook: 1 = never issue the first S entry's load of CTA 0
+    uint64_t timeout_ns;      // bound of every wait
     float scale_log2;
 };
 
 __device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, volatile int* abort_flag,
-                                         int32_t* status) {
+                                         int32_t* status, uint64_t timeout_ns) {
     if (ptx::mbar_try_wait(addr, parity)) return true;
     const uint64_t t0 = ptx::global_timer_ns();
     while (true) {
         if (ptx::mbar_try_wait_suspend(addr, parity, kSuspendHintNs)) return true;
         if (*abort_flag) return false;
-        if (ptx::global_timer_ns() - t0 > kTimeoutNs) {
+        if (ptx::global_timer_ns() - t0 > timeout_ns) {
             *abort_flag = 1;
             raise_status(status, MLA_STATUS_TIMEOUT);
             return false;
@@ -143,7 +169,104 @@ __device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, volatil
     }
 }
 
-// Unit whose page range contains global page g (prefix is non-decreasing).
+// ---------------------------------------------------------------------------
+// Work schedule.  Unit u = (b T_q + t) n_hb + hb covers the keys 0 .. kv - 1
+// of query row (b, t), kv = L_b - T_q + t + 1, i.e. ceil(kv / 64) pages; a
+// sequence whose length is out of range has no pages (its outputs are
+// defined as zero / -inf by the merge kernel).  pf is the exclusive prefix of
+// the page counts, T = pf[U] the total.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ int unit_keys(const int32_t* seq_lens, int u, int n_hb, int T_q, int max_blocks) {
+    const int bt = u / n_hb;
+    const int b = bt / T_q;
+    const int t = bt - b * T_q;
+    const int L = __ldg(seq_lens + b);
+    return (L >= T_q && L <= max_blocks * kPage) ? L - T_q + t + 1 : 0;
+}
+
+// Last unit v with pf[v] <= g (for g < T: the unit holding page g).
+__device__ __forceinline__ int unit_of_page(const int32_t* pf, int U, int g) {
+    int lo = 0, hi = U - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pf[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Raw cut c: floor(c T / C).  Without a bound on the parts per unit that is
+// the cut (equal ranges); with max_splits = s > 0 it moves up to the next
+// allowed cut, where unit u's P pages are cut into k = min(s, P) pieces at
+// pf[u] + floor(j P / k), j = 0 .. k, so no unit lies in more than s ranges.
+__device__ int raw_cut(int c, int T, const int32_t* pf, int U, int max_splits) {
+    if (c <= 0) return 0;
+    if (c >= kClusters) return T;
+    const int g = static_cast<int>(static_cast<long long>(c) * T / kClusters);
+    if (max_splits <= 0 || g >= T) return g;
+    const int u = unit_of_page(pf, U, g);
+    const int a = pf[u], P = pf[u + 1] - a;   // a <= g < pf[u + 1], so P > 0
+    const int k = min(max_splits, P);
+    const int j = static_cast<int>((static_cast<long long>(g - a) * k + P - 1) / P);   // ceil((g-a) k / P)
+    return a + static_cast<int>(static_cast<long long>(j) * P / k);
+}
+
+// Cluster boundaries cuts[0 .. C]: the distinct raw cuts in order, then T
+// repeated, so cluster c covers pages [cuts[c], cuts[c + 1]) and every
+// non-empty range comes before every empty one (a unit's ranges are always
+// consecutive clusters).  All threads of the block call it; tmp holds C + 1
+// ints of scratch.
+__device__ void compute_cuts(int* cuts, int* tmp, const int32_t* pf, int U, int T, int max_splits) {
+    for (int c = threadIdx.x; c <= kClusters; c += blockDim.x) tmp[c] = raw_cut(c, T, pf, U, max_splits);
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        constexpr int kPer = (kClusters + 1 + 31) / 32;
+        int n = 0;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int c = lane * kPer + k;
+            if (c <= kClusters && (c == 0 || tmp[c] != tmp[c - 1])) ++n;
+        }
+        int x = n;   // inclusive warp scan of the distinct counts
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        const int total = __shfl_sync(0xffffffffu, x, 31);
+        int pos = x - n;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int c = lane * kPer + k;
+            if (c <= kClusters && (c == 0 || tmp[c] != tmp[c - 1])) cuts[pos++] = tmp[c];
+        }
+        for (int c = total + lane; c <= kClusters; c += 32) cuts[c] = T;
+    }
+    __syncthreads();
+}
+
+// Cluster whose range holds page g < T (the last cluster starting at or before g).
+__device__ int cluster_of_page(int g, const int* cuts) {
+    int lo = 0, hi = kClusters - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cuts[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Merge metadata of unit u: {kv_len, first cluster, parts, sequence}.
+__device__ int4 unit_meta_of(int u, const int32_t* pf, const int* cuts, const int32_t* seq_lens, int n_hb,
+                             int T_q, int max_blocks) {
+    const int kv = unit_keys(seq_lens, u, n_hb, T_q, max_blocks);
+    const int b = u / n_hb / T_q;
+    const int a = pf[u], e = pf[u + 1];
+    if (e <= a) return make_int4(0, 0, 0, b);
+    const int c0 = cluster_of_page(a, cuts);
+    const int c1 = cluster_of_page(e - 1, cuts);
+    return make_int4(kv, c0, c1 - c0 + 1, b);
+}
 
 // One tile of a cluster's work: up to 4 consecutive pages of one unit.
 struct Tile {
@@ -151,24 +274,31 @@ struct Tile {
     int bt;         // query row b T_q + t of the unit
     int hb;         // head block of the unit
     int b;          // sequence of the unit
+    int kv;         // keys of the unit (kv_len)
     int page0;      // first page, within the unit
     int np;         // pages in this tile (1..4)
-    bool first;     // first tile of a unit segment (new Q, O starts from zero)
+    bool first;     // first tile of a unit segment (new query, O starts from zero)
     bool last;      // last tile of a unit segment (epilogue follows)
     bool unit_end;  // the unit's last page is in this tile
+    bool whole;     // the whole unit lies in this cluster's range (no partial)
 };
 
-// Walks a cluster's pages [g0, g1) as tiles.  The prefix entry of unit v is
-// pf[v - off] (pf: a shared-memory copy of the cluster's range of the prefix,
-// or the global array with off = 0).  The unit's (query row, head block,
-// sequence) are kept up to date incrementally, without divisions.
+// Walks a cluster's pages [g0, g1) as tiles.  kvs[v - off] is the key count
+// of unit v (a shared-memory slice of the cluster's units, or a global array
+// with off = 0); unit u0 starts at global page ubeg0.  The unit's page range
+// and (query row, head block, sequence) are kept up to date incrementally.
 struct TileWalker {
-    const int32_t* pf;
-    int off, g, g0, g1, u;
+    const int32_t* kvs;
+    int off, g, g0, g1, u, ubeg, uend, kv;
     int bt, hb, b, t, n_hb, T_q;
-    __device__ int prefix(int v) const { return pf[v - off]; }
+    __device__ void load_unit() {
+        kv = kvs[u - off];
+        uend = ubeg + (kv + kPage - 1) / kPage;
+    }
     __device__ void step_unit() {
         ++u;
+        ubeg = uend;
+        load_unit();
         if (++hb == n_hb) {
             hb = 0;
             ++bt;
@@ -178,8 +308,8 @@ struct TileWalker {
             }
         }
     }
-    __device__ void init(const int32_t* pf_, int off_, int u0, int g0_, int g1_, int n_hb_, int T_q_) {
-        pf = pf_;
+    __device__ void init(const int32_t* kvs_, int off_, int u0, int ubeg0, int g0_, int g1_, int n_hb_, int T_q_) {
+        kvs = kvs_;
         off = off_;
         g = g0_;
         g0 = g0_;
@@ -187,36 +317,84 @@ struct TileWalker {
         n_hb = n_hb_;
         T_q = T_q_;
         u = u0;
+        ubeg = ubeg0;
         bt = u0 / n_hb;
         hb = u0 - bt * n_hb;
         b = bt / T_q;
         t = bt - b * T_q;
-        while (g < g1 && prefix(u + 1) <= g) step_unit();
+        if (g < g1) {
+            load_unit();
+            while (g < g1 && uend <= g) step_unit();
+        }
     }
     __device__ bool done() const { return g >= g1; }
     __device__ Tile next() {
         Tile r;
-        const int ubeg = prefix(u), uend = prefix(u + 1);
         r.u = u;
         r.bt = bt;
         r.hb = hb;
         r.b = b;
+        r.kv = kv;
         r.page0 = g - ubeg;
         r.first = (g == g0) || (g == ubeg);
+        r.whole = ubeg >= g0 && uend <= g1;
         const int seg_end = min(g1, uend);   // tiles start at the segment start
         r.np = min(kTilePages, seg_end - g);
         r.last = g + r.np == seg_end;
         r.unit_end = g + r.np == uend;
         g += r.np;
-        while (g < g1 && prefix(u + 1) <= g) step_unit();
+        while (g < g1 && uend <= g) step_unit();
         return r;
     }
 };
 
+// Block-wide exclusive scan of the units' page counts into sc[0 .. U] (U <=
+// kInKernelUnits); every thread of the CTA takes part.  Returns T = sc[U].
+__device__ int schedule_scan(int* sc, int* warp_tot, const int32_t* seq_lens, int U, int n_hb, int T_q,
+                             int max_blocks) {
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int per = (U + kThreads - 1) / kThreads;
+    const int beg = min(U, tid * per), end = min(U, beg + per);
+    int local = 0;
+    for (int u = beg; u < end; ++u) {
+        const int pages = (unit_keys(seq_lens, u, n_hb, T_q, max_blocks) + kPage - 1) / kPage;
+        sc[u + 1] = pages;
+        local += pages;
+    }
+    int v = local;   // inclusive warp scan
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+    }
+    if (lane == 31) warp_tot[w] = v;
+    __syncthreads();
+    if (w == 0) {
+        int x = lane < kThreads / 32 ? warp_tot[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane < kThreads / 32) warp_tot[lane] = x;   // inclusive over warps
+    }
+    __syncthreads();
+    int run = v - local + (w > 0 ? warp_tot[w - 1] : 0);
+    for (int u = beg; u < end; ++u) {
+        run += sc[u + 1];
+        sc[u + 1] = run;
+    }
+    if (tid == 0) sc[0] = 0;
+    __syncthreads();
+    const int T = sc[U];
+    __syncthreads();   // warp_tot may be reused by the caller
+    return T;
+}
+
 // P.V operand split: CTA r supplies latent chunks 4r .. 4r+3 (columns
 // [256r, 256r+256)); instruction h (N = 256) takes chunks 4r+2h, 4r+2h+1 from
 // each CTA, so TMEM column 128h + j of lane half r holds latent column
-// 256r + 128h + j.
+// 256r + 128h + j.  V ring entry (page, h) holds exactly those two chunks.
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
@@ -230,8 +408,11 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
 
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    volatile int* progress = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);   // tiles issued by the S producer
+    int* warp_tot = reinterpret_cast<int*>(smem + kOffMisc + 16);                   // 12 ints
     auto bar = [&](int i) { return sbase + kOffBar + 8u * static_cast<uint32_t>(i); };
     auto leader_bar = [&](int i) { return ptx::map_to_rank(bar(i), 0); };
+    const uint64_t tmo = p.timeout_ns;
 
     griddep_launch_dependents();
     if (threadIdx.x == 0) {
@@ -243,6 +424,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             ptx::mbar_init(bar(BAR_VR_FULL + s), 1);
             ptx::mbar_init(bar(BAR_VR_EMPTY + s), 1);
         }
+        for (int c = 0; c < kChunks; ++c) ptx::mbar_init(bar(BAR_Q_FULL + c), 1);
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(bar(BAR_S_FULL + b), 1);
             ptx::mbar_init(bar(BAR_S_FREE + b), 16);   // 8 softmax warps x 2 CTAs
@@ -256,10 +438,12 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         ptx::mbar_init(bar(BAR_DRAIN), 1);
         ptx::mbar_init(bar(BAR_DRAIN_PV), 1);
         *abort_flag = 0;
+        *progress = 0;
         ptx::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
         ptx::prefetch_tmap(&p.tm_pool);
+        ptx::prefetch_tmap(&p.tm_pool_v);
         ptx::prefetch_tmap(&p.tm_qa);
         ptx::prefetch_tmap(&p.tm_qr);
     }
@@ -272,28 +456,60 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     ptx::cluster_sync();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    // everything below reads what the schedule kernel (and the kernels before
-    // it: q_abs, q^R, the appended cache rows) wrote
+    // everything below reads what the kernels before this one wrote (q_abs,
+    // q^R, the appended cache rows) or what an earlier decode call may still
+    // read (the workspace)
     griddep_wait();
 
-    // this cluster's contiguous range of global pages [g0, g1) and the unit of
-    // page g0, precomputed by the schedule kernel (empty range: no work)
-    const int4 cinfo = p.cluster_info[cluster];
-    const int g0 = cinfo.x, g1 = cinfo.y, u0 = cinfo.z;
-    const int n_pre = cinfo.w - u0 + 2;   // prefix entries of units u0 .. cinfo.w, + 1
-    int32_t* pre_s = reinterpret_cast<int32_t*>(smem + kSmemUsed);
-    const int pre_cap = static_cast<int>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + kSmemBytes - reinterpret_cast<uintptr_t>(pre_s)) / 4);
-    const bool pre_in_smem = g0 < g1 && n_pre <= pre_cap;
-    if (pre_in_smem)
-        for (int k = threadIdx.x; k < n_pre; k += kThreads) pre_s[k] = p.prefix[u0 + k];
-    __syncthreads();
-    const int32_t* pf_base = pre_in_smem ? pre_s : p.prefix;
-    const int pf_off = pre_in_smem ? u0 : 0;
+    // ---- this cluster's contiguous range of global pages [g0, g1), its first
+    // unit u0 (starting at global page ubeg0) and the key counts of its units
+    int32_t* kv_s = reinterpret_cast<int32_t*>(smem + kOffSlice);
+    int g0 = 0, g1 = 0, u0 = 0, ubeg0 = 0;
+    const int32_t* kv_base = kv_s;
+    int kv_off = 0;
+    if (p.in_kernel_schedule) {
+        int* sc = reinterpret_cast<int*>(smem + kOffSRing);   // scratch: the ring area is unused until the loads start
+        const int T = schedule_scan(sc, warp_tot, p.seq_lens, p.U, p.n_hb, p.T_q, p.max_blocks);
+        int* cuts = reinterpret_cast<int*>(smem + kOffCuts);
+        compute_cuts(cuts, sc + kInKernelUnits + 1, sc, p.U, T, p.max_splits);
+        g0 = cuts[cluster];
+        g1 = cuts[cluster + 1];
+        if (g0 < g1) {
+            u0 = unit_of_page(sc, p.U, g0);
+            ubeg0 = sc[u0];
+            const int u1 = unit_of_page(sc, p.U, g1 - 1);
+            for (int k = threadIdx.x; k <= u1 - u0; k += kThreads)
+                kv_s[k] = unit_keys(p.seq_lens, u0 + k, p.n_hb, p.T_q, p.max_blocks);
+        }
+        kv_off = u0;
+        // merge metadata and length checks, spread over the grid's threads
+        for (int u = blockIdx.x * kThreads + threadIdx.x; u < p.U; u += gridDim.x * kThreads) {
+            const int4 m = unit_meta_of(u, sc, cuts, p.seq_lens, p.n_hb, p.T_q, p.max_blocks);
+            p.unit_meta[u] = m;
+            if (m.x == 0 && (u % (p.n_hb * p.T_q)) == 0) raise_status(p.status, MLA_STATUS_BAD_SEQ_LEN);
+        }
+    } else {
+        const int4 cinfo = p.cluster_info[cluster];
+        g0 = cinfo.x;
+        g1 = cinfo.y;
+        u0 = cinfo.z;
+        const int n_units = cinfo.w - u0 + 1;   // units u0 .. cinfo.w
+        if (g0 < g1) {
+            ubeg0 = p.prefix[u0];
+            if (n_units <= kSliceCap) {
+                for (int k = threadIdx.x; k < n_units; k += kThreads) kv_s[k] = p.unit_kv[u0 + k];
+                kv_off = u0;
+            } else {
+                kv_base = p.unit_kv;
+                kv_off = 0;
+            }
+        }
+    }
+    ptx::fence_proxy_async_smem();   // the scan's reads of the ring area precede the loads into it
+    __syncthreads();   // slice written; the scan scratch is free for the rings
+    ptx::fence_proxy_async_smem();   // the scan's reads of the ring area precede the loads into it
+    __syncthreads();   // slice written; the scan scratch is free for the rings
 
-    // Two load streams, each consumed in order by one MMA issuer:
-    //   S ring: S(i) = 9 entries (column chunk c of this CTA's pages 2r, 2r+1)
-    //   V ring: V(i) = 2 entries per page (latent chunks owned for P.V h = 0, 1)
     // Block-table entries are plain global loads.  Each producer issues them a
     // tile or two before it needs them, so that their latency overlaps the
     // ring waits of the tiles in between; an entry is validated where it is
@@ -308,20 +524,23 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         }
         return blk * kPage;
     };
+    auto walker = [&](TileWalker& w) { w.init(kv_base, kv_off, u0, ubeg0, g0, g1, p.n_hb, p.T_q); };
 
     if (warp == 0) {
         // ------------------------------------------------------------ S stream
         // Entry c of a tile holds column chunk c (64 columns) of this CTA's two
-        // pages (keys) and of its 64 heads' query rows: the query is re-read from
-        // L2 with every tile instead of staying resident, which leaves room for
-        // deeper rings.  Lanes 0 and 1 load the pages, lane 2 the query chunk;
-        // lane 0 of the leader CTA arms the full barrier with both CTAs' bytes.
-        // Lane l < 2 owns this CTA's page 2r + l of every tile: its block for
-        // tiles i, i+1, i+2 sits in b0, b1, b2 while tile i is issued.
+        // pages (keys).  Lanes 0 and 1 load the pages; on the first tile of a
+        // unit segment lane 2 loads query chunk c into the resident query
+        // block.  The ring is at most one tile deep, so once entry c of this
+        // tile has a free slot, the S MMAs of the previous tile that read query
+        // chunk c have completed.  Lane 0 of the leader CTA arms the full
+        // barriers with both CTAs' bytes.  Lane l < 2 owns this CTA's page
+        // 2r + l of every tile: its block for tiles i, i+1, i+2 sits in b0, b1,
+        // b2 while tile i is issued.
         const int my_pg = 2 * static_cast<int>(rank) + (lane & 1);
         TileWalker w, wa;
-        w.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
-        wa.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
+        walker(w);
+        walker(wa);
         int b0 = 0, b1 = 0, b2 = 0;
         bool h0 = false, h1 = false, h2 = false;
         // (the loads are unconditional, to a valid entry, so that nothing waits
@@ -337,43 +556,50 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         look(b0, h0);
         look(b1, h1);
         look(b2, h2);
-        int e = 0;
+        int e = 0, tiles = 0;
         bool ok = g0 < g1;
         while (ok && !w.done()) {
             const Tile cur = w.next();
             const int qrow = cur.bt * p.n_h + cur.hb * 128 + 64 * static_cast<int>(rank);
             const int row = h0 ? blk_row(b0) : 0;
-            const uint32_t tx = static_cast<uint32_t>(cur.np + 2) * kBox;    // both CTAs' pages and query chunks
-            for (int c = 0; c < 9; ++c, ++e) {
+            const uint32_t tx = static_cast<uint32_t>(cur.np) * kBox;    // both CTAs' page chunks
+            for (int c = 0; c < kChunks; ++c, ++e) {
                 const int slot = e % kSRing;
-                const uint32_t dst = sbase + kOffSRing + slot * kSEntry;
                 bool good = true;
                 if (lane < 3) {
-                    good = wait_bar(bar(BAR_SR_EMPTY + slot), ((e / kSRing) & 1) ^ 1, abort_flag, p.status);
-                    if (good && lane == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_SR_FULL + slot), tx);
-                    // one TMA instruction for the three lanes' boxes
+                    good = wait_bar(bar(BAR_SR_EMPTY + slot), ((e / kSRing) & 1) ^ 1, abort_flag, p.status, tmo);
                     const bool q_lane = lane == 2;
-                    const void* tm = q_lane ? (c < 8 ? static_cast<const void*>(&p.tm_qa) : &p.tm_qr) : &p.tm_pool;
-                    const int bx = q_lane ? (c < 8 ? 64 * c : 0) : 64 * c;
-                    const int by = q_lane ? qrow : row;
-                    if (good && (h0 || q_lane))
-                        ptx::tma_load_2d_pair_normal(dst + (q_lane ? 2 : (lane & 1)) * kBox, tm, bx, by,
-                                                     leader_bar(BAR_SR_FULL + slot));
+                    if (good && rank == 0) {
+                        if (lane == 0) ptx::mbar_arrive_expect_tx(bar(BAR_SR_FULL + slot), tx);
+                        if (q_lane && cur.first) ptx::mbar_arrive_expect_tx(bar(BAR_Q_FULL + c), 2 * kBox);
+                    }
+                    const bool withheld = p.withhold_load && rank == 0 && e == 0 && lane == 0;
+                    if (good && (q_lane ? cur.first : (h0 && !withheld))) {
+                        const void* tm = q_lane ? (c < 8 ? static_cast<const void*>(&p.tm_qa) : &p.tm_qr) : &p.tm_pool;
+                        const int bx = q_lane ? (c < 8 ? 64 * c : 0) : 64 * c;
+                        const int by = q_lane ? qrow : row;
+                        const uint32_t dst = q_lane ? sbase + kOffQ + c * kBox
+                                                    : sbase + kOffSRing + slot * kSEntry + (lane & 1) * kBox;
+                        ptx::tma_load_2d_pair_normal(dst, tm, bx, by,
+                                                     leader_bar(q_lane ? BAR_Q_FULL + c : BAR_SR_FULL + slot));
+                    }
                 }
                 if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
             }
             b0 = b1; h0 = h1;
             b1 = b2; h1 = h2;
             look(b2, h2);
+            if (lane == 0) *progress = ++tiles;
         }
     } else if (warp == 3) {
         // ------------------------------------------------------------ V stream
-        // Lane pg < 4 holds the block of page pg of the current tile (v0) and of
-        // the next one (v1).
+        // Entries (page, h): this CTA's latent chunks 4r + 2h, 4r + 2h + 1 of
+        // one page, one 3-D box.  Lane pg < 4 holds the block of page pg of the
+        // current tile (v0) and of the next one (v1).
         const uint64_t pol_v = ptx::l2_policy_evict_first();   // last use of these lines
         TileWalker w, wa;
-        w.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
-        wa.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
+        walker(w);
+        walker(wa);
         int v0 = 0, v1 = 0;
         auto look = [&](int& v) {
             if (!wa.done()) {
@@ -387,43 +613,49 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         bool ok = g0 < g1;
         while (ok && !w.done()) {
             const Tile cur = w.next();
-            for (int pg = 0; pg < cur.np && ok; ++pg, ++e) {
+            for (int pg = 0; pg < cur.np && ok; ++pg) {
                 const int row = blk_row(__shfl_sync(0xffffffffu, v0, pg));
-                const int slot = e % kVRing;
-                bool good = true;
-                if (lane == 0) {
-                    good = wait_bar(bar(BAR_VR_EMPTY + slot), ((e / kVRing) & 1) ^ 1, abort_flag, p.status);
-                    if (good && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_VR_FULL + slot), 2 * kVEntry);
-                    // this CTA's 4 latent chunks of the page in one box: [chunk][row][64 columns]
-                    if (good)
-                        ptx::tma_load_3d_pair(sbase + kOffVRing + slot * kVEntry, &p.tm_pool_v, 0, row,
-                                              4 * static_cast<int>(rank), leader_bar(BAR_VR_FULL + slot), pol_v);
+                for (int h = 0; h < 2; ++h, ++e) {
+                    const int slot = e % kVRing;
+                    bool good = true;
+                    if (lane == 0) {
+                        good = wait_bar(bar(BAR_VR_EMPTY + slot), ((e / kVRing) & 1) ^ 1, abort_flag, p.status, tmo);
+                        if (good && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_VR_FULL + slot), 2 * kVEntry);
+                        if (good)
+                            ptx::tma_load_3d_pair(sbase + kOffVRing + slot * kVEntry, &p.tm_pool_v, 0, row,
+                                                  4 * static_cast<int>(rank) + 2 * h, leader_bar(BAR_VR_FULL + slot),
+                                                  pol_v);
+                    }
+                    if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
                 }
-                if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
             }
             v0 = v1;
             look(v1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ S = Q K^T issuer
-        // S(i) occupies entries 9 i .. 9 i + 8 of the S ring (keys as B, query as A).
+        // S(i) occupies entries 9 i .. 9 i + 8 of the S ring (keys as B, the
+        // resident query as A).  The first tile of a segment also waits for
+        // each query chunk of the segment.
         if (rank == 0 && lane == 0 && g0 < g1) {
             TileWalker w;
-            w.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
-            int i = 0;
+            walker(w);
+            int i = 0, nseg = 0;
             bool ok = true;
             while (ok && !w.done()) {
-                w.next();
-                const int e0 = 9 * i;
+                const Tile t = w.next();
+                const int e0 = kChunks * i;
                 const int sb = i & 1;
-                if (!(ok = wait_bar(bar(BAR_S_FREE + sb), ((i >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+                if (!(ok = wait_bar(bar(BAR_S_FREE + sb), ((i >> 1) & 1) ^ 1, abort_flag, p.status, tmo))) break;
                 ptx::tc_fence_after();   // the softmax's reads of this S buffer are done
-                for (int c = 0; c < 9; ++c) {
+                for (int c = 0; c < kChunks; ++c) {
                     const int e = e0 + c;
-                    if (!(ok = wait_bar(bar(BAR_SR_FULL + e % kSRing), (e / kSRing) & 1, abort_flag, p.status))) break;
+                    if (t.first && !(ok = wait_bar(bar(BAR_Q_FULL + c), nseg & 1, abort_flag, p.status, tmo))) break;
+                    if (!(ok = wait_bar(bar(BAR_SR_FULL + e % kSRing), (e / kSRing) & 1, abort_flag, p.status, tmo)))
+                        break;
                     const uint32_t ent = sbase + kOffSRing + (e % kSRing) * kSEntry;
                     const uint64_t b0 = ptx::smem_desc_sw128(ent, 16, 1024);
-                    const uint64_t a0 = ptx::smem_desc_sw128(ent + 2 * kBox, 16, 1024);
+                    const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffQ + c * kBox, 16, 1024);
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
                         const uint64_t a = a0 + static_cast<uint64_t>((32 * k4) >> 4);
@@ -433,6 +665,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                     ptx::mma_commit_pair(bar(BAR_SR_EMPTY + e % kSRing), 0x3);
                 }
                 if (!ok) break;
+                if (t.first) ++nseg;
                 ptx::mma_commit_pair(bar(BAR_S_FULL + sb), 0x3);
                 ++i;
             }
@@ -440,69 +673,103 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 // let every MMA this thread issued finish before the teardown frees anything
                 ptx::mma_commit_pair(bar(BAR_DRAIN), 0x1);
                 const uint64_t t0 = ptx::global_timer_ns();
-                while (!ptx::mbar_try_wait(bar(BAR_DRAIN), 0) && ptx::global_timer_ns() - t0 < kTimeoutNs) {
+                while (!ptx::mbar_try_wait(bar(BAR_DRAIN), 0) && ptx::global_timer_ns() - t0 < tmo) {
                 }
             }
         }
     } else if (warp == 2) {
-        // ------------------------------------------------------------ O += P V issuer
-        // V(i) occupies the next 2 np entries of the V ring.
-        if (rank == 0 && lane == 0 && g0 < g1) {
-            TileWalker w;
-            w.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
-            int i = 0, tails = 0, e = 0;
-            bool ok = true;
-            const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffP, 16, 1024);
-            while (ok && !w.done()) {
-                const Tile t = w.next();
-                const int kv_len = __ldg(&p.unit_meta[t.u].x);   // read before the wait hides its latency
-                const bool tail = t.unit_end && (kv_len % kPage) != 0;
-                // P is written in two halves: keys [0,128) (pages 0, 1) by the softmax
-                // warps of TMEM lanes 0-63, keys [128,256) by those of lanes 64-127;
-                // each half is released as soon as its pages' MMAs complete.
-                for (int pg = 0; pg < 4 && ok; ++pg) {
-                    if (pg == 0 || pg == 2) {
-                        if (pg == 2) ptx::mma_commit_pair(bar(BAR_P_FREE + 0), 0x3);
-                        if (!(ok = wait_bar(bar(BAR_P_FULL + (pg >> 1)), i & 1, abort_flag, p.status))) break;
-                        ptx::tc_fence_after();
-                    }
-                    if (pg >= t.np) continue;
-                    if (tail && pg == t.np - 1) {
-                        // the unit's last page holds rows past the end: once its V
-                        // entry has landed, the softmax warps of both CTAs zero those
-                        // rows (entries are consumed in ring order, so the earlier
-                        // pages' slots are already free for this load)
-                        if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status)))
-                            break;
-                        ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 0));
-                        ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 1));
-                        if (!(ok = wait_bar(bar(BAR_TAIL_DONE), tails & 1, abort_flag, p.status))) break;
-                        ++tails;
-                    }
-                    if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status))) break;
-                    for (int h = 0; h < 2; ++h) {
-                        const uint64_t b0 =
-                            ptx::smem_desc_sw128(sbase + kOffVRing + (e % kVRing) * kVEntry + h * 2 * kBox, kBox, 1024);
+        if (rank == 0) {
+            // -------------------------------------------------------- O += P V issuer
+            // V(i) occupies the next 2 np entries of the V ring (2 per page).
+            if (lane == 0 && g0 < g1) {
+                TileWalker w;
+                walker(w);
+                int i = 0, tails = 0, e = 0;
+                bool ok = true;
+                const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffP, 16, 1024);
+                while (ok && !w.done()) {
+                    const Tile t = w.next();
+                    const bool tail = t.unit_end && (t.kv % kPage) != 0;
+                    // P is written in two halves: keys [0,128) (pages 0, 1) by the
+                    // softmax warps of TMEM lanes 0-63, keys [128,256) by those of
+                    // lanes 64-127; each half is released as soon as its pages'
+                    // MMAs complete.
+                    for (int pg = 0; pg < 4 && ok; ++pg) {
+                        if (pg == 0 || pg == 2) {
+                            if (pg == 2) ptx::mma_commit_pair(bar(BAR_P_FREE + 0), 0x3);
+                            if (!(ok = wait_bar(bar(BAR_P_FULL + (pg >> 1)), i & 1, abort_flag, p.status, tmo))) break;
+                            ptx::tc_fence_after();
+                        }
+                        if (pg >= t.np) continue;
+                        if (tail && pg == t.np - 1) {
+                            // the unit's last page holds rows past the end: once both
+                            // of its V entries have landed, the softmax warps of both
+                            // CTAs zero those rows (entries are consumed in ring order,
+                            // so the earlier pages' slots are already free for these)
+                            if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag,
+                                                p.status, tmo)))
+                                break;
+                            if (!(ok = wait_bar(bar(BAR_VR_FULL + (e + 1) % kVRing), ((e + 1) / kVRing) & 1,
+                                                abort_flag, p.status, tmo)))
+                                break;
+                            ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 0));
+                            ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 1));
+                            if (!(ok = wait_bar(bar(BAR_TAIL_DONE), tails & 1, abort_flag, p.status, tmo))) break;
+                            ++tails;
+                        }
+                        for (int h = 0; h < 2 && ok; ++h, ++e) {
+                            if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status,
+                                                tmo)))
+                                break;
+                            const uint64_t b0 =
+                                ptx::smem_desc_sw128(sbase + kOffVRing + (e % kVRing) * kVEntry, kBox, 1024);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t a = a0 + static_cast<uint64_t>((pg * kBox + 32 * kk) >> 4);
-                            const uint64_t bd = b0 + static_cast<uint64_t>((2048 * kk) >> 4);
-                            ptx::mma_pair_ss(tmem_base + kTmemO + 128 * h, a, bd, kIdescPV,
-                                             (t.first && pg == 0 && kk == 0) ? 0u : 1u);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint64_t a = a0 + static_cast<uint64_t>((pg * kBox + 32 * kk) >> 4);
+                                const uint64_t bd = b0 + static_cast<uint64_t>((2048 * kk) >> 4);
+                                ptx::mma_pair_ss(tmem_base + kTmemO + 128 * h, a, bd, kIdescPV,
+                                                 (t.first && pg == 0 && kk == 0) ? 0u : 1u);
+                            }
+                            ptx::mma_commit_pair(bar(BAR_VR_EMPTY + e % kVRing), 0x3);
                         }
                     }
-                    ptx::mma_commit_pair(bar(BAR_VR_EMPTY + e % kVRing), 0x3);
-                    ++e;
+                    if (!ok) break;
+                    ptx::mma_commit_pair(bar(BAR_P_FREE + 1), 0x3);
+                    ++i;
                 }
-                if (!ok) break;
-                ptx::mma_commit_pair(bar(BAR_P_FREE + 1), 0x3);
-                ++i;
+                if (!ok) {
+                    ptx::mma_commit_pair(bar(BAR_DRAIN_PV), 0x1);
+                    const uint64_t t0 = ptx::global_timer_ns();
+                    while (!ptx::mbar_try_wait(bar(BAR_DRAIN_PV), 0) && ptx::global_timer_ns() - t0 < tmo) {
+                    }
+                }
             }
-            if (!ok) {
-                ptx::mma_commit_pair(bar(BAR_DRAIN_PV), 0x1);
-                const uint64_t t0 = ptx::global_timer_ns();
-                while (!ptx::mbar_try_wait(bar(BAR_DRAIN_PV), 0) && ptx::global_timer_ns() - t0 < kTimeoutNs) {
+        } else if (kPrefetchAhead > 0 && g0 < g1 && lane < kTilePages) {
+            // -------------------------------------------------------- L2 prefetcher
+            // Lane pg brings page pg of each tile of the cluster (both CTAs'
+            // pages) into L2, staying at most kPrefetchAhead tiles ahead of this
+            // CTA's S loads; no shared memory and no completion tracking.
+            TileWalker w;
+            walker(w);
+            int j = 0;
+            const uint64_t t0 = ptx::global_timer_ns();
+            while (!w.done()) {
+                const Tile t = w.next();
+                bool go = true;
+                while (j >= *progress + kPrefetchAhead) {
+                    if (*abort_flag || ptx::global_timer_ns() - t0 > tmo) {
+                        go = false;
+                        break;
+                    }
+                    __nanosleep(256);
                 }
+                if (!go) break;
+                if (lane < t.np) {
+                    const int blk = load_blk(t, lane);
+                    if (blk >= 0 && blk < p.num_blocks)
+                        ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(blk) * kPage * kRow, kPageBytes);
+                }
+                ++j;
             }
         }
     } else {
@@ -520,11 +787,8 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         const int st = sw * 32 + lane;               // 0 .. 255 over the softmax warps
         const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
         float* xmax = reinterpret_cast<float*>(smem + kOffXmax);   // [cg][l]
-        TileWalker w, wa;      // wa runs one tile ahead: the next tile's unit data is loaded early
-        w.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
-        wa.init(pf_base, pf_off, u0, g0, g1, p.n_hb, p.T_q);
-        const int u_first = g0 < g1 ? wa.next().u : 0;
-        int4 meta_nxt = __ldg(&p.unit_meta[u_first]);
+        TileWalker w;
+        walker(w);
         int i = 0, tails = 0;
         int v_before = 0;      // V ring entries of tiles before i
         bool ok = true;
@@ -535,18 +799,14 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         };
         while (ok && !w.done()) {
             const Tile t = w.next();
-            const int4 meta = meta_nxt;
-            int u_nxt = t.u;
-            if (!wa.done()) u_nxt = wa.next().u;
-            meta_nxt = __ldg(&p.unit_meta[u_nxt]);
             // keys of this tile that belong to this segment
-            const int key_end = min(meta.x, kPage * (t.page0 + t.np));
+            const int key_end = min(t.kv, kPage * (t.page0 + t.np));
             if (t.first) {
                 m_used = -INFINITY;
                 l_part = 0.f;
             }
             const int sb = i & 1;
-            ok = wait_bar(bar(BAR_S_FULL + sb), (i >> 1) & 1, abort_flag, p.status);
+            ok = wait_bar(bar(BAR_S_FULL + sb), (i >> 1) & 1, abort_flag, p.status, tmo);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             ptx::tc_fence_after();
             // This thread's 64 scores (row m, keys key0 ..) are read from tensor
@@ -582,9 +842,9 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             // This half of the P buffer must be free (the previous tile's P.V MMAs on
             // it complete); a rescale of O needs the whole previous P.V complete.
             const int hf = hi ? 1 : 0;
-            ok = wait_bar(bar(BAR_P_FREE + hf), (i & 1) ^ 1, abort_flag, p.status);
+            ok = wait_bar(bar(BAR_P_FREE + hf), (i & 1) ^ 1, abort_flag, p.status, tmo);
             if (ok && !hi && __any_sync(0xffffffffu, resc))
-                ok = wait_bar(bar(BAR_P_FREE + 1), (i & 1) ^ 1, abort_flag, p.status);
+                ok = wait_bar(bar(BAR_P_FREE + 1), (i & 1) ^ 1, abort_flag, p.status, tmo);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             ptx::tc_fence_after();
             if (resc) {
@@ -634,23 +894,24 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_P_FULL + hf));
 
-            // V ring position of this tile's entries
+            // V ring position of this tile's entries (two per page)
             const int v_start = v_before;
-            v_before += t.np;
-            if (t.unit_end && (meta.x % kPage) != 0) {
-                // zero rows past the end in this CTA's V entry of the last page (4 chunks)
-                ok = wait_bar(bar(BAR_TAIL_READY), tails & 1, abort_flag, p.status);
+            v_before += 2 * t.np;
+            if (t.unit_end && (t.kv % kPage) != 0) {
+                // zero rows past the end in this CTA's two V entries of the last page
+                // (2 entries x 2 chunks of 64 rows x 128 B)
+                ok = wait_bar(bar(BAR_TAIL_READY), tails & 1, abort_flag, p.status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 ++tails;
-                const int valid = meta.x - kPage * (t.page0 + t.np - 1);
+                const int valid = t.kv - kPage * (t.page0 + t.np - 1);
                 const int bad = kPage - valid;
-                const int et = v_start + (t.np - 1);
-                unsigned char* ent = smem + kOffVRing + (et % kVRing) * kVEntry;
+                const int et = v_start + 2 * (t.np - 1);
                 for (int x = st; x < 4 * bad * 8; x += 256) {
-                    const int chunk = x / (bad * 8);
-                    const int rem = x - chunk * bad * 8;
+                    const int blk4 = x / (bad * 8);          // entry (blk4 >> 1), chunk (blk4 & 1)
+                    const int rem = x - blk4 * bad * 8;
                     const int row = valid + (rem >> 3), ch = rem & 7;
-                    reinterpret_cast<uint4*>(ent + chunk * kBox + row * 128)[ch] = make_uint4(0, 0, 0, 0);
+                    unsigned char* ent = smem + kOffVRing + ((et + (blk4 >> 1)) % kVRing) * kVEntry;
+                    reinterpret_cast<uint4*>(ent + (blk4 & 1) * kBox + row * 128)[ch] = make_uint4(0, 0, 0, 0);
                 }
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
@@ -660,7 +921,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             if (t.last) {
                 // ---- epilogue of this unit segment: wait for P.V of this tile (all
                 // warps' P of this tile is in, so every read of the maxima is done)
-                ok = wait_bar(bar(BAR_P_FREE + 1), i & 1, abort_flag, p.status);
+                ok = wait_bar(bar(BAR_P_FREE + 1), i & 1, abort_flag, p.status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 ptx::tc_fence_after();
                 xmax[cg * 128 + l] = l_part;   // partial row sums
@@ -671,7 +932,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 const float lse = lsum > 0.f ? (m_used + __log2f(lsum)) * kLn2 : -INFINITY;
                 const int bt = t.bt, hb = t.hb;
                 const int head_in_unit = 64 * static_cast<int>(rank) + m;
-                const bool whole = meta.z == 1;
+                const bool whole = t.whole;
                 const size_t grow = static_cast<size_t>(bt) * p.n_h + hb * 128 + head_in_unit;
                 const size_t slot = static_cast<size_t>(cluster) + t.u;
                 // This warp's 32 rows (consecutive heads) x 32 columns go through a
@@ -751,40 +1012,33 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
 }
 
 // ---------------------------------------------------------------------------
-// Work schedule: tiles per unit, exclusive prefix, first cluster and number of
-// clusters per unit.  One block of 1024 threads.
+// Work schedule for very large unit counts (U > kInKernelUnits): the exclusive
+// prefix of pages per unit, the units' key counts, the merge metadata and
+// each cluster's page range, computed by one block of 1024 threads with the
+// same cut rule as the decode kernel's own scan.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024)
-mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, int n_hb,
-                          int max_blocks, int C, int32_t* __restrict__ prefix,
+mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int T_q, int n_hb, int max_blocks,
+                          int max_splits, int U, int32_t* __restrict__ prefix, int32_t* __restrict__ kv_out,
                           int4* __restrict__ unit_meta, int4* __restrict__ cluster_info, int32_t* status) {
     __shared__ int warp_tot[32];
     __shared__ int carry;
     __shared__ int pre_s[kSchedSmemUnits + 1];   // the prefix again, for the searches below
     griddep_launch_dependents();
     griddep_wait();   // the workspace may still be read by an earlier decode call's kernels
-    const int U = B * T_q * n_hb;
     const bool in_smem = U <= kSchedSmemUnits;
     if (threadIdx.x == 0) carry = 0;
     __syncthreads();
     for (int base = 0; base < U; base += 1024) {
         const int u = base + threadIdx.x;
-        int tiles = 0, kv = 0, b = 0;
+        int pages = 0;
         if (u < U) {
-            const int bt = u / n_hb;
-            b = bt / T_q;
-            const int t = bt - b * T_q;
-            const int L = seq_lens[b];
-            if (L >= T_q && L <= max_blocks * kPage) {
-                kv = L - T_q + t + 1;
-                tiles = (kv + kPage - 1) / kPage;
-            } else if (t == 0 && (u % n_hb) == 0) {
-                raise_status(status, MLA_STATUS_BAD_SEQ_LEN);
-            }
-            unit_meta[u] = make_int4(kv, 0, 0, b);
+            const int kv = unit_keys(seq_lens, u, n_hb, T_q, max_blocks);
+            kv_out[u] = kv;
+            pages = (kv + kPage - 1) / kPage;
         }
-        // block exclusive scan of `tiles`
-        int v = tiles;
+        // block inclusive scan of `pages`
+        int v = pages;
         const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -816,96 +1070,109 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, 
         if (threadIdx.x == 1023) carry = incl;
         __syncthreads();
     }
-    __syncthreads();
     const int* pf = in_smem ? pre_s : prefix;
-    const long long T = carry;
-    const long long Ce = T < C ? T : C;   // clusters that get work (all non-empty ranges)
+    const int T = carry;
+    __shared__ int cuts[kClusters + 1], cut_tmp[kClusters + 1];
+    compute_cuts(cuts, cut_tmp, pf, U, T, max_splits);
     for (int u = threadIdx.x; u < U; u += 1024) {
-        const int a = pf[u], e = pf[u + 1];
-        if (e > a) {
-            // cluster c covers tiles [floor(c T / Ce), floor((c+1) T / Ce)); tile g
-            // lies in cluster floor(((g + 1) Ce - 1) / T)
-            const int c0 = static_cast<int>(((static_cast<long long>(a) + 1) * Ce - 1) / T);
-            const int c1 = static_cast<int>((static_cast<long long>(e) * Ce - 1) / T);
-            unit_meta[u].y = c0;
-            unit_meta[u].z = c1 - c0 + 1;
-        }
+        const int4 m = unit_meta_of(u, pf, cuts, seq_lens, n_hb, T_q, max_blocks);
+        unit_meta[u] = m;
+        if (m.x == 0 && (u % (n_hb * T_q)) == 0) raise_status(status, MLA_STATUS_BAD_SEQ_LEN);
     }
-    // per cluster: page range and the unit holding its first page
-    __syncthreads();
-    for (int c = threadIdx.x; c < C; c += 1024) {
-        int4 ci = make_int4(0, 0, 0, 0);
-        if (c < Ce) {
-            const int a = static_cast<int>((static_cast<long long>(c) * T) / Ce);
-            const int e = static_cast<int>((static_cast<long long>(c + 1) * T) / Ce);
-            int lo = 0, hi = U - 1;   // last unit with prefix <= a
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (pf[mid] <= a) lo = mid; else hi = mid - 1;
-            }
-            int lo2 = lo, hi2 = U - 1;   // last unit with prefix <= e - 1 (holds the range's last page)
-            while (lo2 < hi2) {
-                const int mid = (lo2 + hi2 + 1) >> 1;
-                if (pf[mid] <= e - 1) lo2 = mid; else hi2 = mid - 1;
-            }
-            ci = make_int4(a, e, lo, lo2);
-        }
-        cluster_info[c] = ci;
+    for (int c = threadIdx.x; c < kClusters; c += 1024) {
+        const int a = cuts[c], e = cuts[c + 1];
+        cluster_info[c] = a < e ? make_int4(a, e, unit_of_page(pf, U, a), unit_of_page(pf, U, e - 1))
+                                : make_int4(0, 0, 0, 0);
     }
 }
 
 // LSE merge of the partial slots of every unit covered by more than one
-// cluster; grid (128 rows, U units), 128 threads x 4 columns.
-__global__ void __launch_bounds__(128)
+// cluster: one warp per (unit, head row), a lane per 16 latent columns.  The
+// slots of unit u are meta.y + u .. meta.y + u + meta.z - 1.  Units of an
+// invalid sequence (kv_len 0) get zeros and lse = -inf.
+__global__ void __launch_bounds__(256)
 mla_sm100_merge_kernel(const int4* __restrict__ unit_meta, const float* __restrict__ part_o,
                        const float* __restrict__ part_lse, uint16_t* __restrict__ out_latent,
-                       float* __restrict__ out_lse, int n_h, int n_hb) {
+                       float* __restrict__ out_lse, int n_h, int n_hb, int U) {
     griddep_launch_dependents();
     griddep_wait();
-    const int row = blockIdx.x, u = blockIdx.y;
+    const int lane = threadIdx.x & 31;
+    const int wg = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int u = wg >> 7, row = wg & 127;
+    if (u >= U) return;
     const int4 meta = unit_meta[u];
     const int bt = u / n_hb, hb = u - bt * n_hb;
     const size_t grow = static_cast<size_t>(bt) * n_h + hb * 128 + row;
-    if (meta.x == 0) {   // invalid sequence length: defined output
-        reinterpret_cast<uint2*>(out_latent + grow * kDc)[threadIdx.x] = make_uint2(0, 0);
-        if (threadIdx.x == 0) out_lse[grow] = -INFINITY;
+    uint4* dst = reinterpret_cast<uint4*>(out_latent + grow * kDc + lane * 16);
+    if (meta.x == 0) {
+        dst[0] = make_uint4(0, 0, 0, 0);
+        dst[1] = make_uint4(0, 0, 0, 0);
+        if (lane == 0) out_lse[grow] = -INFINITY;
         return;
     }
-    if (meta.z <= 1) return;
+    const int parts = meta.z;
+    if (parts <= 1) return;
+    const size_t slot0 = static_cast<size_t>(meta.y) + u;
     float mx = -INFINITY;
-    for (int i = 0; i < meta.z; ++i)
-        mx = fmaxf(mx, part_lse[static_cast<size_t>(meta.y + i + u) * 128 + row]);
+    for (int i = lane; i < parts; i += 32) mx = fmaxf(mx, part_lse[(slot0 + i) * 128 + row]);
+    mx = warp_max(mx);
     float z = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = 0; i < meta.z; ++i) {
-        const size_t slot = static_cast<size_t>(meta.y + i + u);
-        const float ls = part_lse[slot * 128 + row];
-        const float w = ls == -INFINITY ? 0.f : ex2((ls - mx) * kLog2e);
-        z += w;
-        const float4 v = reinterpret_cast<const float4*>(part_o + (slot * 128 + row) * kDc)[threadIdx.x];
-        acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
-        acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+    float acc[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+    for (int i0 = 0; i0 < parts; i0 += 32) {
+        const int i = i0 + lane;
+        const float ls = i < parts ? part_lse[(slot0 + i) * 128 + row] : -INFINITY;
+        const float wl = ls == -INFINITY ? 0.f : ex2((ls - mx) * kLog2e);
+        z += wl;
+        const int n = min(32, parts - i0);
+        // four slots' loads in flight before they are combined
+        for (int j0 = 0; j0 < n; j0 += 4) {
+            float4 v[4][4];
+            float wj[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int j = min(j0 + jj, n - 1);
+                const float wsh = __shfl_sync(0xffffffffu, wl, j);
+                wj[jj] = j0 + jj < n ? wsh : 0.f;
+                const float4* src = reinterpret_cast<const float4*>(part_o + ((slot0 + i0 + j) * 128 + row) * kDc) +
+                                    lane * 4;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v[jj][k] = src[k];
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    acc[4 * k + 0] = fmaf(wj[jj], v[jj][k].x, acc[4 * k + 0]);
+                    acc[4 * k + 1] = fmaf(wj[jj], v[jj][k].y, acc[4 * k + 1]);
+                    acc[4 * k + 2] = fmaf(wj[jj], v[jj][k].z, acc[4 * k + 2]);
+                    acc[4 * k + 3] = fmaf(wj[jj], v[jj][k].w, acc[4 * k + 3]);
+                }
+        }
     }
+    z = warp_sum(z);
     const float inv = z > 0.f ? 1.f / z : 0.f;
-    uint2 pk;
-    pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    reinterpret_cast<uint2*>(out_latent + grow * kDc)[threadIdx.x] = pk;
-    if (threadIdx.x == 0) out_lse[grow] = z > 0.f ? mx + logf(z) : -INFINITY;
+    uint32_t pk[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2(acc[2 * k] * inv, acc[2 * k + 1] * inv);
+    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    if (lane == 0) out_lse[grow] = z > 0.f ? mx + logf(z) : -INFINITY;
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 
-// The pool viewed as [chunk (9)][row][64 columns]: one box loads several
-// 64-column chunks of the same rows into consecutive 8 KB blocks.
+// The pool viewed as [chunk (9)][row][64 columns]: one box loads two 64-column
+// chunks of the same 64 rows into consecutive 8 KB blocks.
 bool make_map_chunks(CUtensorMap* m, const void* base, uint64_t rows) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
-    const cuuint64_t dims[3] = {64, rows, 9};
+    const cuuint64_t dims[3] = {64, rows, kChunks};
     const cuuint64_t strides[2] = {kRow * 2, 128};
-    const cuuint32_t box[3] = {64, 64, 4};
+    const cuuint32_t box[3] = {64, 64, 2};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -915,19 +1182,23 @@ bool make_map_chunks(CUtensorMap* m, const void* base, uint64_t rows) {
 size_t r256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct Sm100Ws {
-    size_t prefix, meta, cinfo, part_lse, part_o, total;
+    size_t prefix, kv, meta, cinfo, part_lse, part_o, total;
 };
 
 Sm100Ws sm100_ws(int U) {
     Sm100Ws w;
     w.prefix = 0;
-    w.meta = w.prefix + r256(static_cast<size_t>(U + 1) * 4);
+    w.kv = w.prefix + r256(static_cast<size_t>(U + 1) * 4);
+    w.meta = w.kv + r256(static_cast<size_t>(U) * 4);
     w.cinfo = w.meta + r256(static_cast<size_t>(U) * 16);
     w.part_lse = w.cinfo + r256(static_cast<size_t>(kClusters) * 16);
     w.part_o = w.part_lse + r256(static_cast<size_t>(kClusters + U) * 128 * 4);
     w.total = w.part_o + r256(static_cast<size_t>(kClusters + U) * 128 * kDc * 4);
     return w;
 }
+
+// Test hook state: the next launch withholds one load and uses this wait bound.
+std::atomic<uint64_t> g_test_wait_limit_ns{0};
 
 }  // namespace
 
@@ -938,9 +1209,16 @@ size_t sm100_workspace_bytes(int n_h, int d_c, int B, int T_q) {
     return sm100_ws(B * T_q * (n_h / 128)).total;
 }
 
-int sm100_launches(int, int, int) { return 3; }
+int sm100_launches(int B, int T_q, int n_h) {
+    const int U = B * T_q * (n_h / 128);
+    return U <= kInKernelUnits ? 2 : 3;
+}
 
-cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int /*max_splits*/, cudaStream_t stream) {
+size_t sm100_unit_meta_offset(int n_h, int B, int T_q) { return sm100_ws(B * T_q * (n_h / 128)).meta; }
+
+void sm100_arm_timeout_test(uint64_t wait_limit_ns) { g_test_wait_limit_ns.store(wait_limit_ns); }
+
+cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int max_splits, cudaStream_t stream) {
     const int n_hb = P.n_h / 128;
     const int U = P.B * P.T_q * n_hb;
     if (U > 65535) return cudaErrorInvalidValue;
@@ -956,8 +1234,10 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int /*max_split
         return cudaErrorInvalidValue;
     k.pool = P.pool;
     k.block_table = P.block_table;
-    k.prefix = reinterpret_cast<const int32_t*>(base + w.prefix);
-    k.unit_meta = reinterpret_cast<const int4*>(base + w.meta);
+    k.seq_lens = P.seq_lens;
+    k.prefix = reinterpret_cast<int32_t*>(base + w.prefix);
+    k.unit_kv = reinterpret_cast<int32_t*>(base + w.kv);
+    k.unit_meta = reinterpret_cast<int4*>(base + w.meta);
     k.cluster_info = reinterpret_cast<const int4*>(base + w.cinfo);
     k.out_latent = P.out_latent;
     k.out_lse = P.out_lse;
@@ -966,27 +1246,34 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int /*max_split
     k.status = P.status;
     k.n_h = P.n_h;
     k.n_hb = n_hb;
+    k.B = P.B;
     k.T_q = P.T_q;
     k.U = U;
-    k.C = kClusters;
     k.num_blocks = P.num_blocks;
     k.max_blocks = P.max_blocks;
+    k.max_splits = max_splits;
+    k.in_kernel_schedule = U <= kInKernelUnits ? 1 : 0;
+    const uint64_t test_limit = g_test_wait_limit_ns.exchange(0);
+    k.withhold_load = test_limit != 0 ? 1 : 0;
+    k.timeout_ns = test_limit != 0 ? test_limit : 2000000000ull;
     k.scale_log2 = P.scale_log2;
 
-    cudaError_t e = launch_pdl(mla_sm100_schedule_kernel, dim3(1), dim3(1024), 0, stream, P.seq_lens, P.B, P.T_q,
-                               n_hb, P.max_blocks, static_cast<int>(kClusters),
-                               reinterpret_cast<int32_t*>(base + w.prefix), reinterpret_cast<int4*>(base + w.meta),
-                               reinterpret_cast<int4*>(base + w.cinfo), P.status);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
+    if (!k.in_kernel_schedule) {
+        e = launch_pdl(mla_sm100_schedule_kernel, dim3(1), dim3(1024), 0, stream, P.seq_lens, P.T_q, n_hb,
+                       P.max_blocks, max_splits, U, k.prefix, k.unit_kv, k.unit_meta,
+                       reinterpret_cast<int4*>(base + w.cinfo), P.status);
+        if (e != cudaSuccess) return e;
+    }
     static std::atomic<uint64_t> smem_set{0};
     e = allow_smem_once(mla_decode_sm100_kernel, static_cast<int>(kSmemBytes), smem_set);
     if (e != cudaSuccess) return e;
     e = launch_pdl(mla_decode_sm100_kernel, dim3(2 * kClusters), dim3(kThreads), kSmemBytes, stream, k);
     if (e != cudaSuccess) return e;
-    dim3 mgrid(128, U);
-    return launch_pdl(mla_sm100_merge_kernel, mgrid, dim3(128), 0, stream, k.unit_meta,
-                      static_cast<const float*>(k.part_o), static_cast<const float*>(k.part_lse), P.out_latent,
-                      P.out_lse, P.n_h, n_hb);
+    const int rows = U * 128;
+    return launch_pdl(mla_sm100_merge_kernel, dim3((rows + 7) / 8), dim3(256), 0, stream,
+                      static_cast<const int4*>(k.unit_meta), static_cast<const float*>(k.part_o),
+                      static_cast<const float*>(k.part_lse), P.out_latent, P.out_lse, P.n_h, n_hb, U);
 }
 
 }  // namespace mla

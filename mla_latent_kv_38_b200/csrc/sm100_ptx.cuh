@@ -82,19 +82,6 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t addr, uint32_t pa
     return ok != 0;
 }
 
-// non-blocking probe (for polling several barriers from one thread)
-__device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // ---- TMA ----------------------------------------------------------------------
 
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
@@ -103,25 +90,9 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     return p;
 }
 
-__device__ __forceinline__ uint64_t l2_policy_evict_last() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
-// 2D tiled load into this CTA's shared memory; completion bytes are reported
-// to the mbarrier at `mbar_cluster_addr`, which may sit in the peer CTA of the
-// pair.  No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, int x, int y,
-                                                 uint32_t mbar_cluster_addr, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(mbar_cluster_addr), "r"(x), "r"(y), "l"(policy)
-        : "memory");
-}
-
-// 3D tiled load (same conventions as the 2D form).
+// 3D tiled load into this CTA's shared memory with an L2 eviction hint;
+// completion bytes are reported to the mbarrier at `mbar_cluster_addr`, which
+// may sit in the peer CTA of the pair.  No multicast.
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void* tmap, int x, int y, int z,
                                                  uint32_t mbar_cluster_addr, uint64_t policy) {
     asm volatile(
@@ -131,7 +102,7 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void* tmap,
         : "memory");
 }
 
-// Same without an L2 eviction hint (normal priority).
+// 2D tiled load (same conventions, no L2 eviction hint).
 __device__ __forceinline__ void tma_load_2d_pair_normal(uint32_t dst, const void* tmap, int x, int y,
                                                         uint32_t mbar_cluster_addr) {
     asm volatile(
@@ -141,8 +112,8 @@ __device__ __forceinline__ void tma_load_2d_pair_normal(uint32_t dst, const void
         : "memory");
 }
 
-// Bring `bytes` (multiple of 16) of contiguous global memory into L2; no
-// completion tracking, no shared memory involved.
+// Bring `bytes` (multiple of 16, 16-byte aligned address) of contiguous
+// global memory into L2; no completion tracking, no shared memory involved.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* gaddr, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gaddr)), "r"(bytes)
                  : "memory");
@@ -266,14 +237,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
         : "memory");
 }
 
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int x, int y, int z, uint32_t mbar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(mbar), "r"(x), "r"(y), "r"(z)
-        : "memory");
-}
-
 __device__ __forceinline__ void tmem_alloc1(uint32_t dst, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst), "r"(ncols)
                  : "memory");
@@ -310,13 +273,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo,
     return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
            (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
            (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// Same with 64-byte swizzle (K-major rows of 64 bytes, 8-row atoms of 512 B).
-__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-    return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
-           (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (4ull << 61);
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulation.

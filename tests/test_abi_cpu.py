@@ -121,7 +121,13 @@ def test_rope_append_host_validation(M):
 
 def test_decode_launch_counts(M):
     v2 = _cfg(M)
-    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 32, 1, 0) == 3   # schedule, decode, merge
+    # tensor-core kernels: decode (which computes its own schedule) + merge; a
+    # separate scheduling kernel only beyond 2048 units of (query row, 128 heads)
+    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 32, 1, 0) == 2
+    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 32, 1, 3) == 2
+    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 2048, 1, 0) == 2
+    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 2049, 1, 0) == 3
+    assert M.raw_call("mla_decode_launches", ctypes.byref(_cfg(M, n_h=256)), 1025, 1, 0) == 3
     # portable kernels: one launch without splits, decode + merge with them
     simt = _cfg(M, impl=1)
     assert M.raw_call("mla_decode_launches", ctypes.byref(simt), 32, 1, 1) == 1
@@ -139,6 +145,21 @@ def test_decode_launch_counts(M):
     # the workspace query answers 0 for arguments the decode call would reject
     assert M.mla_decode_workspace_bytes(v2, 0, 1, 0) == 0
     assert M.mla_decode_workspace_bytes(_cfg(M, block_size=32), 32, 1, 0) == 0
+
+
+def test_workspace_covers_only_the_kernels_that_run(M):
+    """The tensor-core decode's workspace holds its schedule arrays and its
+    (74 + U) partial slots of 128 rows x (512 + 1) fp32, and nothing for the
+    portable kernel's partials (and the other way round)."""
+    v2 = _cfg(M)
+    U = 32
+    slots = (74 + U) * 128 * (512 + 1) * 4
+    tc = M.mla_decode_workspace_bytes(v2, 32, 1, 0)
+    assert slots < tc < slots + (1 << 16), tc
+    assert M.mla_decode_workspace_bytes(v2, 32, 1, 7) == tc           # max_splits changes no size
+    simt = M.mla_decode_workspace_bytes(_cfg(M, impl=1), 32, 1, 3)
+    assert 3 * 32 * 128 * (512 + 1) * 4 <= simt < 3 * 32 * 128 * (512 + 1) * 4 + 1024, simt
+    assert M.mla_decode_workspace_bytes(_cfg(M, impl=1), 32, 1, 1) == 256   # no splits: the status word only
 
 
 def test_noalloc_rejects_before_touching_a_device(M):

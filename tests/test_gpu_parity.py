@@ -120,14 +120,43 @@ def test_many_units_whole_and_split(M):
     check_sequences(dc, [0, 1, 150, 298, 299])
 
 
-@pytest.mark.parametrize("splits", [1, 2, 3, 7])
+SPLIT_SPEC = dict(seq_lens=np.array([1000, 37, 513], np.int32), seed=6)
+
+
+@pytest.mark.parametrize("splits", [0, 1, 2, 3, 7])
 @pytest.mark.parametrize("impl", [0, 1])
 def test_split_count_invariance(M, splits, impl):
-    spec = CaseSpec(**V2, seq_lens=np.array([1000, 37, 513], np.int32), seed=6)
+    spec = CaseSpec(**V2, **SPLIT_SPEC)
     dc = _dc(spec, impl=impl, max_splits=splits)
     dc.step()
     torch.cuda.synchronize()
     check_sequences(dc, range(spec.B))
+    U = spec.B * spec.T_q * spec.n_h // 128
+    parts = M.mla_decode_split_counts(dc.cfg, spec.B, spec.T_q, splits, dc.ws, U).tolist()
+    if impl == 1:
+        assert parts == [splits if splits else parts[0]] * U
+        return
+    # tensor-core decode: 16, 1 and 9 pages over 74 SM pairs; the bound caps
+    # the parts of every unit, and each unit is split as far as the bound and
+    # its page count allow (the equal cut puts every page in its own range)
+    pages = [16, 1, 9]
+    want = [min(splits, n) if splits else n for n in pages]
+    assert parts == want, (splits, parts)
+
+
+def test_split_counts_differ_with_the_bound(M):
+    """The tensor-core decode's per-unit split counts, read back from the
+    workspace, follow max_splits (and the results stay within tolerance)."""
+    spec = CaseSpec(**V2, **SPLIT_SPEC)
+    seen = []
+    for splits in (1, 2, 3, 7):
+        dc = _dc(spec, impl=0, max_splits=splits)
+        dc.step()
+        torch.cuda.synchronize()
+        check_sequences(dc, range(spec.B))
+        seen.append(tuple(M.mla_decode_split_counts(dc.cfg, spec.B, 1, splits, dc.ws, 3).tolist()))
+        assert max(seen[-1]) <= splits
+    assert len(set(seen)) == 4, seen
 
 
 # Head shapes for the projections: the DeepSeek-V2 shape, and shapes that take

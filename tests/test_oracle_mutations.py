@@ -35,6 +35,16 @@ MUTATIONS = {
     "rope_table_cos_sin_swapped": ("return np.concatenate([np.cos(theta), np.sin(theta)], axis=1).astype(np.float32)",
                                    "return np.concatenate([np.sin(theta), np.cos(theta)], axis=1).astype(np.float32)"),
     "rope_emulation_sign": ("a = (x1 * c) - (x2 * s)", "a = (x1 * c) + (x2 * s)"),
+    # one rounding of the exact difference / sum instead of a rounding per step
+    "rope_emulation_single_rounding": (
+        "a = (x1 * c) - (x2 * s)\n    b = (x2 * c) + (x1 * s)",
+        "a = ((x1.astype(np.float64) * c) - (x2.astype(np.float64) * s)).astype(np.float32)\n"
+        "    b = ((x2.astype(np.float64) * c) + (x1.astype(np.float64) * s)).astype(np.float32)"),
+    # a fused multiply-add: the first product is not rounded before the difference
+    "rope_emulation_fused": (
+        "a = (x1 * c) - (x2 * s)\n    b = (x2 * c) + (x1 * s)",
+        "a = (x1.astype(np.float64) * c - (x2 * s)).astype(np.float32)\n"
+        "    b = (x2.astype(np.float64) * c + (x1 * s)).astype(np.float32)"),
     "gather_wrong_slot": ("return int(block_table[b, pos // block_size]), pos % block_size",
                           "return int(block_table[b, pos // block_size]), (pos + 1) % block_size"),
 }

@@ -99,6 +99,63 @@ def test_rope_f32_table_emulation_tracks_fp64_rotation():
     assert np.max(np.abs(got - want) / (np.abs(want) + 1e-3)) < 2 ** -8 + 1e-4
 
 
+def _round_rne(x, mant_bits):
+    """Exact round-to-nearest-even of a rational to `mant_bits` significand bits
+    (normal range only), written out on fractions.Fraction."""
+    from fractions import Fraction
+    if x == 0:
+        return Fraction(0)
+    sign = -1 if x < 0 else 1
+    x, e = abs(Fraction(x)), 0
+    while x >= 2:
+        x, e = x / 2, e + 1
+    while x < 1:
+        x, e = x * 2, e - 1
+    scaled = x * 2 ** (mant_bits - 1)
+    q, rem = divmod(scaled.numerator, scaled.denominator)
+    half = Fraction(rem, scaled.denominator)
+    if half > Fraction(1, 2) or (half == Fraction(1, 2) and q % 2 == 1):
+        q += 1
+    return sign * Fraction(q, 2 ** (mant_bits - 1)) * Fraction(2) ** e
+
+
+def test_rope_emulation_rounds_each_product_then_the_sum():
+    """The GPU's RoPE rounds x1*c and x2*s to float32 separately, then their
+    difference (sum) to float32, then to bf16.  On these inputs the two
+    products nearly cancel, so a fused multiply-add (one rounding of
+    x1*c - fl(x2*s)) or a single rounding of the exact value lands on another
+    bf16 -- the expected bits below are the separately rounded result,
+    evaluated in exact rational arithmetic."""
+    from fractions import Fraction
+    f32 = lambda v: _round_rne(v, 24)
+    bf16 = lambda v: _round_rne(v, 8)
+
+    def bits_value(b):
+        return Fraction(float(O.bf16_to_f64(np.array([b], np.uint16))[0]))
+
+    # (x1 bits, x2 bits, cos, sin as float32), d_r = 2: out = [x1 c - x2 s, x2 c + x1 s]
+    cases = [
+        (0x3F31, 0x3F91, np.float32(0.8069711), np.float32(0.59059095), 0, 0xBDE4),   # a: -0.111328125
+        (0xBF73, 0x3F74, np.float32(0.70473045), np.float32(0.70947516), 1, 0xBAE6),  # b: -0.0017547607421875
+    ]
+    for x1b, x2b, c, sn, which, want_bits in cases:
+        x1, x2 = bits_value(x1b), bits_value(x2b)
+        cf, sf = Fraction(float(c)), Fraction(float(sn))
+        if which == 0:
+            sep = bf16(f32(f32(x1 * cf) - f32(x2 * sf)))
+            fused = bf16(f32(x1 * cf - f32(x2 * sf)))
+            once = bf16(x1 * cf - x2 * sf)
+        else:
+            sep = bf16(f32(f32(x2 * cf) + f32(x1 * sf)))
+            fused = bf16(f32(x2 * cf + f32(x1 * sf)))
+            once = bf16(x2 * cf + x1 * sf)
+        assert sep != fused and sep != once          # the case tells the schemes apart
+        assert sep == bits_value(want_bits)          # the expected bits, written out
+        table = np.array([[c, sn]], np.float32)      # one position, cos | sin
+        got = O.rope_emulate_bf16(np.array([[x1b, x2b]], np.uint16), np.array([0]), table)
+        assert int(got[0, which]) == want_bits, (hex(int(got[0, which])), hex(want_bits))
+
+
 # --------------------------------------------------------------------------
 # Hand-computed tiny case: n_h = 1, d_c = 2, d_h = 1, d_r = 2, L = 2, T_q = 1
 # --------------------------------------------------------------------------

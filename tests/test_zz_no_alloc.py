@@ -50,7 +50,10 @@ def test_noalloc_matches_workspace_decode_twice(M):
     torch.cuda.synchronize()
     ref_lat, ref_lse = dc.latent.clone(), dc.lse.clone()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    for call, splits in enumerate((3, 5)):      # two calls in a row, different split counts
+    # calls in a row: more splits, then fewer (the partials' lse block moves,
+    # and the array still holds the larger call's values), then none (the
+    # array is not used at all)
+    for call, splits in enumerate((5, 3, 1)):
         lat = torch.full_like(dc.latent, float("nan"))
         lse = torch.full_like(dc.lse, float("nan"))
         M.mla_decode_noalloc(dc.cfg, dc.q_abs, dc.q_r, dc.pool, spec.num_blocks, dc.block_table,
@@ -58,9 +61,29 @@ def test_noalloc_matches_workspace_decode_twice(M):
                              status)
         torch.cuda.synchronize()
         assert M.mla_read_status(status) == 0
-        _close(lat, ref_lat, f"latent, call {call}")
+        _close(lat, ref_lat, f"latent, call {call} ({splits} splits)")
         d = (lse - ref_lse).abs().max().item()
         assert d <= LSE_ABS, (call, d)
+
+
+def test_noalloc_reports_a_bad_block(M):
+    """A block-table entry outside the pool is flagged in the caller's status
+    word; that row is read as zeros, never out of bounds, so the outputs stay
+    finite."""
+    from mla_latent_kv_38_b200.runner import DeviceCase
+    spec = CaseSpec(n_h=128, d_c=512, d_h=128, d_r=64, seq_lens=np.array([130, 70], np.int32), seed=23)
+    dc = DeviceCase(spec, impl=M.IMPL_SIMT)
+    dc.step()
+    torch.cuda.synchronize()
+    dc.block_table[0, 1] = spec.num_blocks + 5
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lat = torch.full_like(dc.latent, float("nan"))
+    lse = torch.full_like(dc.lse, float("nan"))
+    M.mla_decode_noalloc(dc.cfg, dc.q_abs, dc.q_r, dc.pool, spec.num_blocks, dc.block_table,
+                         spec.max_blocks, dc.seq_lens, spec.B, spec.T_q, 3, lat, lse, status)
+    torch.cuda.synchronize()
+    assert M.mla_read_status(status) & M.MLA_STATUS_BAD_BLOCK
+    assert torch.isfinite(lat.float()).all() and torch.isfinite(lse).all()
 
 
 def test_noalloc_rejects_requests_beyond_the_array(M):
