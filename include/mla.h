@@ -162,13 +162,13 @@ size_t mla_decode_workspace_bytes(const mla_config_t* cfg, int B, int T_q, int m
  *   length AFTER the step's append, 1 <= T_q <= seq_lens[b].
  *   max_splits: upper bound on the parts the key range of one query row is
  *   split into (0 = the library chooses):
- *     tcgen05 kernels: the pages of all (query row, block of 128 heads) units
- *       are laid end to end and cut into 74 contiguous ranges, one per pair of
- *       SMs.  0 cuts them into equal ranges (a unit may span several); s > 0
- *       moves every cut to the next of the points that divide each unit's P
- *       pages into min(s, P) near-equal pieces, so no unit lies in more than
- *       s ranges (1 = no unit is split).  mla_decode_split_counts reports the
- *       parts each unit got.
+ *     tcgen05 kernels: the 256-key tiles of all (query row, block of 128
+ *       heads) units are laid end to end and cut into 74 contiguous ranges,
+ *       one per pair of SMs.  0 cuts them into equal ranges (a unit may span
+ *       several); s > 0 moves every cut to the next of the points that divide
+ *       each unit's P tiles into min(s, P) near-equal pieces, so no unit lies
+ *       in more than s ranges (1 = no unit is split).
+ *       mla_decode_split_counts reports the parts each unit got.
  *     portable kernels: exactly max_splits parts (0: a count from B, T_q, n_h).
  * Partial results (fp32 latent rows and log-sum-exp) of split rows go to the
  * workspace and are merged by a log-sum-exp reduction kernel.  The workspace

@@ -24,25 +24,22 @@
 //    runs as 2 x N = 256 per 16 keys: the B operand is split by latent
 //    columns, so each CTA loads all 4 pages of its 256 latent columns (these
 //    second reads hit L2).
-//  * The query block of a unit (64 heads x 576 columns per CTA, 72 KB) stays
-//    in shared memory for the whole unit segment; a new segment reloads it one
-//    64-column chunk at a time, each chunk as soon as the last S MMA that read
-//    the old one has completed.  The cache arrives by TMA (128-byte swizzle) in
-//    two rings, each with one producer warp and one in-order MMA consumer:
-//    16 KB S entries (one 64-column chunk of the CTA's 2 pages) and 16 KB V
-//    entries (2 latent chunks of one page, one 3-D box).
-//  * An otherwise idle warp of the second CTA issues bulk L2 prefetches of the
-//    cluster's pages a fixed number of tiles ahead of the loads, so that HBM
-//    streams at full rate while the MMA / softmax pipeline fills, drains and
-//    crosses unit segments.
-//  * Warp roles per CTA: warp 0 S producer (query and key chunks), warp 1
-//    tensor-memory allocation and (CTA 0) the S MMAs, warp 2 (CTA 0) the P.V
-//    MMAs / (CTA 1) the L2 prefetcher, warp 3 V producer, warps 4-11 softmax
-//    and epilogue (two warps per tensor-memory lane quadrant).  S is double
+//  * All operands arrive by TMA (128-byte swizzle) in two rings, each with one
+//    producer warp and one in-order MMA consumer: 24 KB S entries (one
+//    64-column chunk of the CTA's 2 pages and of its 64 query rows; the query
+//    is re-read from L2 each tile, which leaves shared memory to the rings) and
+//    32 KB V entries (the CTA's 4 latent chunks of one page, one 3-D box).  The
+//    loads run at DRAM latency, so the bytes in flight per SM set the rate; a
+//    thread's TMA copies run one after another, so every ring slot has its own
+//    issuing thread.
+//  * Warp roles per CTA: warp 0 S producer, warp 1 tensor-memory allocation
+//    and (CTA 0) the S MMAs, warp 2 (CTA 0) the P.V MMAs, warp 3 V producer,
+//    warps 4-11 softmax and epilogue (two warps per tensor-memory lane
+//    quadrant).  S is double
 //    buffered; P is written to shared memory in two key halves, each released
 //    as soon as its MMAs complete.  The running max is rescaled lazily (only
 //    when it grows by 2^8).
-//  * Work: the pages of all (sequence, token, head block) units are laid end
+//  * Work: the tiles of all (sequence, token, head block) units are laid end
 //    to end and cut into contiguous ranges, one per cluster (persistent, 74
 //    clusters on 148 SMs).  Each CTA computes the cut from the sequence
 //    lengths itself (a block-wide scan), so no separate scheduling launch
@@ -71,43 +68,42 @@ constexpr int kDc = 512, kDr = 64, kRow = 576;    // row = c^KV || k^R
 constexpr int kPage = 64;                         // cache rows per page (TMA box height)
 constexpr int kTilePages = 4;                     // a tile = 4 pages = 256 keys (MMA N)
 constexpr int kChunks = 9;                        // 64-column chunks of a row (8 latent + 1 RoPE)
-constexpr int kSRing = 4;                         // 16 KB entries, S operand stream
-constexpr int kVRing = 3;                         // 16 KB entries, P.V operand stream
-constexpr int kPrefetchAhead = 2;                 // tiles the L2 prefetcher runs ahead of the S loads
-constexpr uint32_t kPageBytes = kPage * kRow * 2; // 73,728
+constexpr int kSRing = 4;                         // 24 KB entries, S operand stream (query chunk + key chunks)
+constexpr int kVRing = 3;                         // 32 KB entries, P.V operand stream
+constexpr int kSLaneGroups = 4;                   // S ring slots are issued by this many groups of lanes in turn
 
 constexpr uint32_t kBox = 8192;                   // one page x 64 columns (128 B rows)
-constexpr uint32_t kSEntry = 2 * kBox;            // chunk c of the CTA's 2 pages
-constexpr uint32_t kVEntry = 2 * kBox;            // 2 latent chunks of one page
+constexpr uint32_t kSEntry = 3 * kBox;            // chunk c of the CTA's 2 pages (keys) and of its 64 query rows
+constexpr uint32_t kVEntry = 4 * kBox;            // the CTA's 4 latent chunks of one page
 constexpr uint32_t kPBytes = 4 * kBox;            // 64 heads x 256 keys (4 blocks of 64 keys)
-constexpr uint32_t kOffQ = 0;                     // 9 chunks of the CTA's 64 query rows
-constexpr uint32_t kOffSRing = kOffQ + kChunks * kBox;
+constexpr uint32_t kOffSRing = 0;
 constexpr uint32_t kOffVRing = kOffSRing + kSRing * kSEntry;
 constexpr uint32_t kOffP = kOffVRing + kVRing * kVEntry;
 constexpr uint32_t kOffXmax = kOffP + kPBytes;    // 4 x 64 floats: partial row maxima (or sums)
 constexpr uint32_t kOffBar = kOffXmax + 1024;
 constexpr uint32_t kMaxBars = 40;
-constexpr uint32_t kOffMisc = kOffBar + 8 * kMaxBars;   // tmem base, abort flag, progress counter
+constexpr uint32_t kOffMisc = kOffBar + 8 * kMaxBars;   // tmem base, abort flag
 constexpr uint32_t kOffCuts = kOffMisc + 64;      // cluster boundaries (75 ints)
 constexpr uint32_t kOffSlice = kOffCuts + 320;    // key counts of the cluster's units
 // Dynamic shared memory: the buffers above from a 1024-byte aligned base.
 constexpr uint32_t kSmemBytes = 232448;
 constexpr int kSliceCap = static_cast<int>((kSmemBytes - 1024 - kOffSlice) / 4);
 // Units up to which every CTA computes the schedule itself (the scan's scratch
-// is the ring area, and the cluster's prefix slice always fits in shared memory).
+// is the ring area).  The key counts of the cluster's units go to shared
+// memory when they fit, else to the CTA's own region of the workspace.
 constexpr int kInKernelUnits = 2048;
-static_assert(kOffSlice + 4 * (kInKernelUnits + 1) + 1024 <= kSmemBytes, "shared memory budget");
-static_assert(4 * (kInKernelUnits + 1 + kClusters + 1) <= static_cast<int>(kOffP - kOffSRing), "schedule scratch");
+static_assert(kOffSlice + 1024 <= kSmemBytes, "shared memory budget");
+static_assert(4 * (4 * kInKernelUnits + 2 + kClusters + 1 + 32) <= static_cast<int>(kOffP - kOffSRing), "schedule scratch");
 static_assert(4 * (kClusters + 1) <= 320, "cut area");
-static_assert(kSRing <= kChunks, "query chunk reuse needs the S ring to be at most one tile deep");
+static_assert(kSRing % kSLaneGroups == 0, "each lane group keeps its own ring slots");
+static_assert(4 * kSLaneGroups <= 32, "lane groups of the S producer warp");
 
 enum {
     BAR_SR_FULL = 0,                         // + slot (leader: both CTAs' bytes)
     BAR_SR_EMPTY = BAR_SR_FULL + kSRing,     // + slot (each CTA, MMA commit)
     BAR_VR_FULL = BAR_SR_EMPTY + kSRing,
     BAR_VR_EMPTY = BAR_VR_FULL + kVRing,
-    BAR_Q_FULL = BAR_VR_EMPTY + kVRing,      // + chunk (leader: both CTAs' query bytes)
-    BAR_S_FULL = BAR_Q_FULL + kChunks,       // + S buffer
+    BAR_S_FULL = BAR_VR_EMPTY + kVRing,      // + S buffer
     BAR_S_FREE = BAR_S_FULL + 2,             // + S buffer (leader, 8 warps x 2 CTAs)
     BAR_P_FULL = BAR_S_FREE + 2,             // + P half (leader, 4 warps x 2 CTAs)
     BAR_P_FREE = BAR_P_FULL + 2,             // + P half (each CTA, MMA commit)
@@ -127,19 +123,19 @@ constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 256, 0, 0);
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 256, 0, 1);
 
 constexpr uint32_t kSuspendHintNs = 100000;      // a waiting thread sleeps up to 0.1 ms per try
-constexpr int kSchedSmemUnits = 8192;             // units whose prefix the schedule kernel keeps in shared memory
+constexpr int kSchedSmemUnits = 4096;             // units whose prefixes the schedule kernel keeps in shared memory
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
 
 struct Sm100Params {
     CUtensorMap tm_pool;      // pool as [rows][576], box 64 cols x 64 rows
-    CUtensorMap tm_pool_v;    // pool as [chunk][rows][64], box 64 cols x 64 rows x 2 chunks
+    CUtensorMap tm_pool_v;    // pool as [chunk][rows][64], box 64 cols x 64 rows x 4 chunks
     CUtensorMap tm_qa;        // q_abs as [n_tok*n_h][512], box 64 x 64
     CUtensorMap tm_qr;        // q_r   as [n_tok*n_h][64],  box 64 x 64
-    const uint16_t* pool;     // for the L2 prefetches of whole pages
     const int32_t* block_table;
     const int32_t* seq_lens;
     int32_t* prefix;          // (U + 1) exclusive prefix of pages per unit (schedule kernel only)
     int32_t* unit_kv;         // (U) keys per unit (schedule kernel only)
+    int32_t* kv_cta;          // (148 x U) per-CTA key counts when the slice exceeds shared memory
     int4* unit_meta;          // (U) {kv_len, first cluster, parts, sequence}
     const int4* cluster_info; // (C) {first page, end page, first unit, last unit} (schedule kernel only)
     uint16_t* out_latent;
@@ -181,7 +177,7 @@ __device__ __forceinline__ int unit_keys(const int32_t* seq_lens, int u, int n_h
     const int bt = u / n_hb;
     const int b = bt / T_q;
     const int t = bt - b * T_q;
-    const int L = __ldg(seq_lens + b);
+    const int L = seq_lens[b];   // global or shared memory
     return (L >= T_q && L <= max_blocks * kPage) ? L - T_q + t + 1 : 0;
 }
 
@@ -195,29 +191,40 @@ __device__ __forceinline__ int unit_of_page(const int32_t* pf, int U, int g) {
     return lo;
 }
 
-// Raw cut c: floor(c T / C).  Without a bound on the parts per unit that is
-// the cut (equal ranges); with max_splits = s > 0 it moves up to the next
-// allowed cut, where unit u's P pages are cut into k = min(s, P) pieces at
-// pf[u] + floor(j P / k), j = 0 .. k, so no unit lies in more than s ranges.
-__device__ int raw_cut(int c, int T, const int32_t* pf, int U, int max_splits) {
+// Work is cut at whole tiles (4 pages, 256 keys, counted from each unit's
+// start), so that a range that crosses a unit boundary carries no extra
+// partial tile.  Raw cut c (in tiles): floor(c Tt / C), Tt = tf[U] the total
+// tiles.  With max_splits = s > 0 it moves up to the next allowed cut, where
+// unit u's P tiles are cut into k = min(s, P) pieces at tf[u] + floor(j P / k),
+// j = 0 .. k, so no unit lies in more than s ranges.
+__device__ int raw_cut_tile(int c, int Tt, const int32_t* tf, int U, int max_splits) {
     if (c <= 0) return 0;
-    if (c >= kClusters) return T;
-    const int g = static_cast<int>(static_cast<long long>(c) * T / kClusters);
-    if (max_splits <= 0 || g >= T) return g;
-    const int u = unit_of_page(pf, U, g);
-    const int a = pf[u], P = pf[u + 1] - a;   // a <= g < pf[u + 1], so P > 0
+    if (c >= kClusters) return Tt;
+    const int g = static_cast<int>(static_cast<long long>(c) * Tt / kClusters);
+    if (max_splits <= 0 || g >= Tt) return g;
+    const int u = unit_of_page(tf, U, g);
+    const int a = tf[u], P = tf[u + 1] - a;   // a <= g < tf[u + 1], so P > 0
     const int k = min(max_splits, P);
     const int j = static_cast<int>((static_cast<long long>(g - a) * k + P - 1) / P);   // ceil((g-a) k / P)
     return a + static_cast<int>(static_cast<long long>(j) * P / k);
 }
 
-// Cluster boundaries cuts[0 .. C]: the distinct raw cuts in order, then T
-// repeated, so cluster c covers pages [cuts[c], cuts[c + 1]) and every
+// First page of global tile gt (T pages, Tt tiles in all).
+__device__ int tile_to_page(int gt, int Tt, int T, const int32_t* tf, const int32_t* pf, int U) {
+    if (gt >= Tt) return T;
+    const int u = unit_of_page(tf, U, gt);    // tf[u] <= gt < tf[u + 1]
+    return pf[u] + kTilePages * (gt - tf[u]);
+}
+
+// Cluster boundaries cuts[0 .. C] in pages: the distinct raw cuts in order,
+// then T repeated, so cluster c covers pages [cuts[c], cuts[c + 1]) and every
 // non-empty range comes before every empty one (a unit's ranges are always
 // consecutive clusters).  All threads of the block call it; tmp holds C + 1
 // ints of scratch.
-__device__ void compute_cuts(int* cuts, int* tmp, const int32_t* pf, int U, int T, int max_splits) {
-    for (int c = threadIdx.x; c <= kClusters; c += blockDim.x) tmp[c] = raw_cut(c, T, pf, U, max_splits);
+__device__ void compute_cuts(int* cuts, int* tmp, const int32_t* pf, const int32_t* tf, int U, int T, int Tt,
+                             int max_splits) {
+    for (int c = threadIdx.x; c <= kClusters; c += blockDim.x)
+        tmp[c] = tile_to_page(raw_cut_tile(c, Tt, tf, U, max_splits), Tt, T, tf, pf, U);
     __syncthreads();
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
@@ -348,47 +355,70 @@ struct TileWalker {
     }
 };
 
-// Block-wide exclusive scan of the units' page counts into sc[0 .. U] (U <=
-// kInKernelUnits); every thread of the CTA takes part.  Returns T = sc[U].
-__device__ int schedule_scan(int* sc, int* warp_tot, const int32_t* seq_lens, int U, int n_hb, int T_q,
-                             int max_blocks) {
+// Block-wide exclusive scans of the units' page and tile counts into pf[0 ..
+// U] and tf[0 .. U] (U <= kInKernelUnits); every thread of the CTA takes
+// part; warp_tot holds 2 x 12 ints of scratch.  Returns {T, Tt} = {pf[U], tf[U]}.
+__device__ int2 schedule_scan(int* pf, int* tf, int* warp_tot, const int32_t* seq_lens, int U, int n_hb, int T_q,
+                              int max_blocks) {
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int per = (U + kThreads - 1) / kThreads;
     const int beg = min(U, tid * per), end = min(U, beg + per);
-    int local = 0;
+    int lp = 0, lt = 0;
     for (int u = beg; u < end; ++u) {
         const int pages = (unit_keys(seq_lens, u, n_hb, T_q, max_blocks) + kPage - 1) / kPage;
-        sc[u + 1] = pages;
-        local += pages;
+        const int tiles = (pages + kTilePages - 1) / kTilePages;
+        pf[u + 1] = pages;
+        tf[u + 1] = tiles;
+        lp += pages;
+        lt += tiles;
     }
-    int v = local;   // inclusive warp scan
+    int vp = lp, vt = lt;   // inclusive warp scans
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += y;
+        const int yp = __shfl_up_sync(0xffffffffu, vp, o);
+        const int yt = __shfl_up_sync(0xffffffffu, vt, o);
+        if (lane >= o) {
+            vp += yp;
+            vt += yt;
+        }
     }
-    if (lane == 31) warp_tot[w] = v;
+    if (lane == 31) {
+        warp_tot[w] = vp;
+        warp_tot[16 + w] = vt;
+    }
     __syncthreads();
     if (w == 0) {
-        int x = lane < kThreads / 32 ? warp_tot[lane] : 0;
+        int xp = lane < kThreads / 32 ? warp_tot[lane] : 0;
+        int xt = lane < kThreads / 32 ? warp_tot[16 + lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
+            const int yp = __shfl_up_sync(0xffffffffu, xp, o);
+            const int yt = __shfl_up_sync(0xffffffffu, xt, o);
+            if (lane >= o) {
+                xp += yp;
+                xt += yt;
+            }
         }
-        if (lane < kThreads / 32) warp_tot[lane] = x;   // inclusive over warps
+        if (lane < kThreads / 32) {   // inclusive over warps
+            warp_tot[lane] = xp;
+            warp_tot[16 + lane] = xt;
+        }
     }
     __syncthreads();
-    int run = v - local + (w > 0 ? warp_tot[w - 1] : 0);
+    int rp = vp - lp + (w > 0 ? warp_tot[w - 1] : 0);
+    int rt = vt - lt + (w > 0 ? warp_tot[16 + w - 1] : 0);
     for (int u = beg; u < end; ++u) {
-        run += sc[u + 1];
-        sc[u + 1] = run;
+        rp += pf[u + 1];
+        pf[u + 1] = rp;
+        rt += tf[u + 1];
+        tf[u + 1] = rt;
     }
-    if (tid == 0) sc[0] = 0;
+    if (tid == 0) {
+        pf[0] = 0;
+        tf[0] = 0;
+    }
     __syncthreads();
-    const int T = sc[U];
-    __syncthreads();   // warp_tot may be reused by the caller
-    return T;
+    return make_int2(pf[U], tf[U]);
 }
 
 // P.V operand split: CTA r supplies latent chunks 4r .. 4r+3 (columns
@@ -408,8 +438,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
 
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-    volatile int* progress = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);   // tiles issued by the S producer
-    int* warp_tot = reinterpret_cast<int*>(smem + kOffMisc + 16);                   // 12 ints
     auto bar = [&](int i) { return sbase + kOffBar + 8u * static_cast<uint32_t>(i); };
     auto leader_bar = [&](int i) { return ptx::map_to_rank(bar(i), 0); };
     const uint64_t tmo = p.timeout_ns;
@@ -424,7 +452,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             ptx::mbar_init(bar(BAR_VR_FULL + s), 1);
             ptx::mbar_init(bar(BAR_VR_EMPTY + s), 1);
         }
-        for (int c = 0; c < kChunks; ++c) ptx::mbar_init(bar(BAR_Q_FULL + c), 1);
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(bar(BAR_S_FULL + b), 1);
             ptx::mbar_init(bar(BAR_S_FREE + b), 16);   // 8 softmax warps x 2 CTAs
@@ -438,7 +465,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         ptx::mbar_init(bar(BAR_DRAIN), 1);
         ptx::mbar_init(bar(BAR_DRAIN_PV), 1);
         *abort_flag = 0;
-        *progress = 0;
         ptx::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -456,6 +482,19 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     ptx::cluster_sync();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // The sequence lengths and the block table are read first after the wait:
+    // bring them into L2 now (a prefetch changes no data, and L2 is coherent
+    // with the writes of a kernel still running, so it may precede the wait).
+    // Each CTA takes every 148th 128-byte line.
+    if (warp >= 4) {
+        const char* lens_b = reinterpret_cast<const char*>(p.seq_lens);
+        const char* tab_b = reinterpret_cast<const char*>(p.block_table);
+        const long n_lens = (static_cast<long>(p.B) * 4 + 127) / 128;
+        const long n_tab = (static_cast<long>(p.B) * p.max_blocks * 4 + 127) / 128;
+        for (long k = blockIdx.x + static_cast<long>(gridDim.x) * (threadIdx.x - 128); k < n_lens + n_tab;
+             k += static_cast<long>(gridDim.x) * (kThreads - 128))
+            ptx::prefetch_l2_line(k < n_lens ? lens_b + 128 * k : tab_b + 128 * (k - n_lens));
+    }
     // everything below reads what the kernels before this one wrote (q_abs,
     // q^R, the appended cache rows) or what an earlier decode call may still
     // read (the workspace)
@@ -468,23 +507,36 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     const int32_t* kv_base = kv_s;
     int kv_off = 0;
     if (p.in_kernel_schedule) {
-        int* sc = reinterpret_cast<int*>(smem + kOffSRing);   // scratch: the ring area is unused until the loads start
-        const int T = schedule_scan(sc, warp_tot, p.seq_lens, p.U, p.n_hb, p.T_q, p.max_blocks);
+        // scratch: the ring area is unused until the loads start
+        int* sc = reinterpret_cast<int*>(smem + kOffSRing);          // page prefix, U + 1
+        int* tfx = sc + kInKernelUnits + 1;                           // tile prefix, U + 1
+        int* ctmp = tfx + kInKernelUnits + 1;                         // cut scratch, C + 1
+        int* lens = ctmp + kClusters + 1;                             // sequence lengths, B <= U
+        int* wtot = lens + kInKernelUnits;                            // scan scratch, 32
+        for (int b = threadIdx.x; b < p.B; b += kThreads) lens[b] = __ldg(p.seq_lens + b);
+        __syncthreads();
+        const int2 TT = schedule_scan(sc, tfx, wtot, lens, p.U, p.n_hb, p.T_q, p.max_blocks);
+        const int T = TT.x;
         int* cuts = reinterpret_cast<int*>(smem + kOffCuts);
-        compute_cuts(cuts, sc + kInKernelUnits + 1, sc, p.U, T, p.max_splits);
+        compute_cuts(cuts, ctmp, sc, tfx, p.U, T, TT.y, p.max_splits);
         g0 = cuts[cluster];
         g1 = cuts[cluster + 1];
         if (g0 < g1) {
             u0 = unit_of_page(sc, p.U, g0);
             ubeg0 = sc[u0];
             const int u1 = unit_of_page(sc, p.U, g1 - 1);
+            int32_t* dst = kv_s;
+            if (u1 - u0 + 1 > kSliceCap) {   // only this CTA reads its region
+                dst = p.kv_cta + static_cast<size_t>(blockIdx.x) * p.U;
+                kv_base = dst;
+            }
             for (int k = threadIdx.x; k <= u1 - u0; k += kThreads)
-                kv_s[k] = unit_keys(p.seq_lens, u0 + k, p.n_hb, p.T_q, p.max_blocks);
+                dst[k] = unit_keys(lens, u0 + k, p.n_hb, p.T_q, p.max_blocks);
         }
         kv_off = u0;
         // merge metadata and length checks, spread over the grid's threads
         for (int u = blockIdx.x * kThreads + threadIdx.x; u < p.U; u += gridDim.x * kThreads) {
-            const int4 m = unit_meta_of(u, sc, cuts, p.seq_lens, p.n_hb, p.T_q, p.max_blocks);
+            const int4 m = unit_meta_of(u, sc, cuts, lens, p.n_hb, p.T_q, p.max_blocks);
             p.unit_meta[u] = m;
             if (m.x == 0 && (u % (p.n_hb * p.T_q)) == 0) raise_status(p.status, MLA_STATUS_BAD_SEQ_LEN);
         }
@@ -507,8 +559,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     }
     ptx::fence_proxy_async_smem();   // the scan's reads of the ring area precede the loads into it
     __syncthreads();   // slice written; the scan scratch is free for the rings
-    ptx::fence_proxy_async_smem();   // the scan's reads of the ring area precede the loads into it
-    __syncthreads();   // slice written; the scan scratch is free for the rings
 
     // Block-table entries are plain global loads.  Each producer issues them a
     // tile or two before it needs them, so that their latency overlaps the
@@ -529,15 +579,18 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     if (warp == 0) {
         // ------------------------------------------------------------ S stream
         // Entry c of a tile holds column chunk c (64 columns) of this CTA's two
-        // pages (keys).  Lanes 0 and 1 load the pages; on the first tile of a
-        // unit segment lane 2 loads query chunk c into the resident query
-        // block.  The ring is at most one tile deep, so once entry c of this
-        // tile has a free slot, the S MMAs of the previous tile that read query
-        // chunk c have completed.  Lane 0 of the leader CTA arms the full
-        // barriers with both CTAs' bytes.  Lane l < 2 owns this CTA's page
-        // 2r + l of every tile: its block for tiles i, i+1, i+2 sits in b0, b1,
-        // b2 while tile i is issued.
-        const int my_pg = 2 * static_cast<int>(rank) + (lane & 1);
+        // pages (keys) and of its 64 query rows, one 8 KB box each; the query is
+        // re-read from L2 with every tile, which leaves the shared memory to
+        // the rings (the loads run at DRAM latency, so the bytes in flight set
+        // the rate).  A thread's TMA copies run one after another, so ring slot
+        // s is issued by its own group of lanes 4g + {0, 1, 2}, g = s mod
+        // kSLaneGroups: lane j = 0, 1 loads own page j, lane 2 the query chunk.
+        // The group's lane 0 in the leader CTA arms the full barrier with both
+        // CTAs' bytes.  The page lanes hold the block of their page for tiles
+        // i, i+1, i+2 in b0, b1, b2.
+        const int grp = lane >> 2, j = lane & 3;
+        const bool active = grp < kSLaneGroups && j < 3;
+        const int my_pg = 2 * static_cast<int>(rank) + (j & 1);
         TileWalker w, wa;
         walker(w);
         walker(wa);
@@ -549,39 +602,33 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             h = false;
             if (!wa.done()) {
                 const Tile t = wa.next();
-                h = lane < 2 && my_pg < t.np;
+                h = active && j < 2 && my_pg < t.np;
                 b = load_blk(t, min(my_pg, t.np - 1));
             }
         };
         look(b0, h0);
         look(b1, h1);
         look(b2, h2);
-        int e = 0, tiles = 0;
+        int e = 0;
         bool ok = g0 < g1;
         while (ok && !w.done()) {
             const Tile cur = w.next();
             const int qrow = cur.bt * p.n_h + cur.hb * 128 + 64 * static_cast<int>(rank);
             const int row = h0 ? blk_row(b0) : 0;
-            const uint32_t tx = static_cast<uint32_t>(cur.np) * kBox;    // both CTAs' page chunks
+            const uint32_t tx = static_cast<uint32_t>(cur.np + 2) * kBox;    // both CTAs' page and query chunks
             for (int c = 0; c < kChunks; ++c, ++e) {
                 const int slot = e % kSRing;
                 bool good = true;
-                if (lane < 3) {
+                if (active && grp == slot % kSLaneGroups) {
                     good = wait_bar(bar(BAR_SR_EMPTY + slot), ((e / kSRing) & 1) ^ 1, abort_flag, p.status, tmo);
-                    const bool q_lane = lane == 2;
-                    if (good && rank == 0) {
-                        if (lane == 0) ptx::mbar_arrive_expect_tx(bar(BAR_SR_FULL + slot), tx);
-                        if (q_lane && cur.first) ptx::mbar_arrive_expect_tx(bar(BAR_Q_FULL + c), 2 * kBox);
-                    }
-                    const bool withheld = p.withhold_load && rank == 0 && e == 0 && lane == 0;
-                    if (good && (q_lane ? cur.first : (h0 && !withheld))) {
+                    if (good && j == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_SR_FULL + slot), tx);
+                    const bool q_lane = j == 2;
+                    const bool withheld = p.withhold_load && rank == 0 && e == 0 && j == 0;
+                    if (good && (q_lane || h0) && !withheld) {
                         const void* tm = q_lane ? (c < 8 ? static_cast<const void*>(&p.tm_qa) : &p.tm_qr) : &p.tm_pool;
                         const int bx = q_lane ? (c < 8 ? 64 * c : 0) : 64 * c;
-                        const int by = q_lane ? qrow : row;
-                        const uint32_t dst = q_lane ? sbase + kOffQ + c * kBox
-                                                    : sbase + kOffSRing + slot * kSEntry + (lane & 1) * kBox;
-                        ptx::tma_load_2d_pair_normal(dst, tm, bx, by,
-                                                     leader_bar(q_lane ? BAR_Q_FULL + c : BAR_SR_FULL + slot));
+                        ptx::tma_load_2d_pair_normal(sbase + kOffSRing + slot * kSEntry + j * kBox, tm, bx,
+                                                     q_lane ? qrow : row, leader_bar(BAR_SR_FULL + slot));
                     }
                 }
                 if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
@@ -589,12 +636,12 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             b0 = b1; h0 = h1;
             b1 = b2; h1 = h2;
             look(b2, h2);
-            if (lane == 0) *progress = ++tiles;
         }
     } else if (warp == 3) {
         // ------------------------------------------------------------ V stream
-        // Entries (page, h): this CTA's latent chunks 4r + 2h, 4r + 2h + 1 of
-        // one page, one 3-D box.  Lane pg < 4 holds the block of page pg of the
+        // Entry per page: this CTA's latent chunks 4r .. 4r+3 of the page, one
+        // 3-D box, issued by lane (slot) so that consecutive copies come from
+        // different threads.  Lane pg < 4 holds the block of page pg of the
         // current tile (v0) and of the next one (v1).
         const uint64_t pol_v = ptx::l2_policy_evict_first();   // last use of these lines
         TileWalker w, wa;
@@ -613,49 +660,43 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         bool ok = g0 < g1;
         while (ok && !w.done()) {
             const Tile cur = w.next();
-            for (int pg = 0; pg < cur.np && ok; ++pg) {
+            for (int pg = 0; pg < cur.np && ok; ++pg, ++e) {
                 const int row = blk_row(__shfl_sync(0xffffffffu, v0, pg));
-                for (int h = 0; h < 2; ++h, ++e) {
-                    const int slot = e % kVRing;
-                    bool good = true;
-                    if (lane == 0) {
-                        good = wait_bar(bar(BAR_VR_EMPTY + slot), ((e / kVRing) & 1) ^ 1, abort_flag, p.status, tmo);
-                        if (good && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_VR_FULL + slot), 2 * kVEntry);
-                        if (good)
-                            ptx::tma_load_3d_pair(sbase + kOffVRing + slot * kVEntry, &p.tm_pool_v, 0, row,
-                                                  4 * static_cast<int>(rank) + 2 * h, leader_bar(BAR_VR_FULL + slot),
-                                                  pol_v);
-                    }
-                    if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
+                const int slot = e % kVRing;
+                bool good = true;
+                if (lane == slot) {
+                    good = wait_bar(bar(BAR_VR_EMPTY + slot), ((e / kVRing) & 1) ^ 1, abort_flag, p.status, tmo);
+                    if (good && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_VR_FULL + slot), 2 * kVEntry);
+                    if (good)
+                        ptx::tma_load_3d_pair(sbase + kOffVRing + slot * kVEntry, &p.tm_pool_v, 0, row,
+                                              4 * static_cast<int>(rank), leader_bar(BAR_VR_FULL + slot), pol_v);
                 }
+                if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
             }
             v0 = v1;
             look(v1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ S = Q K^T issuer
-        // S(i) occupies entries 9 i .. 9 i + 8 of the S ring (keys as B, the
-        // resident query as A).  The first tile of a segment also waits for
-        // each query chunk of the segment.
+        // S(i) occupies entries 9 i .. 9 i + 8 of the S ring (keys as B, query as A).
         if (rank == 0 && lane == 0 && g0 < g1) {
             TileWalker w;
             walker(w);
-            int i = 0, nseg = 0;
+            int i = 0;
             bool ok = true;
             while (ok && !w.done()) {
-                const Tile t = w.next();
+                w.next();
                 const int e0 = kChunks * i;
                 const int sb = i & 1;
                 if (!(ok = wait_bar(bar(BAR_S_FREE + sb), ((i >> 1) & 1) ^ 1, abort_flag, p.status, tmo))) break;
                 ptx::tc_fence_after();   // the softmax's reads of this S buffer are done
                 for (int c = 0; c < kChunks; ++c) {
                     const int e = e0 + c;
-                    if (t.first && !(ok = wait_bar(bar(BAR_Q_FULL + c), nseg & 1, abort_flag, p.status, tmo))) break;
                     if (!(ok = wait_bar(bar(BAR_SR_FULL + e % kSRing), (e / kSRing) & 1, abort_flag, p.status, tmo)))
                         break;
                     const uint32_t ent = sbase + kOffSRing + (e % kSRing) * kSEntry;
                     const uint64_t b0 = ptx::smem_desc_sw128(ent, 16, 1024);
-                    const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffQ + c * kBox, 16, 1024);
+                    const uint64_t a0 = ptx::smem_desc_sw128(ent + 2 * kBox, 16, 1024);
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
                         const uint64_t a = a0 + static_cast<uint64_t>((32 * k4) >> 4);
@@ -665,7 +706,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                     ptx::mma_commit_pair(bar(BAR_SR_EMPTY + e % kSRing), 0x3);
                 }
                 if (!ok) break;
-                if (t.first) ++nseg;
                 ptx::mma_commit_pair(bar(BAR_S_FULL + sb), 0x3);
                 ++i;
             }
@@ -680,7 +720,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     } else if (warp == 2) {
         if (rank == 0) {
             // -------------------------------------------------------- O += P V issuer
-            // V(i) occupies the next 2 np entries of the V ring (2 per page).
+            // V(i) occupies the next np entries of the V ring (one per page).
             if (lane == 0 && g0 < g1) {
                 TileWalker w;
                 walker(w);
@@ -702,27 +742,23 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                         }
                         if (pg >= t.np) continue;
                         if (tail && pg == t.np - 1) {
-                            // the unit's last page holds rows past the end: once both
-                            // of its V entries have landed, the softmax warps of both
-                            // CTAs zero those rows (entries are consumed in ring order,
-                            // so the earlier pages' slots are already free for these)
+                            // the unit's last page holds rows past the end: once its V
+                            // entry has landed, the softmax warps of both CTAs zero those
+                            // rows (entries are consumed in ring order, so the earlier
+                            // pages' slots are already free for this load)
                             if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag,
                                                 p.status, tmo)))
-                                break;
-                            if (!(ok = wait_bar(bar(BAR_VR_FULL + (e + 1) % kVRing), ((e + 1) / kVRing) & 1,
-                                                abort_flag, p.status, tmo)))
                                 break;
                             ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 0));
                             ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 1));
                             if (!(ok = wait_bar(bar(BAR_TAIL_DONE), tails & 1, abort_flag, p.status, tmo))) break;
                             ++tails;
                         }
-                        for (int h = 0; h < 2 && ok; ++h, ++e) {
-                            if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status,
-                                                tmo)))
-                                break;
-                            const uint64_t b0 =
-                                ptx::smem_desc_sw128(sbase + kOffVRing + (e % kVRing) * kVEntry, kBox, 1024);
+                        if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status, tmo)))
+                            break;
+                        for (int h = 0; h < 2; ++h) {
+                            const uint64_t b0 = ptx::smem_desc_sw128(
+                                sbase + kOffVRing + (e % kVRing) * kVEntry + h * 2 * kBox, kBox, 1024);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
                                 const uint64_t a = a0 + static_cast<uint64_t>((pg * kBox + 32 * kk) >> 4);
@@ -730,8 +766,9 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                                 ptx::mma_pair_ss(tmem_base + kTmemO + 128 * h, a, bd, kIdescPV,
                                                  (t.first && pg == 0 && kk == 0) ? 0u : 1u);
                             }
-                            ptx::mma_commit_pair(bar(BAR_VR_EMPTY + e % kVRing), 0x3);
                         }
+                        ptx::mma_commit_pair(bar(BAR_VR_EMPTY + e % kVRing), 0x3);
+                        ++e;
                     }
                     if (!ok) break;
                     ptx::mma_commit_pair(bar(BAR_P_FREE + 1), 0x3);
@@ -743,33 +780,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                     while (!ptx::mbar_try_wait(bar(BAR_DRAIN_PV), 0) && ptx::global_timer_ns() - t0 < tmo) {
                     }
                 }
-            }
-        } else if (kPrefetchAhead > 0 && g0 < g1 && lane < kTilePages) {
-            // -------------------------------------------------------- L2 prefetcher
-            // Lane pg brings page pg of each tile of the cluster (both CTAs'
-            // pages) into L2, staying at most kPrefetchAhead tiles ahead of this
-            // CTA's S loads; no shared memory and no completion tracking.
-            TileWalker w;
-            walker(w);
-            int j = 0;
-            const uint64_t t0 = ptx::global_timer_ns();
-            while (!w.done()) {
-                const Tile t = w.next();
-                bool go = true;
-                while (j >= *progress + kPrefetchAhead) {
-                    if (*abort_flag || ptx::global_timer_ns() - t0 > tmo) {
-                        go = false;
-                        break;
-                    }
-                    __nanosleep(256);
-                }
-                if (!go) break;
-                if (lane < t.np) {
-                    const int blk = load_blk(t, lane);
-                    if (blk >= 0 && blk < p.num_blocks)
-                        ptx::prefetch_l2_bulk(p.pool + static_cast<size_t>(blk) * kPage * kRow, kPageBytes);
-                }
-                ++j;
             }
         }
     } else {
@@ -839,6 +849,31 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             const float alpha = ex2(m_used - new_m);
             m_used = new_m;
 
+            // The weights of row m, keys key0 + [0, 64): computed into registers
+            // first, which ends this thread's reads of the S buffer.
+            float ps2[2] = {0.f, 0.f};
+            const float neg_m = -m_used;
+            uint32_t pk[32];
+            {
+                uint32_t r[2][32];
+                ptx::tmem_ld32(s_col, r[0]);
+                ptx::tmem_ld32(s_col + 32, r[1]);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 64; j += 2) {
+                    const float s0 = __uint_as_float(r[j >> 5][j & 31]), s1 = __uint_as_float(r[j >> 5][(j & 31) + 1]);
+                    const float p0 = j < nvalid ? ex2(fmaf(s0, p.scale_log2, neg_m)) : 0.f;
+                    const float p1 = j + 1 < nvalid ? ex2(fmaf(s1, p.scale_log2, neg_m)) : 0.f;
+                    ps2[(j >> 1) & 1] += p0 + p1;
+                    pk[j >> 1] = pack_bf16x2(p0, p1);
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster_relaxed(leader_bar(BAR_S_FREE + sb));
+            const float ps = ps2[0] + ps2[1];
+            l_part = l_part * alpha + ps;
+
             // This half of the P buffer must be free (the previous tile's P.V MMAs on
             // it complete); a rescale of O needs the whole previous P.V complete.
             const int hf = hi ? 1 : 0;
@@ -861,57 +896,36 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
             }
             // P row m, keys key0 + [0, 64) = one 64-key block (2 hi + cg) of P:
             // K-major, 128-byte rows, 128-byte swizzle (16-byte chunk index XOR row & 7)
-            float ps2[2] = {0.f, 0.f};
-            const float neg_m = -m_used;
             {
-                uint32_t r[2][32];
-                ptx::tmem_ld32(s_col, r[0]);
-                ptx::tmem_ld32(s_col + 32, r[1]);
-                ptx::tmem_wait_ld();
-                uint32_t pk[32];
-#pragma unroll
-                for (int j = 0; j < 64; j += 2) {
-                    const float s0 = __uint_as_float(r[j >> 5][j & 31]), s1 = __uint_as_float(r[j >> 5][(j & 31) + 1]);
-                    const float p0 = j < nvalid ? ex2(fmaf(s0, p.scale_log2, neg_m)) : 0.f;
-                    const float p1 = j + 1 < nvalid ? ex2(fmaf(s1, p.scale_log2, neg_m)) : 0.f;
-                    ps2[(j >> 1) & 1] += p0 + p1;
-                    pk[j >> 1] = pack_bf16x2(p0, p1);
-                }
                 unsigned char* Pb = smem + kOffP + (2 * hf + cg) * kBox + m * 128;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch)
                     *reinterpret_cast<uint4*>(Pb + ((ch ^ (m & 7)) * 16)) =
                         make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
             }
-            const float ps = ps2[0] + ps2[1];
-            l_part = l_part * alpha + ps;
-            // both reads of the S buffer are done
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive_cluster_relaxed(leader_bar(BAR_S_FREE + sb));
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive_cluster(leader_bar(BAR_P_FULL + hf));
 
-            // V ring position of this tile's entries (two per page)
+            // V ring position of this tile's entries (one per page)
             const int v_start = v_before;
-            v_before += 2 * t.np;
+            v_before += t.np;
             if (t.unit_end && (t.kv % kPage) != 0) {
-                // zero rows past the end in this CTA's two V entries of the last page
-                // (2 entries x 2 chunks of 64 rows x 128 B)
+                // zero rows past the end in this CTA's V entry of the last page
+                // (4 chunks of 64 rows x 128 B)
                 ok = wait_bar(bar(BAR_TAIL_READY), tails & 1, abort_flag, p.status, tmo);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 ++tails;
                 const int valid = t.kv - kPage * (t.page0 + t.np - 1);
                 const int bad = kPage - valid;
-                const int et = v_start + 2 * (t.np - 1);
+                const int et = v_start + (t.np - 1);
+                unsigned char* ent = smem + kOffVRing + (et % kVRing) * kVEntry;
                 for (int x = st; x < 4 * bad * 8; x += 256) {
-                    const int blk4 = x / (bad * 8);          // entry (blk4 >> 1), chunk (blk4 & 1)
-                    const int rem = x - blk4 * bad * 8;
+                    const int chunk = x / (bad * 8);
+                    const int rem = x - chunk * bad * 8;
                     const int row = valid + (rem >> 3), ch = rem & 7;
-                    unsigned char* ent = smem + kOffVRing + ((et + (blk4 >> 1)) % kVRing) * kVEntry;
-                    reinterpret_cast<uint4*>(ent + (blk4 & 1) * kBox + row * 128)[ch] = make_uint4(0, 0, 0, 0);
+                    reinterpret_cast<uint4*>(ent + chunk * kBox + row * 128)[ch] = make_uint4(0, 0, 0, 0);
                 }
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
@@ -935,56 +949,38 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 const bool whole = t.whole;
                 const size_t grow = static_cast<size_t>(bt) * p.n_h + hb * 128 + head_in_unit;
                 const size_t slot = static_cast<size_t>(cluster) + t.u;
-                // This warp's 32 rows (consecutive heads) x 32 columns go through a
-                // 4 KB shared-memory tile in the free P buffer (16-byte chunks
-                // swizzled by row), so that each global store instruction writes
-                // whole row segments instead of 32 scattered 16-byte pieces.
-                unsigned char* stage = smem + kOffP + sw * 4096;
-                const size_t grow0 = grow - lane;
-                const size_t prow0 = slot * 128 + head_in_unit - lane;
+                // Each thread writes its own row segment straight from the
+                // registers: 128 latent columns (bf16 when the unit is whole,
+                // else the fp32 partial), read from tensor memory 64 at a time.
                 const int h = cg;   // this thread's 128 O columns
                 const int col0 = 128 * h + (hi ? 256 : 0);
 #pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t o[32];
-                    ptx::tmem_ld32(t_lane + kTmemO + 128 * h + 32 * q, o);
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    uint32_t o[2][32];
+                    ptx::tmem_ld32(t_lane + kTmemO + 128 * h + 64 * q2, o[0]);
+                    ptx::tmem_ld32(t_lane + kTmemO + 128 * h + 64 * q2 + 32, o[1]);
                     ptx::tmem_wait_ld();
-                    const int col = col0 + 32 * q;
-                    if (whole) {
-                        // 32 bf16 = 64 B per row, 4 chunks at position k ^ ((row >> 1) & 3)
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            uint4 wv;
-                            wv.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
-                            wv.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
-                            wv.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
-                            wv.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
-                            *reinterpret_cast<uint4*>(stage + lane * 64 + ((k ^ ((lane >> 1) & 3)) * 16)) = wv;
+                    for (int qq = 0; qq < 2; ++qq) {
+                        const int col = col0 + 64 * q2 + 32 * qq;
+                        if (whole) {
+                            uint4* dst = reinterpret_cast<uint4*>(p.out_latent + grow * kDc + col);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                uint4 wv;
+                                wv.x = pack_bf16x2(__uint_as_float(o[qq][8 * k + 0]) * inv, __uint_as_float(o[qq][8 * k + 1]) * inv);
+                                wv.y = pack_bf16x2(__uint_as_float(o[qq][8 * k + 2]) * inv, __uint_as_float(o[qq][8 * k + 3]) * inv);
+                                wv.z = pack_bf16x2(__uint_as_float(o[qq][8 * k + 4]) * inv, __uint_as_float(o[qq][8 * k + 5]) * inv);
+                                wv.w = pack_bf16x2(__uint_as_float(o[qq][8 * k + 6]) * inv, __uint_as_float(o[qq][8 * k + 7]) * inv);
+                                dst[k] = wv;
+                            }
+                        } else {
+                            float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * 128 + head_in_unit) * kDc + col);
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                dst[k] = make_float4(__uint_as_float(o[qq][4 * k]) * inv, __uint_as_float(o[qq][4 * k + 1]) * inv,
+                                                     __uint_as_float(o[qq][4 * k + 2]) * inv, __uint_as_float(o[qq][4 * k + 3]) * inv);
                         }
-                        __syncwarp();
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int row = 8 * j + (lane >> 2), k = lane & 3;
-                            const uint4 wv =
-                                *reinterpret_cast<const uint4*>(stage + row * 64 + ((k ^ ((row >> 1) & 3)) * 16));
-                            *reinterpret_cast<uint4*>(p.out_latent + (grow0 + row) * kDc + col + 8 * k) = wv;
-                        }
-                        __syncwarp();
-                    } else {
-                        // 32 floats = 128 B per row, 8 chunks at position k ^ (row & 7)
-#pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            *reinterpret_cast<float4*>(stage + lane * 128 + ((k ^ (lane & 7)) * 16)) =
-                                make_float4(__uint_as_float(o[4 * k]) * inv, __uint_as_float(o[4 * k + 1]) * inv,
-                                            __uint_as_float(o[4 * k + 2]) * inv, __uint_as_float(o[4 * k + 3]) * inv);
-                        __syncwarp();
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int row = 4 * j + (lane >> 3), k = lane & 7;
-                            const float4 v = *reinterpret_cast<const float4*>(stage + row * 128 + ((k ^ (row & 7)) * 16));
-                            *reinterpret_cast<float4*>(p.part_o + (prow0 + row) * kDc + col + 4 * k) = v;
-                        }
-                        __syncwarp();
                     }
                 }
                 if (!hi && cg == 0) {
@@ -1013,67 +1009,83 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
 
 // ---------------------------------------------------------------------------
 // Work schedule for very large unit counts (U > kInKernelUnits): the exclusive
-// prefix of pages per unit, the units' key counts, the merge metadata and
-// each cluster's page range, computed by one block of 1024 threads with the
-// same cut rule as the decode kernel's own scan.
+// prefixes of pages and tiles per unit, the units' key counts, the merge
+// metadata and each cluster's page range, computed by one block of 1024
+// threads with the same cut rule as the decode kernel's own scan.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024)
 mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int T_q, int n_hb, int max_blocks,
-                          int max_splits, int U, int32_t* __restrict__ prefix, int32_t* __restrict__ kv_out,
-                          int4* __restrict__ unit_meta, int4* __restrict__ cluster_info, int32_t* status) {
-    __shared__ int warp_tot[32];
-    __shared__ int carry;
-    __shared__ int pre_s[kSchedSmemUnits + 1];   // the prefix again, for the searches below
+                          int max_splits, int U, int32_t* __restrict__ prefix, int32_t* __restrict__ tprefix,
+                          int32_t* __restrict__ kv_out, int4* __restrict__ unit_meta, int4* __restrict__ cluster_info,
+                          int32_t* status) {
+    __shared__ int warp_tot[2][32];
+    __shared__ int carry[2];
+    __shared__ int pre_s[kSchedSmemUnits + 1];    // the prefixes again, for the searches below
+    __shared__ int tpre_s[kSchedSmemUnits + 1];
     griddep_launch_dependents();
     griddep_wait();   // the workspace may still be read by an earlier decode call's kernels
     const bool in_smem = U <= kSchedSmemUnits;
-    if (threadIdx.x == 0) carry = 0;
+    if (threadIdx.x == 0) carry[0] = carry[1] = 0;
     __syncthreads();
     for (int base = 0; base < U; base += 1024) {
         const int u = base + threadIdx.x;
-        int pages = 0;
+        int v[2] = {0, 0};   // pages, tiles
         if (u < U) {
             const int kv = unit_keys(seq_lens, u, n_hb, T_q, max_blocks);
             kv_out[u] = kv;
-            pages = (kv + kPage - 1) / kPage;
+            v[0] = (kv + kPage - 1) / kPage;
+            v[1] = (v[0] + kTilePages - 1) / kTilePages;
         }
-        // block inclusive scan of `pages`
-        int v = pages;
         const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, v, o);
-            if (lane >= o) v += y;
-        }
-        if (lane == 31) warp_tot[w] = v;
-        __syncthreads();
-        if (w == 0) {
-            int t = warp_tot[lane];
+        for (int q = 0; q < 2; ++q) {   // block inclusive scans
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, t, o);
-                if (lane >= o) t += y;
+                const int y = __shfl_up_sync(0xffffffffu, v[q], o);
+                if (lane >= o) v[q] += y;
             }
-            warp_tot[lane] = t;
+            if (lane == 31) warp_tot[q][w] = v[q];
         }
         __syncthreads();
-        const int incl = v + (w > 0 ? warp_tot[w - 1] : 0) + carry;
+        if (w == 0) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                int t = warp_tot[q][lane];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, t, o);
+                    if (lane >= o) t += y;
+                }
+                warp_tot[q][lane] = t;
+            }
+        }
+        __syncthreads();
+        const int ip = v[0] + (w > 0 ? warp_tot[0][w - 1] : 0) + carry[0];
+        const int it = v[1] + (w > 0 ? warp_tot[1][w - 1] : 0) + carry[1];
         if (u < U) {
-            prefix[u + 1] = incl;
-            if (in_smem) pre_s[u + 1] = incl;
+            prefix[u + 1] = ip;
+            tprefix[u + 1] = it;
+            if (in_smem) {
+                pre_s[u + 1] = ip;
+                tpre_s[u + 1] = it;
+            }
         }
         if (u == 0) {
-            prefix[0] = 0;
-            if (in_smem) pre_s[0] = 0;
+            prefix[0] = tprefix[0] = 0;
+            if (in_smem) pre_s[0] = tpre_s[0] = 0;
         }
         __syncthreads();
-        if (threadIdx.x == 1023) carry = incl;
+        if (threadIdx.x == 1023) {
+            carry[0] = ip;
+            carry[1] = it;
+        }
         __syncthreads();
     }
     const int* pf = in_smem ? pre_s : prefix;
-    const int T = carry;
+    const int* tf = in_smem ? tpre_s : tprefix;
+    const int T = carry[0], Tt = carry[1];
     __shared__ int cuts[kClusters + 1], cut_tmp[kClusters + 1];
-    compute_cuts(cuts, cut_tmp, pf, U, T, max_splits);
+    compute_cuts(cuts, cut_tmp, pf, tf, U, T, Tt, max_splits);
     for (int u = threadIdx.x; u < U; u += 1024) {
         const int4 m = unit_meta_of(u, pf, cuts, seq_lens, n_hb, T_q, max_blocks);
         unit_meta[u] = m;
@@ -1165,14 +1177,14 @@ mla_sm100_merge_kernel(const int4* __restrict__ unit_meta, const float* __restri
 // host side
 // ---------------------------------------------------------------------------
 
-// The pool viewed as [chunk (9)][row][64 columns]: one box loads two 64-column
+// The pool viewed as [chunk (9)][row][64 columns]: one box loads four 64-column
 // chunks of the same 64 rows into consecutive 8 KB blocks.
 bool make_map_chunks(CUtensorMap* m, const void* base, uint64_t rows) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     const cuuint64_t dims[3] = {64, rows, kChunks};
     const cuuint64_t strides[2] = {kRow * 2, 128};
-    const cuuint32_t box[3] = {64, 64, 2};
+    const cuuint32_t box[3] = {64, 64, 4};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1182,14 +1194,16 @@ bool make_map_chunks(CUtensorMap* m, const void* base, uint64_t rows) {
 size_t r256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct Sm100Ws {
-    size_t prefix, kv, meta, cinfo, part_lse, part_o, total;
+    size_t prefix, tprefix, kv, kv_cta, meta, cinfo, part_lse, part_o, total;
 };
 
 Sm100Ws sm100_ws(int U) {
     Sm100Ws w;
     w.prefix = 0;
-    w.kv = w.prefix + r256(static_cast<size_t>(U + 1) * 4);
-    w.meta = w.kv + r256(static_cast<size_t>(U) * 4);
+    w.tprefix = w.prefix + r256(static_cast<size_t>(U + 1) * 4);
+    w.kv = w.tprefix + r256(static_cast<size_t>(U + 1) * 4);
+    w.kv_cta = w.kv + r256(static_cast<size_t>(U) * 4);
+    w.meta = w.kv_cta + r256(static_cast<size_t>(2 * kClusters) * U * 4);
     w.cinfo = w.meta + r256(static_cast<size_t>(U) * 16);
     w.part_lse = w.cinfo + r256(static_cast<size_t>(kClusters) * 16);
     w.part_o = w.part_lse + r256(static_cast<size_t>(kClusters + U) * 128 * 4);
@@ -1232,11 +1246,11 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int max_splits,
         !make_map_2d(&k.tm_qa, P.q_abs, kDc, q_rows, kDc * 2, 64, 64) ||
         !make_map_2d(&k.tm_qr, P.q_r, kDr, q_rows, kDr * 2, 64, 64))
         return cudaErrorInvalidValue;
-    k.pool = P.pool;
     k.block_table = P.block_table;
     k.seq_lens = P.seq_lens;
     k.prefix = reinterpret_cast<int32_t*>(base + w.prefix);
     k.unit_kv = reinterpret_cast<int32_t*>(base + w.kv);
+    k.kv_cta = reinterpret_cast<int32_t*>(base + w.kv_cta);
     k.unit_meta = reinterpret_cast<int4*>(base + w.meta);
     k.cluster_info = reinterpret_cast<const int4*>(base + w.cinfo);
     k.out_latent = P.out_latent;
@@ -1261,7 +1275,8 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int max_splits,
     cudaError_t e;
     if (!k.in_kernel_schedule) {
         e = launch_pdl(mla_sm100_schedule_kernel, dim3(1), dim3(1024), 0, stream, P.seq_lens, P.T_q, n_hb,
-                       P.max_blocks, max_splits, U, k.prefix, k.unit_kv, k.unit_meta,
+                       P.max_blocks, max_splits, U, k.prefix, reinterpret_cast<int32_t*>(base + w.tprefix),
+                       k.unit_kv, k.unit_meta,
                        reinterpret_cast<int4*>(base + w.cinfo), P.status);
         if (e != cudaSuccess) return e;
     }

@@ -112,11 +112,9 @@ __device__ __forceinline__ void tma_load_2d_pair_normal(uint32_t dst, const void
         : "memory");
 }
 
-// Bring `bytes` (multiple of 16, 16-byte aligned address) of contiguous
-// global memory into L2; no completion tracking, no shared memory involved.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* gaddr, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gaddr)), "r"(bytes)
-                 : "memory");
+// Bring the 128-byte line holding `gaddr` into L2 (no completion tracking).
+__device__ __forceinline__ void prefetch_l2_line(const void* gaddr) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(gaddr)) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {

@@ -136,11 +136,12 @@ def test_split_count_invariance(M, splits, impl):
     if impl == 1:
         assert parts == [splits if splits else parts[0]] * U
         return
-    # tensor-core decode: 16, 1 and 9 pages over 74 SM pairs; the bound caps
-    # the parts of every unit, and each unit is split as far as the bound and
-    # its page count allow (the equal cut puts every page in its own range)
-    pages = [16, 1, 9]
-    want = [min(splits, n) if splits else n for n in pages]
+    # tensor-core decode: 4, 1 and 3 tiles of 256 keys over 74 SM pairs; the
+    # bound caps the parts of every unit, and each unit is split as far as the
+    # bound and its tile count allow (the equal cut gives every tile its own
+    # range)
+    tiles = [4, 1, 3]
+    want = [min(splits, n) if splits else n for n in tiles]
     assert parts == want, (splits, parts)
 
 
