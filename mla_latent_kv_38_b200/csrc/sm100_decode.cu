@@ -62,7 +62,13 @@
 namespace mla {
 namespace {
 
-constexpr int kThreads = 384;   // 12 warps: S loads, S MMAs, P.V MMAs / prefetch, V loads, 8 x softmax
+constexpr int kThreads = 384;   // 12 warps: S loads, S MMAs, P.V MMAs, V loads, 8 x softmax
+// Registers per thread: 168 at launch (65,536 / 384, rounded down to 8); then
+// the load / MMA warpgroup gives registers up to the two softmax warpgroups.
+constexpr uint32_t kRegsLaunch = 168;
+constexpr uint32_t kRegsIssue = 64;
+constexpr uint32_t kRegsSoftmax = 216;
+static_assert(128 * kRegsIssue + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
 constexpr int kClusters = 74;                     // 148 SMs / 2
 constexpr int kDc = 512, kDr = 64, kRow = 576;    // row = c^KV || k^R
 constexpr int kPage = 64;                         // cache rows per page (TMA box height)
@@ -131,6 +137,8 @@ struct Sm100Params {
     CUtensorMap tm_pool_v;    // pool as [chunk][rows][64], box 64 cols x 64 rows x 4 chunks
     CUtensorMap tm_qa;        // q_abs as [n_tok*n_h][512], box 64 x 64
     CUtensorMap tm_qr;        // q_r   as [n_tok*n_h][64],  box 64 x 64
+    CUtensorMap tm_out;       // out_latent as [n_tok*n_h][512] bf16, box 64 x 32 (stores)
+    CUtensorMap tm_part;      // part_o as [(C+U)*128][512] fp32, box 32 x 32 (stores)
     const int32_t* block_table;
     const int32_t* seq_lens;
     int32_t* prefix;          // (U + 1) exclusive prefix of pages per unit (schedule kernel only)
@@ -442,7 +450,6 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     auto leader_bar = [&](int i) { return ptx::map_to_rank(bar(i), 0); };
     const uint64_t tmo = p.timeout_ns;
 
-    griddep_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSRing; ++s) {
             ptx::mbar_init(bar(BAR_SR_FULL + s), 1);
@@ -576,213 +583,220 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     };
     auto walker = [&](TileWalker& w) { w.init(kv_base, kv_off, u0, ubeg0, g0, g1, p.n_hb, p.T_q); };
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ S stream
-        // Entry c of a tile holds column chunk c (64 columns) of this CTA's two
-        // pages (keys) and of its 64 query rows, one 8 KB box each; the query is
-        // re-read from L2 with every tile, which leaves the shared memory to
-        // the rings (the loads run at DRAM latency, so the bytes in flight set
-        // the rate).  A thread's TMA copies run one after another, so ring slot
-        // s is issued by its own group of lanes 4g + {0, 1, 2}, g = s mod
-        // kSLaneGroups: lane j = 0, 1 loads own page j, lane 2 the query chunk.
-        // The group's lane 0 in the leader CTA arms the full barrier with both
-        // CTAs' bytes.  The page lanes hold the block of their page for tiles
-        // i, i+1, i+2 in b0, b1, b2.
-        const int grp = lane >> 2, j = lane & 3;
-        const bool active = grp < kSLaneGroups && j < 3;
-        const int my_pg = 2 * static_cast<int>(rank) + (j & 1);
-        TileWalker w, wa;
-        walker(w);
-        walker(wa);
-        int b0 = 0, b1 = 0, b2 = 0;
-        bool h0 = false, h1 = false, h2 = false;
-        // (the loads are unconditional, to a valid entry, so that nothing waits
-        // for them until their value is used a tile or two later)
-        auto look = [&](int& b, bool& h) {
-            h = false;
-            if (!wa.done()) {
-                const Tile t = wa.next();
-                h = active && j < 2 && my_pg < t.np;
-                b = load_blk(t, min(my_pg, t.np - 1));
-            }
-        };
-        look(b0, h0);
-        look(b1, h1);
-        look(b2, h2);
-        int e = 0;
-        bool ok = g0 < g1;
-        while (ok && !w.done()) {
-            const Tile cur = w.next();
-            const int qrow = cur.bt * p.n_h + cur.hb * 128 + 64 * static_cast<int>(rank);
-            const int row = h0 ? blk_row(b0) : 0;
-            const uint32_t tx = static_cast<uint32_t>(cur.np + 2) * kBox;    // both CTAs' page and query chunks
-            for (int c = 0; c < kChunks; ++c, ++e) {
-                const int slot = e % kSRing;
-                bool good = true;
-                if (active && grp == slot % kSLaneGroups) {
-                    good = wait_bar(bar(BAR_SR_EMPTY + slot), ((e / kSRing) & 1) ^ 1, abort_flag, p.status, tmo);
-                    if (good && j == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_SR_FULL + slot), tx);
-                    const bool q_lane = j == 2;
-                    const bool withheld = p.withhold_load && rank == 0 && e == 0 && j == 0;
-                    if (good && (q_lane || h0) && !withheld) {
-                        const void* tm = q_lane ? (c < 8 ? static_cast<const void*>(&p.tm_qa) : &p.tm_qr) : &p.tm_pool;
-                        const int bx = q_lane ? (c < 8 ? 64 * c : 0) : 64 * c;
-                        ptx::tma_load_2d_pair_normal(sbase + kOffSRing + slot * kSEntry + j * kBox, tm, bx,
-                                                     q_lane ? qrow : row, leader_bar(BAR_SR_FULL + slot));
-                    }
-                }
-                if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
-            }
-            b0 = b1; h0 = h1;
-            b1 = b2; h1 = h2;
-            look(b2, h2);
-        }
-    } else if (warp == 3) {
-        // ------------------------------------------------------------ V stream
-        // Entry per page: this CTA's latent chunks 4r .. 4r+3 of the page, one
-        // 3-D box, issued by lane (slot) so that consecutive copies come from
-        // different threads.  Lane pg < 4 holds the block of page pg of the
-        // current tile (v0) and of the next one (v1).
-        const uint64_t pol_v = ptx::l2_policy_evict_first();   // last use of these lines
-        TileWalker w, wa;
-        walker(w);
-        walker(wa);
-        int v0 = 0, v1 = 0;
-        auto look = [&](int& v) {
-            if (!wa.done()) {
-                const Tile t = wa.next();
-                v = load_blk(t, min(lane, t.np - 1));
-            }
-        };
-        look(v0);
-        look(v1);
-        int e = 0;
-        bool ok = g0 < g1;
-        while (ok && !w.done()) {
-            const Tile cur = w.next();
-            for (int pg = 0; pg < cur.np && ok; ++pg, ++e) {
-                const int row = blk_row(__shfl_sync(0xffffffffu, v0, pg));
-                const int slot = e % kVRing;
-                bool good = true;
-                if (lane == slot) {
-                    good = wait_bar(bar(BAR_VR_EMPTY + slot), ((e / kVRing) & 1) ^ 1, abort_flag, p.status, tmo);
-                    if (good && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_VR_FULL + slot), 2 * kVEntry);
-                    if (good)
-                        ptx::tma_load_3d_pair(sbase + kOffVRing + slot * kVEntry, &p.tm_pool_v, 0, row,
-                                              4 * static_cast<int>(rank), leader_bar(BAR_VR_FULL + slot), pol_v);
-                }
-                if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
-            }
-            v0 = v1;
-            look(v1);
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ S = Q K^T issuer
-        // S(i) occupies entries 9 i .. 9 i + 8 of the S ring (keys as B, query as A).
-        if (rank == 0 && lane == 0 && g0 < g1) {
-            TileWalker w;
+    if (warp < 4) {
+        // Warpgroup 0 (loads and MMA issue) needs few registers: it gives them to
+        // the softmax warpgroups (setmaxnreg, per warpgroup, at the top of each
+        // branch so that the compiler budgets each branch on its own).
+        ptx::regs_dec<kRegsIssue>();
+        if (warp == 0) {
+            // ------------------------------------------------------------ S stream
+            // Entry c of a tile holds column chunk c (64 columns) of this CTA's two
+            // pages (keys) and of its 64 query rows, one 8 KB box each; the query is
+            // re-read from L2 with every tile, which leaves the shared memory to
+            // the rings (the loads run at DRAM latency, so the bytes in flight set
+            // the rate).  A thread's TMA copies run one after another, so ring slot
+            // s is issued by its own group of lanes 4g + {0, 1, 2}, g = s mod
+            // kSLaneGroups: lane j = 0, 1 loads own page j, lane 2 the query chunk.
+            // The group's lane 0 in the leader CTA arms the full barrier with both
+            // CTAs' bytes.  The page lanes hold the block of their page for tiles
+            // i, i+1, i+2 in b0, b1, b2.
+            const int grp = lane >> 2, j = lane & 3;
+            const bool active = grp < kSLaneGroups && j < 3;
+            const int my_pg = 2 * static_cast<int>(rank) + (j & 1);
+            TileWalker w, wa;
             walker(w);
-            int i = 0;
-            bool ok = true;
+            walker(wa);
+            int b0 = 0, b1 = 0, b2 = 0;
+            bool h0 = false, h1 = false, h2 = false;
+            // (the loads are unconditional, to a valid entry, so that nothing waits
+            // for them until their value is used a tile or two later)
+            auto look = [&](int& b, bool& h) {
+                h = false;
+                if (!wa.done()) {
+                    const Tile t = wa.next();
+                    h = active && j < 2 && my_pg < t.np;
+                    b = load_blk(t, min(my_pg, t.np - 1));
+                }
+            };
+            look(b0, h0);
+            look(b1, h1);
+            look(b2, h2);
+            int e = 0;
+            bool ok = g0 < g1;
             while (ok && !w.done()) {
-                w.next();
-                const int e0 = kChunks * i;
-                const int sb = i & 1;
-                if (!(ok = wait_bar(bar(BAR_S_FREE + sb), ((i >> 1) & 1) ^ 1, abort_flag, p.status, tmo))) break;
-                ptx::tc_fence_after();   // the softmax's reads of this S buffer are done
-                for (int c = 0; c < kChunks; ++c) {
-                    const int e = e0 + c;
-                    if (!(ok = wait_bar(bar(BAR_SR_FULL + e % kSRing), (e / kSRing) & 1, abort_flag, p.status, tmo)))
-                        break;
-                    const uint32_t ent = sbase + kOffSRing + (e % kSRing) * kSEntry;
-                    const uint64_t b0 = ptx::smem_desc_sw128(ent, 16, 1024);
-                    const uint64_t a0 = ptx::smem_desc_sw128(ent + 2 * kBox, 16, 1024);
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const uint64_t a = a0 + static_cast<uint64_t>((32 * k4) >> 4);
-                        const uint64_t bd = b0 + static_cast<uint64_t>((32 * k4) >> 4);
-                        ptx::mma_pair_ss(tmem_base + kTmemS + 128 * sb, a, bd, kIdescS, (c | k4) ? 1u : 0u);
+                const Tile cur = w.next();
+                const int qrow = cur.bt * p.n_h + cur.hb * 128 + 64 * static_cast<int>(rank);
+                const int row = h0 ? blk_row(b0) : 0;
+                const uint32_t tx = static_cast<uint32_t>(cur.np + 2) * kBox;    // both CTAs' page and query chunks
+                for (int c = 0; c < kChunks; ++c, ++e) {
+                    const int slot = e % kSRing;
+                    bool good = true;
+                    if (active && grp == slot % kSLaneGroups) {
+                        good = wait_bar(bar(BAR_SR_EMPTY + slot), ((e / kSRing) & 1) ^ 1, abort_flag, p.status, tmo);
+                        if (good && j == 0 && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_SR_FULL + slot), tx);
+                        const bool q_lane = j == 2;
+                        const bool withheld = p.withhold_load && rank == 0 && e == 0 && j == 0;
+                        if (good && (q_lane || h0) && !withheld) {
+                            const void* tm = q_lane ? (c < 8 ? static_cast<const void*>(&p.tm_qa) : &p.tm_qr) : &p.tm_pool;
+                            const int bx = q_lane ? (c < 8 ? 64 * c : 0) : 64 * c;
+                            ptx::tma_load_2d_pair_normal(sbase + kOffSRing + slot * kSEntry + j * kBox, tm, bx,
+                                                         q_lane ? qrow : row, leader_bar(BAR_SR_FULL + slot));
+                        }
                     }
-                    ptx::mma_commit_pair(bar(BAR_SR_EMPTY + e % kSRing), 0x3);
+                    if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
                 }
-                if (!ok) break;
-                ptx::mma_commit_pair(bar(BAR_S_FULL + sb), 0x3);
-                ++i;
+                b0 = b1; h0 = h1;
+                b1 = b2; h1 = h2;
+                look(b2, h2);
             }
-            if (!ok) {
-                // let every MMA this thread issued finish before the teardown frees anything
-                ptx::mma_commit_pair(bar(BAR_DRAIN), 0x1);
-                const uint64_t t0 = ptx::global_timer_ns();
-                while (!ptx::mbar_try_wait(bar(BAR_DRAIN), 0) && ptx::global_timer_ns() - t0 < tmo) {
+        } else if (warp == 3) {
+            // ------------------------------------------------------------ V stream
+            // Entry per page: this CTA's latent chunks 4r .. 4r+3 of the page, one
+            // 3-D box, issued by lane (slot) so that consecutive copies come from
+            // different threads.  Lane pg < 4 holds the block of page pg of the
+            // current tile (v0) and of the next one (v1).
+            const uint64_t pol_v = ptx::l2_policy_evict_first();   // last use of these lines
+            TileWalker w, wa;
+            walker(w);
+            walker(wa);
+            int v0 = 0, v1 = 0;
+            auto look = [&](int& v) {
+                if (!wa.done()) {
+                    const Tile t = wa.next();
+                    v = load_blk(t, min(lane, t.np - 1));
                 }
+            };
+            look(v0);
+            look(v1);
+            int e = 0;
+            bool ok = g0 < g1;
+            while (ok && !w.done()) {
+                const Tile cur = w.next();
+                for (int pg = 0; pg < cur.np && ok; ++pg, ++e) {
+                    const int row = blk_row(__shfl_sync(0xffffffffu, v0, pg));
+                    const int slot = e % kVRing;
+                    bool good = true;
+                    if (lane == slot) {
+                        good = wait_bar(bar(BAR_VR_EMPTY + slot), ((e / kVRing) & 1) ^ 1, abort_flag, p.status, tmo);
+                        if (good && rank == 0) ptx::mbar_arrive_expect_tx(bar(BAR_VR_FULL + slot), 2 * kVEntry);
+                        if (good)
+                            ptx::tma_load_3d_pair(sbase + kOffVRing + slot * kVEntry, &p.tm_pool_v, 0, row,
+                                                  4 * static_cast<int>(rank), leader_bar(BAR_VR_FULL + slot), pol_v);
+                    }
+                    if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
+                }
+                v0 = v1;
+                look(v1);
             }
-        }
-    } else if (warp == 2) {
-        if (rank == 0) {
-            // -------------------------------------------------------- O += P V issuer
-            // V(i) occupies the next np entries of the V ring (one per page).
-            if (lane == 0 && g0 < g1) {
+        } else if (warp == 1) {
+            // ------------------------------------------------------------ S = Q K^T issuer
+            // S(i) occupies entries 9 i .. 9 i + 8 of the S ring (keys as B, query as A).
+            if (rank == 0 && lane == 0 && g0 < g1) {
                 TileWalker w;
                 walker(w);
-                int i = 0, tails = 0, e = 0;
+                int i = 0;
                 bool ok = true;
-                const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffP, 16, 1024);
                 while (ok && !w.done()) {
-                    const Tile t = w.next();
-                    const bool tail = t.unit_end && (t.kv % kPage) != 0;
-                    // P is written in two halves: keys [0,128) (pages 0, 1) by the
-                    // softmax warps of TMEM lanes 0-63, keys [128,256) by those of
-                    // lanes 64-127; each half is released as soon as its pages'
-                    // MMAs complete.
-                    for (int pg = 0; pg < 4 && ok; ++pg) {
-                        if (pg == 0 || pg == 2) {
-                            if (pg == 2) ptx::mma_commit_pair(bar(BAR_P_FREE + 0), 0x3);
-                            if (!(ok = wait_bar(bar(BAR_P_FULL + (pg >> 1)), i & 1, abort_flag, p.status, tmo))) break;
-                            ptx::tc_fence_after();
-                        }
-                        if (pg >= t.np) continue;
-                        if (tail && pg == t.np - 1) {
-                            // the unit's last page holds rows past the end: once its V
-                            // entry has landed, the softmax warps of both CTAs zero those
-                            // rows (entries are consumed in ring order, so the earlier
-                            // pages' slots are already free for this load)
-                            if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag,
-                                                p.status, tmo)))
-                                break;
-                            ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 0));
-                            ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 1));
-                            if (!(ok = wait_bar(bar(BAR_TAIL_DONE), tails & 1, abort_flag, p.status, tmo))) break;
-                            ++tails;
-                        }
-                        if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status, tmo)))
+                    w.next();
+                    const int e0 = kChunks * i;
+                    const int sb = i & 1;
+                    if (!(ok = wait_bar(bar(BAR_S_FREE + sb), ((i >> 1) & 1) ^ 1, abort_flag, p.status, tmo))) break;
+                    ptx::tc_fence_after();   // the softmax's reads of this S buffer are done
+                    for (int c = 0; c < kChunks; ++c) {
+                        const int e = e0 + c;
+                        if (!(ok = wait_bar(bar(BAR_SR_FULL + e % kSRing), (e / kSRing) & 1, abort_flag, p.status, tmo)))
                             break;
-                        for (int h = 0; h < 2; ++h) {
-                            const uint64_t b0 = ptx::smem_desc_sw128(
-                                sbase + kOffVRing + (e % kVRing) * kVEntry + h * 2 * kBox, kBox, 1024);
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk) {
-                                const uint64_t a = a0 + static_cast<uint64_t>((pg * kBox + 32 * kk) >> 4);
-                                const uint64_t bd = b0 + static_cast<uint64_t>((2048 * kk) >> 4);
-                                ptx::mma_pair_ss(tmem_base + kTmemO + 128 * h, a, bd, kIdescPV,
-                                                 (t.first && pg == 0 && kk == 0) ? 0u : 1u);
-                            }
+                        const uint32_t ent = sbase + kOffSRing + (e % kSRing) * kSEntry;
+                        const uint64_t b0 = ptx::smem_desc_sw128(ent, 16, 1024);
+                        const uint64_t a0 = ptx::smem_desc_sw128(ent + 2 * kBox, 16, 1024);
+    #pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const uint64_t a = a0 + static_cast<uint64_t>((32 * k4) >> 4);
+                            const uint64_t bd = b0 + static_cast<uint64_t>((32 * k4) >> 4);
+                            ptx::mma_pair_ss(tmem_base + kTmemS + 128 * sb, a, bd, kIdescS, (c | k4) ? 1u : 0u);
                         }
-                        ptx::mma_commit_pair(bar(BAR_VR_EMPTY + e % kVRing), 0x3);
-                        ++e;
+                        ptx::mma_commit_pair(bar(BAR_SR_EMPTY + e % kSRing), 0x3);
                     }
                     if (!ok) break;
-                    ptx::mma_commit_pair(bar(BAR_P_FREE + 1), 0x3);
+                    ptx::mma_commit_pair(bar(BAR_S_FULL + sb), 0x3);
                     ++i;
                 }
                 if (!ok) {
-                    ptx::mma_commit_pair(bar(BAR_DRAIN_PV), 0x1);
+                    // let every MMA this thread issued finish before the teardown frees anything
+                    ptx::mma_commit_pair(bar(BAR_DRAIN), 0x1);
                     const uint64_t t0 = ptx::global_timer_ns();
-                    while (!ptx::mbar_try_wait(bar(BAR_DRAIN_PV), 0) && ptx::global_timer_ns() - t0 < tmo) {
+                    while (!ptx::mbar_try_wait(bar(BAR_DRAIN), 0) && ptx::global_timer_ns() - t0 < tmo) {
+                    }
+                }
+            }
+        } else if (warp == 2) {
+            if (rank == 0) {
+                // -------------------------------------------------------- O += P V issuer
+                // V(i) occupies the next np entries of the V ring (one per page).
+                if (lane == 0 && g0 < g1) {
+                    TileWalker w;
+                    walker(w);
+                    int i = 0, tails = 0, e = 0;
+                    bool ok = true;
+                    const uint64_t a0 = ptx::smem_desc_sw128(sbase + kOffP, 16, 1024);
+                    while (ok && !w.done()) {
+                        const Tile t = w.next();
+                        const bool tail = t.unit_end && (t.kv % kPage) != 0;
+                        // P is written in two halves: keys [0,128) (pages 0, 1) by the
+                        // softmax warps of TMEM lanes 0-63, keys [128,256) by those of
+                        // lanes 64-127; each half is released as soon as its pages'
+                        // MMAs complete.
+                        for (int pg = 0; pg < 4 && ok; ++pg) {
+                            if (pg == 0 || pg == 2) {
+                                if (pg == 2) ptx::mma_commit_pair(bar(BAR_P_FREE + 0), 0x3);
+                                if (!(ok = wait_bar(bar(BAR_P_FULL + (pg >> 1)), i & 1, abort_flag, p.status, tmo))) break;
+                                ptx::tc_fence_after();
+                            }
+                            if (pg >= t.np) continue;
+                            if (tail && pg == t.np - 1) {
+                                // the unit's last page holds rows past the end: once its V
+                                // entry has landed, the softmax warps of both CTAs zero those
+                                // rows (entries are consumed in ring order, so the earlier
+                                // pages' slots are already free for this load)
+                                if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag,
+                                                    p.status, tmo)))
+                                    break;
+                                ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 0));
+                                ptx::mbar_arrive_cluster(ptx::map_to_rank(bar(BAR_TAIL_READY), 1));
+                                if (!(ok = wait_bar(bar(BAR_TAIL_DONE), tails & 1, abort_flag, p.status, tmo))) break;
+                                ++tails;
+                            }
+                            if (!(ok = wait_bar(bar(BAR_VR_FULL + e % kVRing), (e / kVRing) & 1, abort_flag, p.status, tmo)))
+                                break;
+                            for (int h = 0; h < 2; ++h) {
+                                const uint64_t b0 = ptx::smem_desc_sw128(
+                                    sbase + kOffVRing + (e % kVRing) * kVEntry + h * 2 * kBox, kBox, 1024);
+    #pragma unroll
+                                for (int kk = 0; kk < 4; ++kk) {
+                                    const uint64_t a = a0 + static_cast<uint64_t>((pg * kBox + 32 * kk) >> 4);
+                                    const uint64_t bd = b0 + static_cast<uint64_t>((2048 * kk) >> 4);
+                                    ptx::mma_pair_ss(tmem_base + kTmemO + 128 * h, a, bd, kIdescPV,
+                                                     (t.first && pg == 0 && kk == 0) ? 0u : 1u);
+                                }
+                            }
+                            ptx::mma_commit_pair(bar(BAR_VR_EMPTY + e % kVRing), 0x3);
+                            ++e;
+                        }
+                        if (!ok) break;
+                        ptx::mma_commit_pair(bar(BAR_P_FREE + 1), 0x3);
+                        ++i;
+                    }
+                    if (!ok) {
+                        ptx::mma_commit_pair(bar(BAR_DRAIN_PV), 0x1);
+                        const uint64_t t0 = ptx::global_timer_ns();
+                        while (!ptx::mbar_try_wait(bar(BAR_DRAIN_PV), 0) && ptx::global_timer_ns() - t0 < tmo) {
+                        }
                     }
                 }
             }
         }
     } else {
+        ptx::regs_inc<kRegsSoftmax>();
         // ------------------------------------------------------------ softmax + epilogue
         // Eight warps, two per tensor-memory lane quadrant: a thread owns lane l
         // (head row m, key half hi of the S tile, latent half hi of O) and
@@ -949,40 +963,64 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 const bool whole = t.whole;
                 const size_t grow = static_cast<size_t>(bt) * p.n_h + hb * 128 + head_in_unit;
                 const size_t slot = static_cast<size_t>(cluster) + t.u;
-                // Each thread writes its own row segment straight from the
-                // registers: 128 latent columns (bf16 when the unit is whole,
-                // else the fp32 partial), read from tensor memory 64 at a time.
+                // This warp's 32 rows (consecutive heads) x the thread's 128
+                // latent columns go out through a 4 KB tile of the free P buffer,
+                // written in the 128-byte swizzled layout of a TMA store box (a
+                // thread's row of 128 bytes, 16-byte chunk k at k ^ (row & 7)),
+                // so each round is one bulk tensor store: 4 rounds of 32 fp32
+                // columns for a partial, 2 rounds of 64 bf16 columns otherwise.
                 const int h = cg;   // this thread's 128 O columns
                 const int col0 = 128 * h + (hi ? 256 : 0);
+                unsigned char* stage = smem + kOffP + sw * 4096;
+                const uint32_t stage_u = sbase + kOffP + sw * 4096;
+                unsigned char* my_row = stage + lane * 128;
+                const int x7 = lane & 7;
+                const int row0 = whole ? static_cast<int>(grow - lane)
+                                       : static_cast<int>(slot * 128 + head_in_unit - lane);
 #pragma unroll 1
-                for (int q2 = 0; q2 < 2; ++q2) {
-                    uint32_t o[2][32];
-                    ptx::tmem_ld32(t_lane + kTmemO + 128 * h + 64 * q2, o[0]);
-                    ptx::tmem_ld32(t_lane + kTmemO + 128 * h + 64 * q2 + 32, o[1]);
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t o[32];
+                    ptx::tmem_ld32(t_lane + kTmemO + 128 * h + 32 * q, o);
                     ptx::tmem_wait_ld();
+                    if (!whole || (q & 1) == 0) {
+                        if (lane == 0) ptx::bulk_wait_read_all();   // the previous store has read the tile
+                        __syncwarp();
+                    }
+                    if (whole) {
+                        // columns 32q .. 32q + 31 are chunks 4 (q & 1) .. + 3 of the staged 64-column row
 #pragma unroll
-                    for (int qq = 0; qq < 2; ++qq) {
-                        const int col = col0 + 64 * q2 + 32 * qq;
-                        if (whole) {
-                            uint4* dst = reinterpret_cast<uint4*>(p.out_latent + grow * kDc + col);
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                uint4 wv;
-                                wv.x = pack_bf16x2(__uint_as_float(o[qq][8 * k + 0]) * inv, __uint_as_float(o[qq][8 * k + 1]) * inv);
-                                wv.y = pack_bf16x2(__uint_as_float(o[qq][8 * k + 2]) * inv, __uint_as_float(o[qq][8 * k + 3]) * inv);
-                                wv.z = pack_bf16x2(__uint_as_float(o[qq][8 * k + 4]) * inv, __uint_as_float(o[qq][8 * k + 5]) * inv);
-                                wv.w = pack_bf16x2(__uint_as_float(o[qq][8 * k + 6]) * inv, __uint_as_float(o[qq][8 * k + 7]) * inv);
-                                dst[k] = wv;
+                        for (int k = 0; k < 4; ++k) {
+                            uint4 wv;
+                            wv.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
+                            wv.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
+                            wv.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
+                            wv.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
+                            *reinterpret_cast<uint4*>(my_row + (((4 * (q & 1) + k) ^ x7) * 16)) = wv;
+                        }
+                        if (q & 1) {
+                            ptx::fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                ptx::tma_store_2d(&p.tm_out, stage_u, col0 + 64 * (q >> 1), row0);
+                                ptx::bulk_commit_group();
                             }
-                        } else {
-                            float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * 128 + head_in_unit) * kDc + col);
+                        }
+                    } else {
 #pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                dst[k] = make_float4(__uint_as_float(o[qq][4 * k]) * inv, __uint_as_float(o[qq][4 * k + 1]) * inv,
-                                                     __uint_as_float(o[qq][4 * k + 2]) * inv, __uint_as_float(o[qq][4 * k + 3]) * inv);
+                        for (int k = 0; k < 8; ++k)
+                            *reinterpret_cast<float4*>(my_row + ((k ^ x7) * 16)) =
+                                make_float4(__uint_as_float(o[4 * k]) * inv, __uint_as_float(o[4 * k + 1]) * inv,
+                                            __uint_as_float(o[4 * k + 2]) * inv, __uint_as_float(o[4 * k + 3]) * inv);
+                        ptx::fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            ptx::tma_store_2d(&p.tm_part, stage_u, col0 + 32 * q, row0);
+                            ptx::bulk_commit_group();
                         }
                     }
                 }
+                if (lane == 0) ptx::bulk_wait_read_all();   // the P buffer is written again by the next tile
+                __syncwarp();
                 if (!hi && cg == 0) {
                     if (whole) p.out_lse[grow] = lse;
                     else p.part_lse[slot * 128 + head_in_unit] = lse;
@@ -994,6 +1032,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     }
 
     // ---------------------------------------------------------------- teardown
+    if (warp >= 4 && lane == 0) ptx::bulk_wait_all();   // the epilogue's stores have completed
     if (*abort_flag) {
         // give copies still in flight time to land before shared memory is released
         const uint64_t t0 = ptx::global_timer_ns();
@@ -1005,6 +1044,9 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
     ptx::cluster_sync();
     ptx::tc_fence_after();
     if (warp == 1) ptx::tmem_dealloc_pair(tmem_base, kTmemCols);
+    // The merge kernel may start only now: launched while this grid still
+    // runs, its pending blocks slowed the decode down measurably.
+    griddep_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
@@ -1244,7 +1286,10 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int max_splits,
     if (!make_map_2d(&k.tm_pool, P.pool, kRow, pool_rows, kRow * 2, 64, 64) ||
         !make_map_chunks(&k.tm_pool_v, P.pool, pool_rows) ||
         !make_map_2d(&k.tm_qa, P.q_abs, kDc, q_rows, kDc * 2, 64, 64) ||
-        !make_map_2d(&k.tm_qr, P.q_r, kDr, q_rows, kDr * 2, 64, 64))
+        !make_map_2d(&k.tm_qr, P.q_r, kDr, q_rows, kDr * 2, 64, 64) ||
+        !make_map_2d(&k.tm_out, P.out_latent, kDc, q_rows, kDc * 2, 64, 32) ||
+        !make_map_2d_f32(&k.tm_part, base + w.part_o, kDc, static_cast<uint64_t>(kClusters + U) * 128, kDc * 4, 32,
+                         32))
         return cudaErrorInvalidValue;
     k.block_table = P.block_table;
     k.seq_lens = P.seq_lens;
