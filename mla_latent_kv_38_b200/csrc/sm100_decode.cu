@@ -99,7 +99,7 @@ constexpr int kSliceCap = static_cast<int>((kSmemBytes - 1024 - kOffSlice) / 4);
 // memory when they fit, else to the CTA's own region of the workspace.
 constexpr int kInKernelUnits = 2048;
 static_assert(kOffSlice + 1024 <= kSmemBytes, "shared memory budget");
-static_assert(4 * (4 * kInKernelUnits + 2 + kClusters + 1 + 32) <= static_cast<int>(kOffP - kOffSRing), "schedule scratch");
+static_assert(4 * (5 * kInKernelUnits + 3 + kClusters + 1 + 48) <= static_cast<int>(kOffP - kOffSRing), "schedule scratch");
 static_assert(4 * (kClusters + 1) <= 320, "cut area");
 static_assert(kSRing % kSLaneGroups == 0, "each lane group keeps its own ring slots");
 static_assert(4 * kSLaneGroups <= 32, "lane groups of the S producer warp");
@@ -129,7 +129,6 @@ constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 256, 0, 0);
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 256, 0, 1);
 
 constexpr uint32_t kSuspendHintNs = 100000;      // a waiting thread sleeps up to 0.1 ms per try
-constexpr int kSchedSmemUnits = 4096;             // units whose prefixes the schedule kernel keeps in shared memory
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
 
 struct Sm100Params {
@@ -201,16 +200,30 @@ __device__ __forceinline__ int unit_of_page(const int32_t* pf, int U, int g) {
 
 // Work is cut at whole tiles (4 pages, 256 keys, counted from each unit's
 // start), so that a range that crosses a unit boundary carries no extra
-// partial tile.  Raw cut c (in tiles): floor(c Tt / C), Tt = tf[U] the total
-// tiles.  With max_splits = s > 0 it moves up to the next allowed cut, where
-// unit u's P tiles are cut into k = min(s, P) pieces at tf[u] + floor(j P / k),
-// j = 0 .. k, so no unit lies in more than s ranges.
-__device__ int raw_cut_tile(int c, int Tt, const int32_t* tf, int U, int max_splits) {
+// partial tile.  The cut balances a cost per cluster: 4 per tile (quarter
+// tiles) plus kSegCost for every unit segment it starts, which stands for
+// the epilogue and pipeline restart of a segment (measured at about 1.5
+// tiles).  wf is the exclusive prefix of the units' costs, W = wf[U]; raw cut
+// c lies at cost floor(c W / C), rounded to the nearest tile of the unit it
+// falls in.  With max_splits = s > 0 it then moves up to the next allowed
+// cut, where unit u's P tiles are cut into k = min(s, P) pieces at
+// tf[u] + floor(j P / k), j = 0 .. k, so no unit lies in more than s ranges.
+constexpr int kSegCost = 6;
+
+__device__ __forceinline__ int unit_cost(int tiles) { return 4 * tiles + (tiles > 0 ? kSegCost : 0); }
+
+__device__ int raw_cut_tile(int c, int Tt, const int32_t* tf, const int32_t* wf, int U, int max_splits) {
     if (c <= 0) return 0;
     if (c >= kClusters) return Tt;
-    const int g = static_cast<int>(static_cast<long long>(c) * Tt / kClusters);
+    const int W = wf[U];
+    const int x = static_cast<int>(static_cast<long long>(c) * W / kClusters);
+    if (x >= W) return Tt;
+    int u = unit_of_page(wf, U, x);           // wf[u] <= x < wf[u + 1]
+    const int tiles = tf[u + 1] - tf[u];
+    const int d = x - wf[u] - kSegCost;
+    const int g = tf[u] + (d <= 0 ? 0 : min(tiles, (d + 2) / 4));
     if (max_splits <= 0 || g >= Tt) return g;
-    const int u = unit_of_page(tf, U, g);
+    u = unit_of_page(tf, U, g);
     const int a = tf[u], P = tf[u + 1] - a;   // a <= g < tf[u + 1], so P > 0
     const int k = min(max_splits, P);
     const int j = static_cast<int>((static_cast<long long>(g - a) * k + P - 1) / P);   // ceil((g-a) k / P)
@@ -229,10 +242,10 @@ __device__ int tile_to_page(int gt, int Tt, int T, const int32_t* tf, const int3
 // non-empty range comes before every empty one (a unit's ranges are always
 // consecutive clusters).  All threads of the block call it; tmp holds C + 1
 // ints of scratch.
-__device__ void compute_cuts(int* cuts, int* tmp, const int32_t* pf, const int32_t* tf, int U, int T, int Tt,
-                             int max_splits) {
+__device__ void compute_cuts(int* cuts, int* tmp, const int32_t* pf, const int32_t* tf, const int32_t* wf, int U,
+                             int T, int Tt, int max_splits) {
     for (int c = threadIdx.x; c <= kClusters; c += blockDim.x)
-        tmp[c] = tile_to_page(raw_cut_tile(c, Tt, tf, U, max_splits), Tt, T, tf, pf, U);
+        tmp[c] = tile_to_page(raw_cut_tile(c, Tt, tf, wf, U, max_splits), Tt, T, tf, pf, U);
     __syncthreads();
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
@@ -363,68 +376,61 @@ struct TileWalker {
     }
 };
 
-// Block-wide exclusive scans of the units' page and tile counts into pf[0 ..
-// U] and tf[0 .. U] (U <= kInKernelUnits); every thread of the CTA takes
-// part; warp_tot holds 2 x 12 ints of scratch.  Returns {T, Tt} = {pf[U], tf[U]}.
-__device__ int2 schedule_scan(int* pf, int* tf, int* warp_tot, const int32_t* seq_lens, int U, int n_hb, int T_q,
-                              int max_blocks) {
+// Block-wide exclusive scans of the units' page counts, tile counts and cut
+// costs into pf, tf, wf[0 .. U] (U <= kInKernelUnits); every thread of the
+// CTA takes part; warp_tot holds 3 x 16 ints of scratch.  Returns {T, Tt}.
+__device__ int2 schedule_scan(int* pf, int* tf, int* wf, int* warp_tot, const int32_t* seq_lens, int U, int n_hb,
+                              int T_q, int max_blocks) {
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int per = (U + kThreads - 1) / kThreads;
     const int beg = min(U, tid * per), end = min(U, beg + per);
-    int lp = 0, lt = 0;
+    int loc[3] = {0, 0, 0};
     for (int u = beg; u < end; ++u) {
         const int pages = (unit_keys(seq_lens, u, n_hb, T_q, max_blocks) + kPage - 1) / kPage;
         const int tiles = (pages + kTilePages - 1) / kTilePages;
         pf[u + 1] = pages;
         tf[u + 1] = tiles;
-        lp += pages;
-        lt += tiles;
+        wf[u + 1] = unit_cost(tiles);
+        loc[0] += pages;
+        loc[1] += tiles;
+        loc[2] += unit_cost(tiles);
     }
-    int vp = lp, vt = lt;   // inclusive warp scans
+    int v[3] = {loc[0], loc[1], loc[2]};   // inclusive warp scans
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int yp = __shfl_up_sync(0xffffffffu, vp, o);
-        const int yt = __shfl_up_sync(0xffffffffu, vt, o);
-        if (lane >= o) {
-            vp += yp;
-            vt += yt;
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+            const int y = __shfl_up_sync(0xffffffffu, v[q], o);
+            if (lane >= o) v[q] += y;
         }
     }
-    if (lane == 31) {
-        warp_tot[w] = vp;
-        warp_tot[16 + w] = vt;
-    }
+    if (lane == 31)
+        for (int q = 0; q < 3; ++q) warp_tot[16 * q + w] = v[q];
     __syncthreads();
     if (w == 0) {
-        int xp = lane < kThreads / 32 ? warp_tot[lane] : 0;
-        int xt = lane < kThreads / 32 ? warp_tot[16 + lane] : 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int yp = __shfl_up_sync(0xffffffffu, xp, o);
-            const int yt = __shfl_up_sync(0xffffffffu, xt, o);
-            if (lane >= o) {
-                xp += yp;
-                xt += yt;
+        for (int q = 0; q < 3; ++q) {
+            int x = lane < kThreads / 32 ? warp_tot[16 * q + lane] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
             }
-        }
-        if (lane < kThreads / 32) {   // inclusive over warps
-            warp_tot[lane] = xp;
-            warp_tot[16 + lane] = xt;
+            if (lane < kThreads / 32) warp_tot[16 * q + lane] = x;   // inclusive over warps
         }
     }
     __syncthreads();
-    int rp = vp - lp + (w > 0 ? warp_tot[w - 1] : 0);
-    int rt = vt - lt + (w > 0 ? warp_tot[16 + w - 1] : 0);
+    int r[3];
+    for (int q = 0; q < 3; ++q) r[q] = v[q] - loc[q] + (w > 0 ? warp_tot[16 * q + w - 1] : 0);
     for (int u = beg; u < end; ++u) {
-        rp += pf[u + 1];
-        pf[u + 1] = rp;
-        rt += tf[u + 1];
-        tf[u + 1] = rt;
+        r[0] += pf[u + 1];
+        pf[u + 1] = r[0];
+        r[1] += tf[u + 1];
+        tf[u + 1] = r[1];
+        r[2] += wf[u + 1];
+        wf[u + 1] = r[2];
     }
-    if (tid == 0) {
-        pf[0] = 0;
-        tf[0] = 0;
-    }
+    if (tid == 0) pf[0] = tf[0] = wf[0] = 0;
     __syncthreads();
     return make_int2(pf[U], tf[U]);
 }
@@ -517,15 +523,16 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         // scratch: the ring area is unused until the loads start
         int* sc = reinterpret_cast<int*>(smem + kOffSRing);          // page prefix, U + 1
         int* tfx = sc + kInKernelUnits + 1;                           // tile prefix, U + 1
-        int* ctmp = tfx + kInKernelUnits + 1;                         // cut scratch, C + 1
+        int* wfx = tfx + kInKernelUnits + 1;                          // cost prefix, U + 1
+        int* ctmp = wfx + kInKernelUnits + 1;                         // cut scratch, C + 1
         int* lens = ctmp + kClusters + 1;                             // sequence lengths, B <= U
-        int* wtot = lens + kInKernelUnits;                            // scan scratch, 32
+        int* wtot = lens + kInKernelUnits;                            // scan scratch, 48
         for (int b = threadIdx.x; b < p.B; b += kThreads) lens[b] = __ldg(p.seq_lens + b);
         __syncthreads();
-        const int2 TT = schedule_scan(sc, tfx, wtot, lens, p.U, p.n_hb, p.T_q, p.max_blocks);
+        const int2 TT = schedule_scan(sc, tfx, wfx, wtot, lens, p.U, p.n_hb, p.T_q, p.max_blocks);
         const int T = TT.x;
         int* cuts = reinterpret_cast<int*>(smem + kOffCuts);
-        compute_cuts(cuts, ctmp, sc, tfx, p.U, T, TT.y, p.max_splits);
+        compute_cuts(cuts, ctmp, sc, tfx, wfx, p.U, T, TT.y, p.max_splits);
         g0 = cuts[cluster];
         g1 = cuts[cluster + 1];
         if (g0 < g1) {
@@ -1051,36 +1058,35 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
 
 // ---------------------------------------------------------------------------
 // Work schedule for very large unit counts (U > kInKernelUnits): the exclusive
-// prefixes of pages and tiles per unit, the units' key counts, the merge
-// metadata and each cluster's page range, computed by one block of 1024
+// prefixes of pages, tiles and cut costs per unit, the units' key counts, the
+// merge metadata and each cluster's page range, computed by one block of 1024
 // threads with the same cut rule as the decode kernel's own scan.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024)
 mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int T_q, int n_hb, int max_blocks,
                           int max_splits, int U, int32_t* __restrict__ prefix, int32_t* __restrict__ tprefix,
-                          int32_t* __restrict__ kv_out, int4* __restrict__ unit_meta, int4* __restrict__ cluster_info,
-                          int32_t* status) {
-    __shared__ int warp_tot[2][32];
-    __shared__ int carry[2];
-    __shared__ int pre_s[kSchedSmemUnits + 1];    // the prefixes again, for the searches below
-    __shared__ int tpre_s[kSchedSmemUnits + 1];
+                          int32_t* __restrict__ wprefix, int32_t* __restrict__ kv_out, int4* __restrict__ unit_meta,
+                          int4* __restrict__ cluster_info, int32_t* status) {
+    __shared__ int warp_tot[3][32];
+    __shared__ int carry[3];
     griddep_launch_dependents();
     griddep_wait();   // the workspace may still be read by an earlier decode call's kernels
-    const bool in_smem = U <= kSchedSmemUnits;
-    if (threadIdx.x == 0) carry[0] = carry[1] = 0;
+    if (threadIdx.x == 0) carry[0] = carry[1] = carry[2] = 0;
     __syncthreads();
+    int32_t* out[3] = {prefix, tprefix, wprefix};
     for (int base = 0; base < U; base += 1024) {
         const int u = base + threadIdx.x;
-        int v[2] = {0, 0};   // pages, tiles
+        int v[3] = {0, 0, 0};   // pages, tiles, cost
         if (u < U) {
             const int kv = unit_keys(seq_lens, u, n_hb, T_q, max_blocks);
             kv_out[u] = kv;
             v[0] = (kv + kPage - 1) / kPage;
             v[1] = (v[0] + kTilePages - 1) / kTilePages;
+            v[2] = unit_cost(v[1]);
         }
         const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {   // block inclusive scans
+        for (int q = 0; q < 3; ++q) {   // block inclusive scans
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, v[q], o);
@@ -1091,7 +1097,7 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int T_q, int n_h
         __syncthreads();
         if (w == 0) {
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
+            for (int q = 0; q < 3; ++q) {
                 int t = warp_tot[q][lane];
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -1102,40 +1108,29 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int T_q, int n_h
             }
         }
         __syncthreads();
-        const int ip = v[0] + (w > 0 ? warp_tot[0][w - 1] : 0) + carry[0];
-        const int it = v[1] + (w > 0 ? warp_tot[1][w - 1] : 0) + carry[1];
-        if (u < U) {
-            prefix[u + 1] = ip;
-            tprefix[u + 1] = it;
-            if (in_smem) {
-                pre_s[u + 1] = ip;
-                tpre_s[u + 1] = it;
-            }
-        }
-        if (u == 0) {
-            prefix[0] = tprefix[0] = 0;
-            if (in_smem) pre_s[0] = tpre_s[0] = 0;
+        int incl[3];
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+            incl[q] = v[q] + (w > 0 ? warp_tot[q][w - 1] : 0) + carry[q];
+            if (u < U) out[q][u + 1] = incl[q];
+            if (u == 0) out[q][0] = 0;
         }
         __syncthreads();
-        if (threadIdx.x == 1023) {
-            carry[0] = ip;
-            carry[1] = it;
-        }
+        if (threadIdx.x == 1023)
+            for (int q = 0; q < 3; ++q) carry[q] = incl[q];
         __syncthreads();
     }
-    const int* pf = in_smem ? pre_s : prefix;
-    const int* tf = in_smem ? tpre_s : tprefix;
     const int T = carry[0], Tt = carry[1];
     __shared__ int cuts[kClusters + 1], cut_tmp[kClusters + 1];
-    compute_cuts(cuts, cut_tmp, pf, tf, U, T, Tt, max_splits);
+    compute_cuts(cuts, cut_tmp, prefix, tprefix, wprefix, U, T, Tt, max_splits);
     for (int u = threadIdx.x; u < U; u += 1024) {
-        const int4 m = unit_meta_of(u, pf, cuts, seq_lens, n_hb, T_q, max_blocks);
+        const int4 m = unit_meta_of(u, prefix, cuts, seq_lens, n_hb, T_q, max_blocks);
         unit_meta[u] = m;
         if (m.x == 0 && (u % (n_hb * T_q)) == 0) raise_status(status, MLA_STATUS_BAD_SEQ_LEN);
     }
     for (int c = threadIdx.x; c < kClusters; c += 1024) {
         const int a = cuts[c], e = cuts[c + 1];
-        cluster_info[c] = a < e ? make_int4(a, e, unit_of_page(pf, U, a), unit_of_page(pf, U, e - 1))
+        cluster_info[c] = a < e ? make_int4(a, e, unit_of_page(prefix, U, a), unit_of_page(prefix, U, e - 1))
                                 : make_int4(0, 0, 0, 0);
     }
 }
@@ -1236,14 +1231,15 @@ bool make_map_chunks(CUtensorMap* m, const void* base, uint64_t rows) {
 size_t r256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct Sm100Ws {
-    size_t prefix, tprefix, kv, kv_cta, meta, cinfo, part_lse, part_o, total;
+    size_t prefix, tprefix, wprefix, kv, kv_cta, meta, cinfo, part_lse, part_o, total;
 };
 
 Sm100Ws sm100_ws(int U) {
     Sm100Ws w;
     w.prefix = 0;
     w.tprefix = w.prefix + r256(static_cast<size_t>(U + 1) * 4);
-    w.kv = w.tprefix + r256(static_cast<size_t>(U + 1) * 4);
+    w.wprefix = w.tprefix + r256(static_cast<size_t>(U + 1) * 4);
+    w.kv = w.wprefix + r256(static_cast<size_t>(U + 1) * 4);
     w.kv_cta = w.kv + r256(static_cast<size_t>(U) * 4);
     w.meta = w.kv_cta + r256(static_cast<size_t>(2 * kClusters) * U * 4);
     w.cinfo = w.meta + r256(static_cast<size_t>(U) * 16);
@@ -1321,6 +1317,7 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int max_splits,
     if (!k.in_kernel_schedule) {
         e = launch_pdl(mla_sm100_schedule_kernel, dim3(1), dim3(1024), 0, stream, P.seq_lens, P.T_q, n_hb,
                        P.max_blocks, max_splits, U, k.prefix, reinterpret_cast<int32_t*>(base + w.tprefix),
+                       reinterpret_cast<int32_t*>(base + w.wprefix),
                        k.unit_kv, k.unit_meta,
                        reinterpret_cast<int4*>(base + w.cinfo), P.status);
         if (e != cudaSuccess) return e;
