@@ -109,14 +109,35 @@ int mla_check_device(void);
  * floats. */
 int mla_rope_table(int d_r, double base, int max_pos, float* host_table);
 
+/* YaRN RoPE table on the HOST, same layout as mla_rope_table, for a context
+ * stretched s times past the training length orig_len ("Техотчёт DeepSeek-V2
+ * (2024)", long context; "DeepSeek-V2 review", 4: YaRN on the decoupled
+ * k^R, 4K -> 128K with s = 40, alpha = 1, beta = 32).  Pair m with frequency
+ * f_m = base^(-2m/d_r) turns r_m = orig_len f_m / (2 pi) times over the
+ * training length; with g_m = clamp((r_m - alpha) / (beta - alpha), 0, 1) it
+ * rotates at f_m ((1 - g_m) / s + g_m): pairs turning fewer than alpha times
+ * are interpolated by s, pairs turning more than beta times are kept.
+ * Evaluated in double, rounded to float.  s >= 1, beta > alpha. */
+int mla_rope_table_yarn(int d_r, double base, int max_pos, double s, double alpha, double beta,
+                        int orig_len, float* host_table);
+
+/* Score scale with the YaRN attention temperature: t / sqrt(d_h + d_r) with
+ * sqrt(t) = coeff ln s + 1 (DeepSeek-V2 uses coeff = 0.0707; 0.1 in the
+ * generic rule), i.e. both q and k multiplied by sqrt(t).  Pass it as
+ * mla_config_t.scale.  Returns 0 for invalid arguments. */
+float mla_yarn_score_scale(int d_h, int d_r, double s, double coeff);
+
 /* q_abs[n, i, :] = W^UK_i^T q_c[n, i, :]  ([notes] "Key에 대한 수식 전개";
  * [ru] "Идея 1").
  *   q_c   (n_tok, n_h, d_h)  bf16
  *   w_uk  (n_h, d_h, d_c)    bf16; W^UK_i = w_uk[i] maps a latent to head i's key
  *   q_abs (n_tok, n_h, d_c)  bf16 out (float accumulation, RNE rounding)
+ *   dev_status one int32 on the device (may be NULL): the tensor-core kernel
+ *              ORs MLA_STATUS_TIMEOUT in when one of its bounded waits runs
+ *              out; q_abs is then incomplete.
  * n_tok = B * T_q, token n = b * T_q + t.  1 <= n_tok <= 65536. */
 int mla_absorb_q(const mla_config_t* cfg, const mla_bf16* q_c, const mla_bf16* w_uk,
-                 mla_bf16* q_abs, int n_tok, void* stream);
+                 mla_bf16* q_abs, int n_tok, int32_t* dev_status, void* stream);
 
 /* Decoupled RoPE and paged append ([review] 2.3; [ru] "Идея 2"; [notes]
  * "Decoupled Rotary Position Embedding", "MLA 코드 구현" forward).
@@ -186,9 +207,10 @@ int mla_decode_launches(const mla_config_t* cfg, int B, int T_q, int max_splits)
 /* Diagnostic: after an mla_decode call with these arguments has completed on
  * `stream`, copies to host_counts the number of parts (key-range splits) of
  * each unit of work, read back from the workspace; synchronises `stream`.
- * tcgen05 kernels: one count per (query row, block of 128 heads), unit
- * u = (b * T_q + t) * (n_h / 128) + head block, n_counts = B * T_q * n_h / 128
- * (0 for a row whose sequence length was invalid).  Portable kernels: the
+ * tcgen05 kernels: one count per (query row, block of 128 heads), in the
+ * kernels' token-major order u = (t * B + b) * (n_h / 128) + head block,
+ * n_counts = B * T_q * n_h / 128 (0 for a row whose sequence length was
+ * invalid).  Portable kernels: the
  * fixed split count, written to all n_counts entries. */
 int mla_decode_split_counts(const mla_config_t* cfg, int B, int T_q, int max_splits,
                             const void* workspace, int32_t* host_counts, int n_counts,
@@ -237,9 +259,10 @@ int mla_decode_noalloc(const mla_config_t* cfg, const mla_bf16* q_abs, const mla
 
 /* o[n, i, :] = W^UV_i latent[n, i, :]  ([notes] "Value에 대한 수식 전개").
  *   latent (n_tok, n_h, d_c) bf16;  w_uv (n_h, d_h, d_c) bf16
- *   out    (n_tok, n_h, d_h) bf16 (float accumulation, RNE rounding) */
+ *   out    (n_tok, n_h, d_h) bf16 (float accumulation, RNE rounding)
+ *   dev_status as for mla_absorb_q. */
 int mla_up_v(const mla_config_t* cfg, const mla_bf16* latent, const mla_bf16* w_uv,
-             mla_bf16* out, int n_tok, void* stream);
+             mla_bf16* out, int n_tok, int32_t* dev_status, void* stream);
 
 /* Zero a device status word (async on stream). */
 int mla_clear_status(int32_t* dev_status, void* stream);

@@ -25,12 +25,14 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 EXPORTED = (
-    "mla_status_str", "mla_check_device", "mla_rope_table", "mla_absorb_q",
+    "mla_status_str", "mla_check_device", "mla_rope_table", "mla_rope_table_yarn",
+    "mla_yarn_score_scale", "mla_absorb_q",
     "mla_rope_append", "mla_decode_workspace_bytes", "mla_decode", "mla_decode_launches",
     "mla_decode_noalloc", "mla_decode_split_counts", "mla_test_arm_decode_timeout", "mla_up_v",
     "mla_clear_status", "mla_read_status",
 )
 
+MLA_ERR_SIZE = -3
 MLA_STATUS_BAD_POSITION = 1
 MLA_STATUS_BAD_BLOCK = 2
 MLA_STATUS_BAD_SEQ_LEN = 4
@@ -67,7 +69,11 @@ _lib.mla_status_str.restype = ctypes.c_char_p
 _lib.mla_status_str.argtypes = [_i]
 _lib.mla_check_device.argtypes = []
 _lib.mla_rope_table.argtypes = [_i, ctypes.c_double, _i, _vp]
-_lib.mla_absorb_q.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp]
+_lib.mla_rope_table_yarn.argtypes = [_i, ctypes.c_double, _i, ctypes.c_double, ctypes.c_double, ctypes.c_double,
+                                     _i, _vp]
+_lib.mla_yarn_score_scale.restype = ctypes.c_float
+_lib.mla_yarn_score_scale.argtypes = [_i, _i, ctypes.c_double, ctypes.c_double]
+_lib.mla_absorb_q.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp, _vp]
 _lib.mla_rope_append.argtypes = [_cfgp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, _vp, _vp]
 _lib.mla_decode_workspace_bytes.restype = _sz
 _lib.mla_decode_workspace_bytes.argtypes = [_cfgp, _i, _i, _i]
@@ -77,7 +83,7 @@ _lib.mla_decode_noalloc.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, 
                                     _vp]
 _lib.mla_decode_split_counts.argtypes = [_cfgp, _i, _i, _i, _vp, _vp, _i, _vp]
 _lib.mla_test_arm_decode_timeout.argtypes = [ctypes.c_uint64]
-_lib.mla_up_v.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp]
+_lib.mla_up_v.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp, _vp]
 _lib.mla_clear_status.argtypes = [_vp, _vp]
 _lib.mla_read_status.argtypes = [_vp, _vp, _vp]
 
@@ -118,9 +124,25 @@ def mla_rope_table(d_r: int, base: float, max_pos: int) -> torch.Tensor:
     return out
 
 
-def mla_absorb_q(cfg: MlaConfig, q_c, w_uk, q_abs, n_tok: int, stream=None):
+def mla_rope_table_yarn(d_r: int, base: float, max_pos: int, s: float = 40.0, alpha: float = 1.0,
+                        beta: float = 32.0, orig_len: int = 4096) -> torch.Tensor:
+    """Host float32 YaRN table (max_pos, d_r) built by the library (cos | sin)."""
+    out = torch.empty((max_pos, d_r), dtype=torch.float32)
+    _check("mla_rope_table_yarn", _lib.mla_rope_table_yarn(d_r, float(base), max_pos, float(s), float(alpha),
+                                                           float(beta), int(orig_len), out.data_ptr()))
+    return out
+
+
+def mla_yarn_score_scale(d_h: int, d_r: int, s: float = 40.0, coeff: float = 0.0707) -> float:
+    v = float(_lib.mla_yarn_score_scale(int(d_h), int(d_r), float(s), float(coeff)))
+    if v <= 0.0:
+        raise MlaError("mla_yarn_score_scale", MLA_ERR_SIZE)
+    return v
+
+
+def mla_absorb_q(cfg: MlaConfig, q_c, w_uk, q_abs, n_tok: int, dev_status=None, stream=None):
     _check("mla_absorb_q", _lib.mla_absorb_q(ctypes.byref(cfg), _ptr(q_c), _ptr(w_uk), _ptr(q_abs),
-                                             int(n_tok), _stream(stream)))
+                                             int(n_tok), _ptr(dev_status), _stream(stream)))
 
 
 def mla_rope_append(cfg: MlaConfig, q_r, k_r, c_kv, positions, rope_table, max_pos: int,
@@ -179,9 +201,9 @@ def mla_test_arm_decode_timeout(wait_limit_ns: int):
     _check("mla_test_arm_decode_timeout", _lib.mla_test_arm_decode_timeout(int(wait_limit_ns)))
 
 
-def mla_up_v(cfg: MlaConfig, latent, w_uv, out, n_tok: int, stream=None):
+def mla_up_v(cfg: MlaConfig, latent, w_uv, out, n_tok: int, dev_status=None, stream=None):
     _check("mla_up_v", _lib.mla_up_v(ctypes.byref(cfg), _ptr(latent), _ptr(w_uv), _ptr(out),
-                                     int(n_tok), _stream(stream)))
+                                     int(n_tok), _ptr(dev_status), _stream(stream)))
 
 
 def mla_clear_status(dev_status, stream=None):

@@ -131,19 +131,49 @@ int mla_rope_table(int d_r, double base, int max_pos, float* host_table) {
     return MLA_OK;
 }
 
+int mla_rope_table_yarn(int d_r, double base, int max_pos, double s, double alpha, double beta, int orig_len,
+                        float* host_table) {
+    if (host_table == nullptr) return MLA_ERR_NULL;
+    if (d_r < 2 || d_r % 2 || max_pos < 1 || !(base > 0.0)) return MLA_ERR_SIZE;
+    if (!(s >= 1.0) || !(beta > alpha) || orig_len < 1) return MLA_ERR_SIZE;
+    const int h = d_r / 2;
+    const double two_pi = 6.283185307179586476925286766559;
+    for (int m = 0; m < h; ++m) {
+        const double f = pow(base, -2.0 * m / d_r);
+        const double turns = orig_len * f / two_pi;   // turns of pair m over the training length
+        double g = (turns - alpha) / (beta - alpha);
+        g = g < 0.0 ? 0.0 : (g > 1.0 ? 1.0 : g);
+        const double fy = f * ((1.0 - g) / s + g);
+        for (int p = 0; p < max_pos; ++p) {
+            const double th = static_cast<double>(p) * fy;
+            host_table[static_cast<size_t>(p) * d_r + m] = static_cast<float>(cos(th));
+            host_table[static_cast<size_t>(p) * d_r + h + m] = static_cast<float>(sin(th));
+        }
+    }
+    return MLA_OK;
+}
+
+float mla_yarn_score_scale(int d_h, int d_r, double s, double coeff) {
+    if (d_h < 1 || d_r < 0 || !(s >= 1.0) || !(coeff >= 0.0)) return 0.f;
+    const double sqrt_t = coeff * log(s) + 1.0;
+    return static_cast<float>(sqrt_t * sqrt_t / sqrt(static_cast<double>(d_h + d_r)));
+}
+
 int mla_absorb_q(const mla_config_t* cfg, const mla_bf16* q_c, const mla_bf16* w_uk,
-                 mla_bf16* q_abs, int n_tok, void* stream) {
+                 mla_bf16* q_abs, int n_tok, int32_t* dev_status, void* stream) {
     int rc = check_config(cfg);
     if (rc) return rc;
     if (!q_c || !w_uk || !q_abs) return MLA_ERR_NULL;
     if (!aligned16(q_c) || !aligned16(w_uk) || !aligned16(q_abs)) return MLA_ERR_ALIGN;
+    if (dev_status && !aligned4(dev_status)) return MLA_ERR_ALIGN;
     if (n_tok < 1 || n_tok > 65536) return MLA_ERR_SIZE;
     const bool sm100_shape = mla::sm100_absorb_supports(cfg->d_h, cfg->d_c);
     if (cfg->impl == 2 && !sm100_shape) return MLA_ERR_CONFIG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cfg->impl == 2 || (cfg->impl == 0 && sm100_shape)) {
         if (mla_check_device() != MLA_OK) return MLA_ERR_UNSUPPORTED;
-        return cuda_rc(mla::launch_absorb_q_sm100(q_c, w_uk, q_abs, n_tok, cfg->n_h, cfg->d_h, cfg->d_c, st));
+        return cuda_rc(
+            mla::launch_absorb_q_sm100(q_c, w_uk, q_abs, n_tok, cfg->n_h, cfg->d_h, cfg->d_c, dev_status, st));
     }
     return cuda_rc(mla::launch_absorb_q_simt(q_c, w_uk, q_abs, n_tok, cfg->n_h, cfg->d_h, cfg->d_c, st));
 }
@@ -271,18 +301,20 @@ int mla_test_arm_decode_timeout(uint64_t wait_limit_ns) {
 }
 
 int mla_up_v(const mla_config_t* cfg, const mla_bf16* latent, const mla_bf16* w_uv, mla_bf16* out,
-             int n_tok, void* stream) {
+             int n_tok, int32_t* dev_status, void* stream) {
     int rc = check_config(cfg);
     if (rc) return rc;
     if (!latent || !w_uv || !out) return MLA_ERR_NULL;
     if (!aligned16(latent) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_ALIGN;
+    if (dev_status && !aligned4(dev_status)) return MLA_ERR_ALIGN;
     if (n_tok < 1 || n_tok > 65536) return MLA_ERR_SIZE;
     const bool sm100_shape = mla::sm100_up_v_supports(cfg->d_h, cfg->d_c);
     if (cfg->impl == 2 && !sm100_shape) return MLA_ERR_CONFIG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cfg->impl == 2 || (cfg->impl == 0 && sm100_shape)) {
         if (mla_check_device() != MLA_OK) return MLA_ERR_UNSUPPORTED;
-        return cuda_rc(mla::launch_up_v_sm100(latent, w_uv, out, n_tok, cfg->n_h, cfg->d_h, cfg->d_c, st));
+        return cuda_rc(
+            mla::launch_up_v_sm100(latent, w_uv, out, n_tok, cfg->n_h, cfg->d_h, cfg->d_c, dev_status, st));
     }
     return cuda_rc(mla::launch_up_v_simt(latent, w_uv, out, n_tok, cfg->n_h, cfg->d_h, cfg->d_c, st));
 }

@@ -173,19 +173,32 @@ __device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, volatil
 }
 
 // ---------------------------------------------------------------------------
-// Work schedule.  Unit u = (b T_q + t) n_hb + hb covers the keys 0 .. kv - 1
-// of query row (b, t), kv = L_b - T_q + t + 1, i.e. ceil(kv / 64) pages; a
-// sequence whose length is out of range has no pages (its outputs are
-// defined as zero / -inf by the merge kernel).  pf is the exclusive prefix of
-// the page counts, T = pf[U] the total.
+// Work schedule.  Units are numbered token-major: u = (t B + b) n_hb + hb
+// for query token t of sequence b and head block hb, so that the T_q units
+// of one sequence lie a quarter (for T_q = 4) of the work apart and run on
+// different clusters at the same time, at the same relative position in the
+// cache: their page reads meet in L2 instead of streaming the cache from
+// HBM T_q times.  Unit u covers the keys 0 .. kv - 1 of query row (b, t),
+// kv = L_b - T_q + t + 1, i.e. ceil(kv / 64) pages; a sequence whose length
+// is out of range has no pages (its outputs are defined as zero / -inf by
+// the merge kernel).  pf is the exclusive prefix of the page counts, T =
+// pf[U] the total.
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ int unit_keys(const int32_t* seq_lens, int u, int n_hb, int T_q, int max_blocks) {
-    const int bt = u / n_hb;
-    const int b = bt / T_q;
-    const int t = bt - b * T_q;
-    const int L = seq_lens[b];   // global or shared memory
-    return (L >= T_q && L <= max_blocks * kPage) ? L - T_q + t + 1 : 0;
+struct UnitIdx {
+    int b, t, hb;
+};
+
+__device__ __forceinline__ UnitIdx unit_index(int u, int n_hb, int B) {
+    const int r = u / n_hb;
+    const int t = r / B;
+    return UnitIdx{r - t * B, t, u - r * n_hb};
+}
+
+__device__ __forceinline__ int unit_keys(const int32_t* seq_lens, int u, int n_hb, int B, int T_q, int max_blocks) {
+    const UnitIdx x = unit_index(u, n_hb, B);
+    const int L = seq_lens[x.b];   // global or shared memory
+    return (L >= T_q && L <= max_blocks * kPage) ? L - T_q + x.t + 1 : 0;
 }
 
 // Last unit v with pf[v] <= g (for g < T: the unit holding page g).
@@ -285,10 +298,10 @@ __device__ int cluster_of_page(int g, const int* cuts) {
 }
 
 // Merge metadata of unit u: {kv_len, first cluster, parts, sequence}.
-__device__ int4 unit_meta_of(int u, const int32_t* pf, const int* cuts, const int32_t* seq_lens, int n_hb,
+__device__ int4 unit_meta_of(int u, const int32_t* pf, const int* cuts, const int32_t* seq_lens, int n_hb, int B,
                              int T_q, int max_blocks) {
-    const int kv = unit_keys(seq_lens, u, n_hb, T_q, max_blocks);
-    const int b = u / n_hb / T_q;
+    const int kv = unit_keys(seq_lens, u, n_hb, B, T_q, max_blocks);
+    const int b = unit_index(u, n_hb, B).b;
     const int a = pf[u], e = pf[u + 1];
     if (e <= a) return make_int4(0, 0, 0, b);
     const int c0 = cluster_of_page(a, cuts);
@@ -298,7 +311,7 @@ __device__ int4 unit_meta_of(int u, const int32_t* pf, const int* cuts, const in
 
 // One tile of a cluster's work: up to 4 consecutive pages of one unit.
 struct Tile {
-    int u;          // unit = (b T_q + t) n_hb + hb
+    int u;          // unit = (t B + b) n_hb + hb
     int bt;         // query row b T_q + t of the unit
     int hb;         // head block of the unit
     int b;          // sequence of the unit
@@ -318,7 +331,7 @@ struct Tile {
 struct TileWalker {
     const int32_t* kvs;
     int off, g, g0, g1, u, ubeg, uend, kv;
-    int bt, hb, b, t, n_hb, T_q;
+    int bt, hb, b, t, n_hb, B, T_q;
     __device__ void load_unit() {
         kv = kvs[u - off];
         uend = ubeg + (kv + kPage - 1) / kPage;
@@ -329,27 +342,30 @@ struct TileWalker {
         load_unit();
         if (++hb == n_hb) {
             hb = 0;
-            ++bt;
-            if (++t == T_q) {
-                t = 0;
-                ++b;
+            if (++b == B) {
+                b = 0;
+                ++t;
             }
+            bt = b * T_q + t;
         }
     }
-    __device__ void init(const int32_t* kvs_, int off_, int u0, int ubeg0, int g0_, int g1_, int n_hb_, int T_q_) {
+    __device__ void init(const int32_t* kvs_, int off_, int u0, int ubeg0, int g0_, int g1_, int n_hb_, int B_,
+                         int T_q_) {
         kvs = kvs_;
         off = off_;
         g = g0_;
         g0 = g0_;
         g1 = g1_;
         n_hb = n_hb_;
+        B = B_;
         T_q = T_q_;
         u = u0;
         ubeg = ubeg0;
-        bt = u0 / n_hb;
-        hb = u0 - bt * n_hb;
-        b = bt / T_q;
-        t = bt - b * T_q;
+        const UnitIdx x = unit_index(u0, n_hb, B);
+        b = x.b;
+        t = x.t;
+        hb = x.hb;
+        bt = b * T_q + t;
         if (g < g1) {
             load_unit();
             while (g < g1 && uend <= g) step_unit();
@@ -380,13 +396,13 @@ struct TileWalker {
 // costs into pf, tf, wf[0 .. U] (U <= kInKernelUnits); every thread of the
 // CTA takes part; warp_tot holds 3 x 16 ints of scratch.  Returns {T, Tt}.
 __device__ int2 schedule_scan(int* pf, int* tf, int* wf, int* warp_tot, const int32_t* seq_lens, int U, int n_hb,
-                              int T_q, int max_blocks) {
+                              int B, int T_q, int max_blocks) {
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int per = (U + kThreads - 1) / kThreads;
     const int beg = min(U, tid * per), end = min(U, beg + per);
     int loc[3] = {0, 0, 0};
     for (int u = beg; u < end; ++u) {
-        const int pages = (unit_keys(seq_lens, u, n_hb, T_q, max_blocks) + kPage - 1) / kPage;
+        const int pages = (unit_keys(seq_lens, u, n_hb, B, T_q, max_blocks) + kPage - 1) / kPage;
         const int tiles = (pages + kTilePages - 1) / kTilePages;
         pf[u + 1] = pages;
         tf[u + 1] = tiles;
@@ -529,7 +545,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         int* wtot = lens + kInKernelUnits;                            // scan scratch, 48
         for (int b = threadIdx.x; b < p.B; b += kThreads) lens[b] = __ldg(p.seq_lens + b);
         __syncthreads();
-        const int2 TT = schedule_scan(sc, tfx, wfx, wtot, lens, p.U, p.n_hb, p.T_q, p.max_blocks);
+        const int2 TT = schedule_scan(sc, tfx, wfx, wtot, lens, p.U, p.n_hb, p.B, p.T_q, p.max_blocks);
         const int T = TT.x;
         int* cuts = reinterpret_cast<int*>(smem + kOffCuts);
         compute_cuts(cuts, ctmp, sc, tfx, wfx, p.U, T, TT.y, p.max_splits);
@@ -545,14 +561,14 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 kv_base = dst;
             }
             for (int k = threadIdx.x; k <= u1 - u0; k += kThreads)
-                dst[k] = unit_keys(lens, u0 + k, p.n_hb, p.T_q, p.max_blocks);
+                dst[k] = unit_keys(lens, u0 + k, p.n_hb, p.B, p.T_q, p.max_blocks);
         }
         kv_off = u0;
         // merge metadata and length checks, spread over the grid's threads
         for (int u = blockIdx.x * kThreads + threadIdx.x; u < p.U; u += gridDim.x * kThreads) {
-            const int4 m = unit_meta_of(u, sc, cuts, lens, p.n_hb, p.T_q, p.max_blocks);
+            const int4 m = unit_meta_of(u, sc, cuts, lens, p.n_hb, p.B, p.T_q, p.max_blocks);
             p.unit_meta[u] = m;
-            if (m.x == 0 && (u % (p.n_hb * p.T_q)) == 0) raise_status(p.status, MLA_STATUS_BAD_SEQ_LEN);
+            if (m.x == 0 && u < p.B * p.n_hb && u % p.n_hb == 0) raise_status(p.status, MLA_STATUS_BAD_SEQ_LEN);
         }
     } else {
         const int4 cinfo = p.cluster_info[cluster];
@@ -588,7 +604,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
         }
         return blk * kPage;
     };
-    auto walker = [&](TileWalker& w) { w.init(kv_base, kv_off, u0, ubeg0, g0, g1, p.n_hb, p.T_q); };
+    auto walker = [&](TileWalker& w) { w.init(kv_base, kv_off, u0, ubeg0, g0, g1, p.n_hb, p.B, p.T_q); };
 
     if (warp < 4) {
         // Warpgroup 0 (loads and MMA issue) needs few registers: it gives them to
@@ -1063,7 +1079,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
 // threads with the same cut rule as the decode kernel's own scan.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024)
-mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int T_q, int n_hb, int max_blocks,
+mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, int n_hb, int max_blocks,
                           int max_splits, int U, int32_t* __restrict__ prefix, int32_t* __restrict__ tprefix,
                           int32_t* __restrict__ wprefix, int32_t* __restrict__ kv_out, int4* __restrict__ unit_meta,
                           int4* __restrict__ cluster_info, int32_t* status) {
@@ -1078,7 +1094,7 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int T_q, int n_h
         const int u = base + threadIdx.x;
         int v[3] = {0, 0, 0};   // pages, tiles, cost
         if (u < U) {
-            const int kv = unit_keys(seq_lens, u, n_hb, T_q, max_blocks);
+            const int kv = unit_keys(seq_lens, u, n_hb, B, T_q, max_blocks);
             kv_out[u] = kv;
             v[0] = (kv + kPage - 1) / kPage;
             v[1] = (v[0] + kTilePages - 1) / kTilePages;
@@ -1124,9 +1140,9 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int T_q, int n_h
     __shared__ int cuts[kClusters + 1], cut_tmp[kClusters + 1];
     compute_cuts(cuts, cut_tmp, prefix, tprefix, wprefix, U, T, Tt, max_splits);
     for (int u = threadIdx.x; u < U; u += 1024) {
-        const int4 m = unit_meta_of(u, prefix, cuts, seq_lens, n_hb, T_q, max_blocks);
+        const int4 m = unit_meta_of(u, prefix, cuts, seq_lens, n_hb, B, T_q, max_blocks);
         unit_meta[u] = m;
-        if (m.x == 0 && (u % (n_hb * T_q)) == 0) raise_status(status, MLA_STATUS_BAD_SEQ_LEN);
+        if (m.x == 0 && u < B * n_hb && u % n_hb == 0) raise_status(status, MLA_STATUS_BAD_SEQ_LEN);
     }
     for (int c = threadIdx.x; c < kClusters; c += 1024) {
         const int a = cuts[c], e = cuts[c + 1];
@@ -1142,7 +1158,7 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int T_q, int n_h
 __global__ void __launch_bounds__(256)
 mla_sm100_merge_kernel(const int4* __restrict__ unit_meta, const float* __restrict__ part_o,
                        const float* __restrict__ part_lse, uint16_t* __restrict__ out_latent,
-                       float* __restrict__ out_lse, int n_h, int n_hb, int U) {
+                       float* __restrict__ out_lse, int n_h, int n_hb, int B, int T_q, int U) {
     griddep_launch_dependents();
     griddep_wait();
     const int lane = threadIdx.x & 31;
@@ -1150,7 +1166,8 @@ mla_sm100_merge_kernel(const int4* __restrict__ unit_meta, const float* __restri
     const int u = wg >> 7, row = wg & 127;
     if (u >= U) return;
     const int4 meta = unit_meta[u];
-    const int bt = u / n_hb, hb = u - bt * n_hb;
+    const UnitIdx x = unit_index(u, n_hb, B);
+    const int bt = x.b * T_q + x.t, hb = x.hb;
     const size_t grow = static_cast<size_t>(bt) * n_h + hb * 128 + row;
     uint4* dst = reinterpret_cast<uint4*>(out_latent + grow * kDc + lane * 16);
     if (meta.x == 0) {
@@ -1217,15 +1234,11 @@ mla_sm100_merge_kernel(const int4* __restrict__ unit_meta, const float* __restri
 // The pool viewed as [chunk (9)][row][64 columns]: one box loads four 64-column
 // chunks of the same 64 rows into consecutive 8 KB blocks.
 bool make_map_chunks(CUtensorMap* m, const void* base, uint64_t rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (fn == nullptr) return false;
     const cuuint64_t dims[3] = {64, rows, kChunks};
     const cuuint64_t strides[2] = {kRow * 2, 128};
     const cuuint32_t box[3] = {64, 64, 4};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_tiled_cached(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 size_t r256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -1315,7 +1328,7 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int max_splits,
 
     cudaError_t e;
     if (!k.in_kernel_schedule) {
-        e = launch_pdl(mla_sm100_schedule_kernel, dim3(1), dim3(1024), 0, stream, P.seq_lens, P.T_q, n_hb,
+        e = launch_pdl(mla_sm100_schedule_kernel, dim3(1), dim3(1024), 0, stream, P.seq_lens, P.B, P.T_q, n_hb,
                        P.max_blocks, max_splits, U, k.prefix, reinterpret_cast<int32_t*>(base + w.tprefix),
                        reinterpret_cast<int32_t*>(base + w.wprefix),
                        k.unit_kv, k.unit_meta,
@@ -1330,7 +1343,7 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int max_splits,
     const int rows = U * 128;
     return launch_pdl(mla_sm100_merge_kernel, dim3((rows + 7) / 8), dim3(256), 0, stream,
                       static_cast<const int4*>(k.unit_meta), static_cast<const float*>(k.part_o),
-                      static_cast<const float*>(k.part_lse), P.out_latent, P.out_lse, P.n_h, n_hb, U);
+                      static_cast<const float*>(k.part_lse), P.out_latent, P.out_lse, P.n_h, n_hb, P.B, P.T_q, U);
 }
 
 }  // namespace mla

@@ -43,6 +43,7 @@ struct ProjParams {
     CUtensorMap tm_a;   // weights, [n_h * d_h][d_c], 64-column boxes
     CUtensorMap tm_b;   // activations, [n_tok][n_h * K], boxes of 64 x nt
     uint16_t* out;      // [n_tok][n_h][m_total]
+    int32_t* status;    // device status word (may be null): MLA_STATUS_TIMEOUT
     int n_tok, n_h, d_h, d_c;
     int K;              // contracted length: d_h (absorb_q) or d_c (up_v)
     int m_total;        // output features per head: d_c (absorb_q) or d_h (up_v)
@@ -144,6 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_proj_sm100_kernel(const __gri
                 ptx::mma1_commit(barD);
                 ok = wait_bounded(barD, t & 1);
             }
+            if (!ok) raise_status(p.status, MLA_STATUS_TIMEOUT);
             s_ok = ok;
         }
         __syncthreads();
@@ -209,8 +211,9 @@ bool sm100_absorb_supports(int d_h, int d_c) { return d_h % 64 == 0 && d_h <= 25
 bool sm100_up_v_supports(int d_h, int d_c) { return d_h % kM == 0 && d_c % 64 == 0 && d_c <= 512; }
 
 cudaError_t launch_absorb_q_sm100(const uint16_t* q_c, const uint16_t* w_uk, uint16_t* q_abs, int n_tok, int n_h,
-                                  int d_h, int d_c, cudaStream_t stream) {
+                                  int d_h, int d_c, int32_t* status, cudaStream_t stream) {
     ProjParams p;
+    p.status = status;
     p.n_tok = n_tok;
     p.n_h = n_h;
     p.d_h = d_h;
@@ -227,8 +230,9 @@ cudaError_t launch_absorb_q_sm100(const uint16_t* q_c, const uint16_t* w_uk, uin
 }
 
 cudaError_t launch_up_v_sm100(const uint16_t* latent, const uint16_t* w_uv, uint16_t* out, int n_tok, int n_h,
-                              int d_h, int d_c, cudaStream_t stream) {
+                              int d_h, int d_c, int32_t* status, cudaStream_t stream) {
     ProjParams p;
+    p.status = status;
     p.n_tok = n_tok;
     p.n_h = n_h;
     p.d_h = d_h;

@@ -27,16 +27,30 @@ class DeviceCase:
     """Buffers and the step of one workload on one GPU."""
 
     def __init__(self, spec: CaseSpec, impl: int = M.IMPL_AUTO, max_splits: int = 0,
-                 device: str = "cuda:0", rope_base: float = 10000.0, fill_history: bool = True):
+                 device: str = "cuda:0", rope_base: float = 10000.0, fill_history: bool = True,
+                 yarn=None):
+        """yarn: None (plain RoPE, scale 1/sqrt(d_h + d_r)) or a dict of
+        mla_rope_table_yarn / mla_yarn_score_scale arguments (s, alpha, beta,
+        orig_len, coeff); the library builds the table and the scale."""
         self.spec = spec
         self.dev = torch.device(device)
         self.impl = impl
         self.max_splits = max_splits
         s = spec
-        self.cfg = M.MlaConfig(s.n_h, s.d_c, s.d_h, s.d_r, s.block_size, 0.0, impl)
+        self.yarn = dict(yarn) if yarn is not None else None
+        scale = 0.0
+        if self.yarn is not None:
+            scale = M.mla_yarn_score_scale(s.d_h, s.d_r, self.yarn.get("s", 40.0), self.yarn.get("coeff", 0.0707))
+        self.cfg = M.MlaConfig(s.n_h, s.d_c, s.d_h, s.d_r, s.block_size, scale, impl)
         dev = self.dev
         self.max_pos = int(np.max(s.seq_lens))
-        self.rope_table = M.mla_rope_table(s.d_r, rope_base, self.max_pos).to(dev)
+        if self.yarn is None:
+            self.rope_table = M.mla_rope_table(s.d_r, rope_base, self.max_pos).to(dev)
+        else:
+            y = self.yarn
+            self.rope_table = M.mla_rope_table_yarn(s.d_r, rope_base, self.max_pos, y.get("s", 40.0),
+                                                    y.get("alpha", 1.0), y.get("beta", 32.0),
+                                                    y.get("orig_len", 4096)).to(dev)
         self.block_table_np = s.block_table()
         self.block_table = torch.from_numpy(self.block_table_np).to(dev)
         self.seq_lens = torch.from_numpy(s.seq_lens.astype(np.int32)).to(dev)
@@ -103,14 +117,14 @@ class DeviceCase:
     def step(self, stream=None):
         """One pass of the whole hot path for the batch."""
         s = self.spec
-        M.mla_absorb_q(self.cfg, self.q_c, self.w_uk, self.q_abs, s.n_tok, stream)
+        M.mla_absorb_q(self.cfg, self.q_c, self.w_uk, self.q_abs, s.n_tok, self.status, stream)
         M.mla_rope_append(self.cfg, self.q_r, self.k_r_new, self.c_kv_new, self.positions,
                           self.rope_table, self.max_pos, self.block_table, s.max_blocks, self.pool,
                           s.num_blocks, s.B, s.T_q, self.status, stream)
         M.mla_decode(self.cfg, self.q_abs, self.q_r, self.pool, s.num_blocks, self.block_table,
                      s.max_blocks, self.seq_lens, s.B, s.T_q, self.max_splits, self.ws,
                      self.ws_bytes, self.latent, self.lse, stream)
-        M.mla_up_v(self.cfg, self.latent, self.w_uv, self.out, s.n_tok, stream)
+        M.mla_up_v(self.cfg, self.latent, self.w_uv, self.out, s.n_tok, self.status, stream)
 
     def decode_only(self, stream=None):
         s = self.spec

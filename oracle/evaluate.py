@@ -29,8 +29,11 @@ def _key(spec):
             tuple(int(x) for x in spec.seq_lens))
 
 
-def reference(spec, b: int, heads=None, want_p=False):
-    """Oracle outputs for sequence b: dict(o, latent, lse[, p]) over `heads`."""
+def reference(spec, b: int, heads=None, want_p=False, inv_freq=None, scale=None):
+    """Oracle outputs for sequence b: dict(o, latent, lse[, p]) over `heads`.
+
+    inv_freq / scale: RoPE frequencies and score scale other than the
+    defaults (YaRN: mla_oracle.yarn_inv_freq, mla_oracle.yarn_score_scale)."""
     L = int(spec.seq_lens[b])
     T_q = spec.T_q
     c = O.bf16_to_f64(spec.c_kv_rows(b, 0, L))
@@ -38,4 +41,5 @@ def reference(spec, b: int, heads=None, want_p=False):
     w_uk, w_uv = _cached("w", spec)
     q_c, q_r = _cached("q", spec)
     sl = slice(b * T_q, (b + 1) * T_q)
-    return O.mla_decode_reference(c, k, q_c[sl], q_r[sl], w_uk, w_uv, heads=heads, want_p=want_p)
+    return O.mla_decode_reference(c, k, q_c[sl], q_r[sl], w_uk, w_uv, scale=scale, inv_freq=inv_freq, heads=heads,
+                                  want_p=want_p)

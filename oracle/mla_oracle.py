@@ -79,7 +79,42 @@ def rope_inv_freq(d_r: int, base: float = 10000.0) -> np.ndarray:
     return base ** (-(2.0 * m) / d_r)
 
 
-def rope_rotate(x: np.ndarray, pos, base: float = 10000.0) -> np.ndarray:
+def yarn_inv_freq(d_r: int, base: float = 10000.0, s: float = 40.0, alpha: float = 1.0, beta: float = 32.0,
+                  orig_len: int = 4096) -> np.ndarray:
+    """YaRN frequencies (NTK-by-parts) of the decoupled RoPE.
+
+    "Техотчёт DeepSeek-V2 (2024)", "Обучение: данные, гиперпараметры,
+    инфраструктура" (long context) and "DeepSeek-V2 review", 4 (Long context):
+    the context grows from 4K to 128K by YaRN on k^R only; each frequency pair
+    is scaled by how many turns it makes over the training length, with
+    s = 40, alpha = 1, beta = 32 (target length s x 4K = 160K).  Reading taken
+    here (the page states the rule in words): pair m with frequency
+    f_m = base^(-2m/d_r) makes r_m = orig_len f_m / (2 pi) turns over the
+    training length; gamma_m = clamp((r_m - alpha) / (beta - alpha), 0, 1);
+    the new frequency is f_m ((1 - gamma_m) / s + gamma_m): pairs that turn
+    fewer than alpha times are interpolated by s, pairs that turn more than
+    beta times are kept, the ramp in between is linear in r_m.
+    """
+    f = rope_inv_freq(d_r, base)
+    turns = orig_len * f / (2.0 * math.pi)
+    gamma = np.clip((turns - alpha) / (beta - alpha), 0.0, 1.0)
+    return f * ((1.0 - gamma) / s + gamma)
+
+
+def yarn_sqrt_temperature(s: float = 40.0, coeff: float = 0.0707) -> float:
+    """sqrt(t) = coeff ln s + 1: the attention temperature of YaRN (0.1 in the
+    generic rule; DeepSeek-V2 tuned it to 0.0707, "Техотчёт DeepSeek-V2",
+    long context).  Reading taken here: both q and k are multiplied by
+    sqrt(t), so every score is multiplied by t."""
+    return coeff * math.log(s) + 1.0
+
+
+def yarn_score_scale(d_h: int, d_r: int, s: float = 40.0, coeff: float = 0.0707) -> float:
+    """t / sqrt(d_h + d_h^R): the score scale with the YaRN temperature."""
+    return yarn_sqrt_temperature(s, coeff) ** 2 / math.sqrt(d_h + d_r)
+
+
+def rope_rotate(x: np.ndarray, pos, base: float = 10000.0, inv_freq=None) -> np.ndarray:
     """Apply RoPE to the last axis of ``x`` at positions ``pos`` (fp64).
 
     Half-split pairing: element m rotates with element m + d_r/2 by angle
@@ -91,15 +126,17 @@ def rope_rotate(x: np.ndarray, pos, base: float = 10000.0) -> np.ndarray:
     x = np.asarray(x, dtype=np.float64)
     d_r = x.shape[-1]
     h = d_r // 2
-    theta = np.asarray(pos, dtype=np.float64)[..., None] * rope_inv_freq(d_r, base)
+    f = rope_inv_freq(d_r, base) if inv_freq is None else np.asarray(inv_freq, dtype=np.float64)
+    theta = np.asarray(pos, dtype=np.float64)[..., None] * f
     c, s = np.cos(theta), np.sin(theta)
     x1, x2 = x[..., :h], x[..., h:]
     return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
 
 
-def rope_table_f32(max_pos: int, d_r: int, base: float = 10000.0) -> np.ndarray:
+def rope_table_f32(max_pos: int, d_r: int, base: float = 10000.0, inv_freq=None) -> np.ndarray:
     """float32 table (max_pos, d_r): row p = [cos(p*f_0..), sin(p*f_0..)] from fp64."""
-    theta = np.arange(max_pos, dtype=np.float64)[:, None] * rope_inv_freq(d_r, base)
+    f = rope_inv_freq(d_r, base) if inv_freq is None else np.asarray(inv_freq, dtype=np.float64)
+    theta = np.arange(max_pos, dtype=np.float64)[:, None] * f
     return np.concatenate([np.cos(theta), np.sin(theta)], axis=1).astype(np.float32)
 
 
@@ -248,7 +285,7 @@ def mla_attention_explicit(c_kv, k_r_rot, q_c, q_r_rot, w_uk, w_uv, scale=None,
     return out
 
 
-def mla_decode_reference(c_kv, k_r, q_c, q_r, w_uk, w_uv, base=10000.0, scale=None,
+def mla_decode_reference(c_kv, k_r, q_c, q_r, w_uk, w_uv, base=10000.0, scale=None, inv_freq=None,
                          heads=None, want_p=False):
     """One decode step of one sequence from raw (pre-RoPE) inputs.
 
@@ -259,9 +296,9 @@ def mla_decode_reference(c_kv, k_r, q_c, q_r, w_uk, w_uv, base=10000.0, scale=No
     """
     L = np.asarray(c_kv).shape[0]
     T_q = np.asarray(q_c).shape[0]
-    k_r_rot = rope_rotate(k_r, np.arange(L), base)
+    k_r_rot = rope_rotate(k_r, np.arange(L), base, inv_freq)
     qpos = np.arange(L - T_q, L)
-    q_r_rot = rope_rotate(q_r, qpos[:, None], base)
+    q_r_rot = rope_rotate(q_r, qpos[:, None], base, inv_freq)
     return mla_attention_explicit(c_kv, k_r_rot, q_c, q_r_rot, w_uk, w_uv, scale,
                                   heads=heads, want_p=want_p)
 

@@ -66,12 +66,14 @@ def test_host_validation_without_device(M):
     bad_block = _cfg(M, block_size=32)
     bad_dc = _cfg(M, d_c=520)
     p = ctypes.c_void_p(FAKE)
-    assert raw("mla_absorb_q", ctypes.byref(bad_block), p, p, p, 4, None) == -2
-    assert raw("mla_absorb_q", ctypes.byref(bad_dc), p, p, p, 4, None) == -2
-    assert raw("mla_absorb_q", ctypes.byref(cfg), None, p, p, 4, None) == -1
-    assert raw("mla_absorb_q", ctypes.byref(cfg), ctypes.c_void_p(FAKE + 2), p, p, 4, None) == -7
-    assert raw("mla_absorb_q", ctypes.byref(cfg), p, p, p, 0, None) == -3
-    assert raw("mla_up_v", ctypes.byref(cfg), p, p, p, 70000, None) == -3
+    assert raw("mla_absorb_q", ctypes.byref(bad_block), p, p, p, 4, None, None) == -2
+    assert raw("mla_absorb_q", ctypes.byref(bad_dc), p, p, p, 4, None, None) == -2
+    assert raw("mla_absorb_q", ctypes.byref(cfg), None, p, p, 4, None, None) == -1
+    assert raw("mla_absorb_q", ctypes.byref(cfg), ctypes.c_void_p(FAKE + 2), p, p, 4, None, None) == -7
+    assert raw("mla_absorb_q", ctypes.byref(cfg), p, p, p, 0, None, None) == -3
+    assert raw("mla_absorb_q", ctypes.byref(cfg), p, p, p, 4, ctypes.c_void_p(FAKE + 2), None) == -7
+    assert raw("mla_up_v", ctypes.byref(cfg), p, p, p, 70000, None, None) == -3
+    assert raw("mla_up_v", ctypes.byref(cfg), p, p, p, 4, ctypes.c_void_p(FAKE + 2), None) == -7
     ws = M.mla_decode_workspace_bytes(cfg, 32, 1, 0)
     assert ws >= 256 and ws % 256 == 0
     assert M.mla_decode_workspace_bytes(cfg, 32, 1, 4) >= M.mla_decode_workspace_bytes(cfg, 32, 1, 1)
@@ -217,3 +219,29 @@ def test_rope_table_argument_checks(M):
     assert M.raw_call("mla_rope_table", 16, ctypes.c_double(10000.0), 4, buf) == 0
     # position 0 is the identity rotation: cos = 1, sin = 0 for every pair
     assert list(buf[:8]) == [1.0] * 8 and list(buf[8:16]) == [0.0] * 8
+
+
+def test_yarn_table_and_scale_match_the_oracle(M):
+    """The library's host-side YaRN table and score scale against the oracle's
+    definitions.  The two sides use different libm implementations, so an
+    entry may differ by one float ulp, or near zero by the rounding of a
+    large angle (about 1e-11 absolute at positions near 1.4e5)."""
+    from oracle import mla_oracle as O
+    for d_r, max_pos in ((64, 140000), (16, 5000)):
+        lib = M.mla_rope_table_yarn(d_r, 10000.0, max_pos).numpy()
+        ref = O.rope_table_f32(max_pos, d_r, inv_freq=O.yarn_inv_freq(d_r))
+        ulp = np.maximum(np.spacing(np.abs(ref).astype(np.float32)), 1e-9)
+        assert np.all(np.abs(lib.astype(np.float64) - ref) <= ulp), d_r
+        assert np.mean(lib != ref) < 1e-4
+    # no stretch: the plain table
+    np.testing.assert_array_equal(M.mla_rope_table_yarn(64, 10000.0, 64, 1.0).numpy(),
+                                  M.mla_rope_table(64, 10000.0, 64).numpy())
+    assert abs(M.mla_yarn_score_scale(128, 64) - O.yarn_score_scale(128, 64)) < 1e-7
+    assert abs(M.mla_yarn_score_scale(128, 64, 40.0, 0.1) - O.yarn_score_scale(128, 64, 40.0, 0.1)) < 1e-7
+    buf = (ctypes.c_float * 64)()
+    assert M.raw_call("mla_rope_table_yarn", 16, ctypes.c_double(10000.0), 4, ctypes.c_double(0.5),
+                      ctypes.c_double(1.0), ctypes.c_double(32.0), 4096, buf) == -3      # s < 1
+    assert M.raw_call("mla_rope_table_yarn", 16, ctypes.c_double(10000.0), 4, ctypes.c_double(40.0),
+                      ctypes.c_double(32.0), ctypes.c_double(1.0), 4096, buf) == -3      # beta <= alpha
+    with pytest.raises(M.MlaError):
+        M.mla_yarn_score_scale(128, 64, 0.5)

@@ -283,32 +283,42 @@ def test_host_argument_errors(M):
 
 
 # ---------------------------------------------------------------------------
-# Full sizes of the five workloads, in the benchmark's launch configuration,
-# checked on sampled sequences and heads.
+# Full sizes of the five workloads, in the benchmark's launch configuration:
+# every head of at least two sequences, plus at least eight seeded sequences
+# (all of them where the workload has fewer) at sampled heads.
 # ---------------------------------------------------------------------------
 
+def _sampled(B, n, seed):
+    rng = np.random.default_rng(seed)
+    return sorted(int(x) for x in rng.choice(B, size=min(n, B), replace=False))
+
+
+# workload: (sequences checked on all heads, sequences checked on SAMPLE_HEADS)
 FULL = {
-    "v2_decode": ([0, 17, 31], [0, 1, 63, 64, 127]),
-    "varlen": ([0, 5, 77, 127], [0, 64, 127]),
-    "long": ([0, 3], [0, 127]),
-    "multi_token": ([0, 63], [0, 65, 127]),
-    "tiny": ([0], None),
+    "tiny": ([0], []),
+    "v2_decode": ([0, 31], _sampled(32, 8, 101)),
+    "varlen": ([0, 77], _sampled(128, 8, 102)),
+    "long": ([0, 3], [1, 2]),
+    "multi_token": ([0, 63], _sampled(64, 8, 103)),
 }
+SAMPLE_HEADS = [0, 1, 63, 64, 65, 127]
 
 
 @pytest.mark.parametrize("name", ["tiny", "v2_decode", "multi_token", "long", "varlen"])
-def test_full_size_sampled(M, name):
+def test_full_size(M, name):
     spec = config_specs()[name]
-    seqs, heads = FULL[name]
+    all_heads, sampled = FULL[name]
     dc = _dc(spec)
     dc.step()
     torch.cuda.synchronize()
     assert dc.decode_status() == 0 and dc.append_status() == 0
-    check_sequences(dc, seqs, heads)
-    # page-table gather of the sampled sequences' cache rows, bit exact
+    check_sequences(dc, all_heads)
+    if sampled:
+        check_sequences(dc, sampled, [h for h in SAMPLE_HEADS if h < spec.n_h])
+    # page-table gather of the fully checked sequences' cache rows, bit exact
     pool = dc.bits(dc.pool)
     tab = O.rope_table_f32(dc.max_pos, spec.d_r)
-    for b in seqs[:2]:
+    for b in all_heads:
         L = int(spec.seq_lens[b])
         rows = O.gather_rows(pool, dc.block_table_np, b, L, spec.block_size)
         assert np.array_equal(rows[:, :spec.d_c], spec.c_kv_rows(b, 0, L))

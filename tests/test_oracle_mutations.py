@@ -45,6 +45,10 @@ MUTATIONS = {
         "a = (x1 * c) - (x2 * s)\n    b = (x2 * c) + (x1 * s)",
         "a = (x1.astype(np.float64) * c - (x2 * s)).astype(np.float32)\n"
         "    b = (x2.astype(np.float64) * c + (x1 * s)).astype(np.float32)"),
+    "yarn_turns_without_two_pi": ("turns = orig_len * f / (2.0 * math.pi)", "turns = orig_len * f"),
+    "yarn_ramp_reversed": ("return f * ((1.0 - gamma) / s + gamma)", "return f * (gamma / s + (1.0 - gamma))"),
+    "yarn_temperature_not_squared": ("return yarn_sqrt_temperature(s, coeff) ** 2 / math.sqrt(d_h + d_r)",
+                                     "return yarn_sqrt_temperature(s, coeff) / math.sqrt(d_h + d_r)"),
     "gather_wrong_slot": ("return int(block_table[b, pos // block_size]), pos % block_size",
                           "return int(block_table[b, pos // block_size]), (pos + 1) % block_size"),
 }

@@ -157,6 +157,69 @@ def test_rope_emulation_rounds_each_product_then_the_sum():
 
 
 # --------------------------------------------------------------------------
+# YaRN on the decoupled RoPE ("Техотчёт DeepSeek-V2 (2024)", long context;
+# "DeepSeek-V2 review", 4): s = 40, alpha = 1, beta = 32, 4K -> 160K
+# --------------------------------------------------------------------------
+
+def test_yarn_with_no_stretch_is_plain_rope():
+    for d_r in (16, 64):
+        np.testing.assert_allclose(O.yarn_inv_freq(d_r, s=1.0), O.rope_inv_freq(d_r), rtol=1e-15, atol=0)
+    assert O.yarn_score_scale(128, 64, s=1.0) == O.default_scale(128, 64)
+
+
+def test_yarn_regimes_at_the_v2_shape():
+    # Derived by hand for d_r = 64, base 10000, a 4096-token training length:
+    # pair m turns 4096 * 10000^(-m/32) / (2 pi) times.  More than 32 turns
+    # (kept) for m <= 10; fewer than 1 turn (interpolated by s) for m >= 23;
+    # the 12 pairs m = 11 .. 22 lie on the ramp.
+    ratio = O.yarn_inv_freq(64) / O.rope_inv_freq(64)
+    kept = np.isclose(ratio, 1.0, rtol=1e-12)
+    interp = np.isclose(ratio, 1.0 / 40.0, rtol=1e-12)
+    assert list(np.flatnonzero(kept)) == list(range(11))
+    assert list(np.flatnonzero(interp)) == list(range(23, 32))
+    ramp = ratio[11:23]
+    assert np.all((ramp > 1.0 / 40.0) & (ramp < 1.0))
+    assert np.all(np.diff(ratio) <= 1e-15)          # slower pairs are stretched more
+
+
+def test_yarn_interpolated_pairs_reach_old_angles_at_stretched_positions():
+    # a pair that turns less than once over the training length makes, over
+    # s times that length, the turn it used to make: its angle at s p equals
+    # the plain angle at p; a fast pair keeps its angle at every position
+    x = _rng(21).standard_normal((5, 64))
+    p = np.array([0, 7, 100, 1000, 4095], np.float64)
+    yarn = O.yarn_inv_freq(64)
+    slow = np.r_[23:32]
+    fast = np.r_[0:11]
+    got = O.rope_rotate(x, 40.0 * p, inv_freq=yarn)
+    want = O.rope_rotate(x, p)
+    np.testing.assert_allclose(got[:, slow], want[:, slow], atol=1e-9)
+    np.testing.assert_allclose(got[:, 32 + slow], want[:, 32 + slow], atol=1e-9)
+    got_fast = O.rope_rotate(x, p, inv_freq=yarn)
+    np.testing.assert_allclose(got_fast[:, fast], want[:, fast], atol=1e-12)
+
+
+def test_yarn_keeps_the_relative_position_property():
+    r = _rng(22)
+    q, k = r.standard_normal(64), r.standard_normal(64)
+    f = O.yarn_inv_freq(64)
+    a = O.rope_rotate(q, 130000, inv_freq=f) @ O.rope_rotate(k, 129000, inv_freq=f)
+    b = O.rope_rotate(q, 1000, inv_freq=f) @ O.rope_rotate(k, 0, inv_freq=f)
+    assert abs(a - b) < 1e-8
+
+
+def test_yarn_temperature_and_target_length():
+    # the page's numbers: s = 40 stretches the 4K training length to 160K
+    assert 40 * 4096 == 160 * 1024
+    # sqrt(t) = 0.0707 ln s + 1 (DeepSeek-V2's coefficient; 0.1 in the generic
+    # rule): ln 40 = 3.6888795, so sqrt(t) = 1.2608038 and t = 1.5896262;
+    # every score is multiplied by t
+    assert abs(O.yarn_sqrt_temperature(40.0) - 1.2608038) < 1e-6
+    assert abs(O.yarn_sqrt_temperature(40.0, 0.1) - 1.3688879) < 1e-6
+    assert abs(O.yarn_score_scale(128, 64) * math.sqrt(192) - 1.5896262) < 1e-6
+
+
+# --------------------------------------------------------------------------
 # Hand-computed tiny case: n_h = 1, d_c = 2, d_h = 1, d_r = 2, L = 2, T_q = 1
 # --------------------------------------------------------------------------
 
