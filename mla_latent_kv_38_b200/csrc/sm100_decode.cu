@@ -1155,7 +1155,14 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, 
 // cluster: one warp per (unit, head row), a lane per 16 latent columns.  The
 // slots of unit u are meta.y + u .. meta.y + u + meta.z - 1.  Units of an
 // invalid sequence (kv_len 0) get zeros and lse = -inf.
-__global__ void __launch_bounds__(256)
+//
+// The partial rows were written by the decode kernel just before and are read
+// from L2 (ld.global.cg).  The first two slots' rows are fetched together with
+// the log-sum-exps, so that a row split in two takes two dependent round trips
+// (metadata, then everything else); further slots follow two at a time.  At
+// most 64 registers a thread: 8 warps of every SM's 4 blocks are resident at
+// once, one wave for the 4,096 rows of 32 split units.
+__global__ void __launch_bounds__(256, 4)
 mla_sm100_merge_kernel(const int4* __restrict__ unit_meta, const float* __restrict__ part_o,
                        const float* __restrict__ part_lse, uint16_t* __restrict__ out_latent,
                        float* __restrict__ out_lse, int n_h, int n_hb, int B, int T_q, int U) {
@@ -1166,62 +1173,64 @@ mla_sm100_merge_kernel(const int4* __restrict__ unit_meta, const float* __restri
     const int u = wg >> 7, row = wg & 127;
     if (u >= U) return;
     const int4 meta = unit_meta[u];
-    const UnitIdx x = unit_index(u, n_hb, B);
-    const int bt = x.b * T_q + x.t, hb = x.hb;
-    const size_t grow = static_cast<size_t>(bt) * n_h + hb * 128 + row;
-    uint4* dst = reinterpret_cast<uint4*>(out_latent + grow * kDc + lane * 16);
+    auto out_row = [&]() {   // this warp's output row
+        const UnitIdx x = unit_index(u, n_hb, B);
+        return static_cast<size_t>(x.b * T_q + x.t) * n_h + x.hb * 128 + row;
+    };
     if (meta.x == 0) {
+        const size_t grow = out_row();
+        uint4* dst = reinterpret_cast<uint4*>(out_latent + grow * kDc + lane * 16);
         dst[0] = make_uint4(0, 0, 0, 0);
         dst[1] = make_uint4(0, 0, 0, 0);
         if (lane == 0) out_lse[grow] = -INFINITY;
         return;
     }
-    const int parts = meta.z;
+    const int parts = meta.z;   // <= kClusters
     if (parts <= 1) return;
     const size_t slot0 = static_cast<size_t>(meta.y) + u;
-    float mx = -INFINITY;
-    for (int i = lane; i < parts; i += 32) mx = fmaxf(mx, part_lse[(slot0 + i) * 128 + row]);
-    mx = warp_max(mx);
-    float z = 0.f;
+    const float* lse_row = part_lse + slot0 * 128 + row;                                       // slot i at + 128 i
+    const float4* o_row = reinterpret_cast<const float4*>(part_o + (slot0 * 128 + row) * kDc) + lane * 4;
+    constexpr size_t kSlot4 = static_cast<size_t>(128) * kDc / 4;                             // float4 per slot
+    auto load_pair = [&](float4 (&v)[2][4], int i) {   // slots i, i + 1 (zeros past the last)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[0][k] = __ldcg(o_row + i * kSlot4 + k);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            v[1][k] = i + 1 < parts ? __ldcg(o_row + (i + 1) * kSlot4 + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    float4 v[2][4];
+    load_pair(v, 0);
+    // log-sum-exp of slot lane + 32 k in ls[k] (parts <= 74 < 96)
+    float ls[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) ls[k] = lane + 32 * k < parts ? __ldcg(lse_row + 128 * (lane + 32 * k)) : -INFINITY;
+    const float mx = warp_max(fmaxf(fmaxf(ls[0], ls[1]), ls[2]));
+    auto w_of = [&](float l) { return l == -INFINITY ? 0.f : ex2((l - mx) * kLog2e); };
+    const float z = warp_sum(w_of(ls[0]) + w_of(ls[1]) + w_of(ls[2]));
+    auto weight = [&](int i) {   // slot i's weight, from the lane that holds its log-sum-exp
+        const float l = i < 32 ? ls[0] : (i < 64 ? ls[1] : ls[2]);
+        return w_of(__shfl_sync(0xffffffffu, l, i & 31));
+    };
     float acc[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-    for (int i0 = 0; i0 < parts; i0 += 32) {
-        const int i = i0 + lane;
-        const float ls = i < parts ? part_lse[(slot0 + i) * 128 + row] : -INFINITY;
-        const float wl = ls == -INFINITY ? 0.f : ex2((ls - mx) * kLog2e);
-        z += wl;
-        const int n = min(32, parts - i0);
-        // four slots' loads in flight before they are combined
-        for (int j0 = 0; j0 < n; j0 += 4) {
-            float4 v[4][4];
-            float wj[4];
+    for (int i = 0; i < parts; i += 2) {
+        if (i > 0) load_pair(v, i);
+        const float w0 = weight(i), w1 = i + 1 < parts ? weight(i + 1) : 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int j = min(j0 + jj, n - 1);
-                const float wsh = __shfl_sync(0xffffffffu, wl, j);
-                wj[jj] = j0 + jj < n ? wsh : 0.f;
-                const float4* src = reinterpret_cast<const float4*>(part_o + ((slot0 + i0 + j) * 128 + row) * kDc) +
-                                    lane * 4;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) v[jj][k] = src[k];
-            }
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    acc[4 * k + 0] = fmaf(wj[jj], v[jj][k].x, acc[4 * k + 0]);
-                    acc[4 * k + 1] = fmaf(wj[jj], v[jj][k].y, acc[4 * k + 1]);
-                    acc[4 * k + 2] = fmaf(wj[jj], v[jj][k].z, acc[4 * k + 2]);
-                    acc[4 * k + 3] = fmaf(wj[jj], v[jj][k].w, acc[4 * k + 3]);
-                }
+        for (int k = 0; k < 4; ++k) {
+            acc[4 * k + 0] = fmaf(w1, v[1][k].x, fmaf(w0, v[0][k].x, acc[4 * k + 0]));
+            acc[4 * k + 1] = fmaf(w1, v[1][k].y, fmaf(w0, v[0][k].y, acc[4 * k + 1]));
+            acc[4 * k + 2] = fmaf(w1, v[1][k].z, fmaf(w0, v[0][k].z, acc[4 * k + 2]));
+            acc[4 * k + 3] = fmaf(w1, v[1][k].w, fmaf(w0, v[0][k].w, acc[4 * k + 3]));
         }
     }
-    z = warp_sum(z);
     const float inv = z > 0.f ? 1.f / z : 0.f;
     uint32_t pk[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2(acc[2 * k] * inv, acc[2 * k + 1] * inv);
+    const size_t grow = out_row();
+    uint4* dst = reinterpret_cast<uint4*>(out_latent + grow * kDc + lane * 16);
     dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     if (lane == 0) out_lse[grow] = z > 0.f ? mx + logf(z) : -INFINITY;
