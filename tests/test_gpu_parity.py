@@ -120,6 +120,25 @@ def test_many_units_whole_and_split(M):
     check_sequences(dc, [0, 1, 150, 298, 299])
 
 
+def test_schedule_kernel_for_many_units(M):
+    """Above 2,048 units (query row, block of 128 heads) the schedule is
+    computed by a separate one-block kernel before the decode (three launches
+    instead of two).  2,100 sequences of 70 to 260 keys: most units lie inside
+    one SM pair's range, those at the cuts are split and merged."""
+    lens = np.array([70 + (37 * b) % 191 for b in range(2100)], np.int32)
+    spec = CaseSpec(**V2, seq_lens=lens, seed=13, permute_blocks=True)
+    dc = _dc(spec)
+    assert M.mla_decode_launches(dc.cfg, spec.B, 1, 0) == 3
+    dc.step()
+    torch.cuda.synchronize()
+    assert dc.decode_status() == 0
+    parts = M.mla_decode_split_counts(dc.cfg, spec.B, 1, 0, dc.ws, spec.B).numpy()
+    assert parts.min() >= 1 and parts.max() >= 2
+    split = [int(b) for b in np.nonzero(parts >= 2)[0]]
+    whole = [int(b) for b in np.nonzero(parts == 1)[0]]
+    check_sequences(dc, sorted(set(split[:3] + split[-2:] + whole[:2] + whole[-2:] + [1049])))
+
+
 SPLIT_SPEC = dict(seq_lens=np.array([1000, 37, 513], np.int32), seed=6)
 
 
