@@ -123,9 +123,11 @@ def test_many_units_whole_and_split(M):
 def test_schedule_kernel_for_many_units(M):
     """Above 2,048 units (query row, block of 128 heads) the schedule is
     computed by a separate one-block kernel before the decode (three launches
-    instead of two).  2,100 sequences of 70 to 260 keys: most units lie inside
-    one SM pair's range, those at the cuts are split and merged."""
-    lens = np.array([70 + (37 * b) % 191 for b in range(2100)], np.int32)
+    instead of two).  2,100 sequences: most of 70 to 260 keys (one 256-key
+    tile, never split: cuts fall between tiles), every seventh of 600 to 899
+    keys (3 or 4 tiles), so that some cuts fall inside a unit, which is then
+    split and merged."""
+    lens = np.array([600 + (37 * b) % 300 if b % 7 == 0 else 70 + (37 * b) % 191 for b in range(2100)], np.int32)
     spec = CaseSpec(**V2, seq_lens=lens, seed=13, permute_blocks=True)
     dc = _dc(spec)
     assert M.mla_decode_launches(dc.cfg, spec.B, 1, 0) == 3
