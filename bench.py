@@ -3,7 +3,7 @@
 on the DeepSeek-V2 decode workload, printed as one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload v2_decode|varlen|long|multi_token|tiny]
+                    [--workload v2_decode|varlen|long|multi_token|tiny|prefill_chunk|prefill]
 
 N > 1 runs under torch.distributed.run, one process per GPU.  Sequences are
 independent, so every rank runs its own full copy of the workload (weak scaling)
@@ -190,8 +190,8 @@ def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
-    from mla_latent_kv_38_b200.workloads import config_specs
-    spec = config_specs()[args.workload]
+    from mla_latent_kv_38_b200.workloads import workload_specs
+    spec = workload_specs()[args.workload]
     rate, secs, desc = oracle_sample_rate(spec, args.steps, args.warmup)
     line = {
         "metric": METRIC, "impl": "reference", "value": rate, "unit": "tokens/s",
@@ -252,9 +252,9 @@ def run_ours(args):
         pg = dist
     from mla_latent_kv_38_b200 import binding as M
     from mla_latent_kv_38_b200.runner import DeviceCase
-    from mla_latent_kv_38_b200.workloads import config_specs
+    from mla_latent_kv_38_b200.workloads import workload_specs
 
-    spec = config_specs()[args.workload]
+    spec = workload_specs()[args.workload]
     dc = DeviceCase(spec, impl=args.kernel_impl, max_splits=args.max_splits, device=f"cuda:{local}")
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)

@@ -193,7 +193,12 @@ size_t mla_decode_workspace_bytes(const mla_config_t* cfg, int B, int T_q, int m
  *     portable kernels: exactly max_splits parts (0: a count from B, T_q, n_h).
  * Partial results (fp32 latent rows and log-sum-exp) of split rows go to the
  * workspace and are merged by a log-sum-exp reduction kernel.  The workspace
- * starts with the device status word (mla_read_status).  T_q <= 16. */
+ * starts with the device status word (mla_read_status).
+ * Sizes: B * T_q <= 65535 query rows (and B * T_q * n_h / 128 <= 65535 units
+ * on the tcgen05 kernels).  T_q > 1 with the generalised mask is also chunked
+ * prefill ([notes] "MLA 코드 구현", "학습 시와 디코딩 시의 흐름"): a chunk of
+ * T_q new tokens, appended by mla_rope_append, attends to the cached prefix
+ * and causally to itself; T_q = seq_lens[b] is prefill from an empty cache. */
 int mla_decode(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q_r,
                const mla_bf16* pool, int num_blocks, const int32_t* block_table,
                int max_blocks_per_seq, const int32_t* seq_lens, int B, int T_q,

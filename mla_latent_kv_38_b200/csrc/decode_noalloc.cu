@@ -65,7 +65,7 @@ extern "C" int mla_decode_noalloc(const mla_config_t* cfg, const mla_bf16* q_abs
     if (!al16(q_abs) || !al16(q_r) || !al16(pool) || !al16(out_latent) || !al4(out_lse) ||
         !al4(block_table) || !al4(seq_lens) || (dev_status && !al4(dev_status)))
         return MLA_ERR_ALIGN;
-    if (B < 1 || T_q < 1 || T_q > 16 || static_cast<long>(B) * T_q > 65535) return MLA_ERR_SIZE;
+    if (B < 1 || T_q < 1 || static_cast<long>(B) * T_q > 65535) return MLA_ERR_SIZE;
     if (num_blocks < 1 || max_blocks_per_seq < 1 || splits < 1 || splits > 256) return MLA_ERR_SIZE;
 
     // Scratch use: split partials, fp32 latent rows then fp32 lse, 256-aligned.

@@ -61,6 +61,16 @@ WsLayout ws_layout(const mla_config_t* c, int B, int T_q, int max_splits) {
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_LAUNCH; }
 
+// Query rows of a decode call: B sequences x T_q tokens, T_q from 1 (decode)
+// to a whole prefill chunk; at most 65,535 rows, and for the tcgen05 kernels
+// at most 65,535 units of (query row, block of 128 heads).
+bool rows_ok(const mla_config_t* c, int B, int T_q) {
+    if (B < 1 || T_q < 1) return false;
+    const long rows = static_cast<long>(B) * T_q;
+    if (rows > 65535) return false;
+    return !uses_sm100(c) || rows * (c->n_h / 128) <= 65535;
+}
+
 }  // namespace
 
 namespace mla {
@@ -200,7 +210,7 @@ int mla_rope_append(const mla_config_t* cfg, mla_bf16* q_r, const mla_bf16* k_r,
 }
 
 size_t mla_decode_workspace_bytes(const mla_config_t* cfg, int B, int T_q, int max_splits) {
-    if (check_config(cfg) || B < 1 || T_q < 1 || max_splits < 0) return 0;
+    if (check_config(cfg) || !rows_ok(cfg, B, T_q) || max_splits < 0) return 0;
     if (cfg->impl == 2 && !mla::sm100_supports(cfg->n_h, cfg->d_c, cfg->d_r)) return 0;
     return ws_layout(cfg, B, T_q, max_splits).total;
 }
@@ -217,7 +227,7 @@ int mla_decode(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q
     if (!aligned16(q_abs) || !aligned16(q_r) || !aligned16(pool) || !aligned16(out_latent) ||
         !aligned4(out_lse) || !aligned4(block_table) || !aligned4(seq_lens))
         return MLA_ERR_ALIGN;
-    if (B < 1 || T_q < 1 || T_q > 16 || static_cast<long>(B) * T_q > 65535) return MLA_ERR_SIZE;
+    if (!rows_ok(cfg, B, T_q)) return MLA_ERR_SIZE;
     if (num_blocks < 1 || max_blocks_per_seq < 1 || max_splits < 0) return MLA_ERR_SIZE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLA_ERR_WORKSPACE;
     const bool sm100_shape = mla::sm100_supports(cfg->n_h, cfg->d_c, cfg->d_r);
@@ -262,7 +272,7 @@ int mla_decode(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q
 int mla_decode_launches(const mla_config_t* cfg, int B, int T_q, int max_splits) {
     int rc = check_config(cfg);
     if (rc) return rc;
-    if (B < 1 || T_q < 1 || T_q > 16 || max_splits < 0) return MLA_ERR_SIZE;
+    if (!rows_ok(cfg, B, T_q) || max_splits < 0) return MLA_ERR_SIZE;
     const bool sm100_shape = mla::sm100_supports(cfg->n_h, cfg->d_c, cfg->d_r);
     if (cfg->impl == 2 && !sm100_shape) return MLA_ERR_CONFIG;
     if (cfg->impl == 2 || (cfg->impl == 0 && sm100_shape))
@@ -275,7 +285,7 @@ int mla_decode_split_counts(const mla_config_t* cfg, int B, int T_q, int max_spl
     int rc = check_config(cfg);
     if (rc) return rc;
     if (!workspace || !host_counts) return MLA_ERR_NULL;
-    if (B < 1 || T_q < 1 || T_q > 16 || max_splits < 0) return MLA_ERR_SIZE;
+    if (!rows_ok(cfg, B, T_q) || max_splits < 0) return MLA_ERR_SIZE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (!uses_sm100(cfg)) {
         const int s = choose_splits(cfg, B, T_q, max_splits);

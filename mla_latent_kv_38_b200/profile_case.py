@@ -12,7 +12,7 @@ import argparse
 import torch
 
 from .runner import DeviceCase
-from .workloads import config_specs
+from .workloads import workload_specs
 
 
 def main():
@@ -22,7 +22,7 @@ def main():
     ap.add_argument("--impl", type=int, default=0)
     ap.add_argument("--decode-only", action="store_true")
     a = ap.parse_args()
-    dc = DeviceCase(config_specs()[a.workload], impl=a.impl)
+    dc = DeviceCase(workload_specs()[a.workload], impl=a.impl)
     for _ in range(a.iters):
         dc.reset_step_inputs()
         if a.decode_only:

@@ -138,3 +138,25 @@ def config_specs():
         "multi_token": CaseSpec(**v2, seq_lens=np.full(64, 8192, np.int32), T_q=4,
                                 name="multi-token B=64 T_q=4 L=8192"),
     }
+
+
+def prefill_specs():
+    """Chunked prefill on the same paged cache (the decode call with T_q new
+    tokens per sequence under the generalised causal mask): a 512-token chunk
+    appended to a 3,584-token prefix, and prefill of 2,048 tokens from an empty
+    cache.  DeepSeek-V2 head shapes."""
+    v2 = dict(n_h=128, d_c=512, d_h=128, d_r=64)
+    return {
+        "prefill_chunk": CaseSpec(**v2, seq_lens=np.full(4, 4096, np.int32), T_q=512,
+                                  name="chunked prefill B=4 chunk 512 L=4096"),
+        "prefill": CaseSpec(**v2, seq_lens=np.full(1, 2048, np.int32), T_q=2048,
+                            name="prefill B=1 T=2048 from an empty cache"),
+    }
+
+
+def workload_specs():
+    """Every named workload: the five decode configurations and the prefill ones."""
+    out = config_specs()
+    out.update(prefill_specs())
+    return out
+

@@ -83,7 +83,7 @@ def test_host_validation_without_device(M):
     args[11] = ctypes.c_void_p(FAKE + 16)          # workspace must be 256-byte aligned
     assert raw("mla_decode", *args) == -4
     args[11] = p
-    args[9] = 17                                    # T_q > 16
+    args[9] = 2048                                  # B * T_q = 65,536 query rows: one too many
     assert raw("mla_decode", *args) == -3
     args[9] = 1
     args[1] = None
@@ -136,12 +136,17 @@ def test_decode_launch_counts(M):
     assert M.raw_call("mla_decode_launches", ctypes.byref(simt), 32, 1, 4) == 2
     # automatic choice: 32 rows x 16 head groups fill 8 x 148 slots with 3 splits
     assert M.raw_call("mla_decode_launches", ctypes.byref(simt), 32, 1, 0) == 2
-    assert M.raw_call("mla_decode_launches", ctypes.byref(simt), 4096, 16, 0) == 1
+    assert M.raw_call("mla_decode_launches", ctypes.byref(simt), 4095, 16, 0) == 1
+    # prefill-sized chunks: T_q is limited only by the row and unit counts
+    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 1, 2048, 0) == 2
+    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 4, 4096, 0) == 3
+    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 2, 32768, 0) == -3
+    assert M.raw_call("mla_decode_launches", ctypes.byref(_cfg(M, n_h=256)), 1, 40000, 0) == -3
     tiny = _cfg(M, n_h=4, d_c=64, d_h=32, d_r=16)
     assert M.raw_call("mla_decode_launches", ctypes.byref(tiny), 1, 1, 0) == 2
     tiny_tc = _cfg(M, n_h=4, d_c=64, d_h=32, d_r=16, impl=2)
     assert M.raw_call("mla_decode_launches", ctypes.byref(tiny_tc), 1, 1, 0) == -2
-    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 32, 17, 0) == -3
+    assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 32, 2048, 0) == -3
     assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 0, 1, 0) == -3
     assert M.raw_call("mla_decode_launches", ctypes.byref(v2), 32, 1, -1) == -3
     # the workspace query answers 0 for arguments the decode call would reject

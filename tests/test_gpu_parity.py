@@ -295,7 +295,7 @@ def test_host_argument_errors(M):
     assert e.value.code == -4
     with pytest.raises(M.MlaError) as e:
         M.mla_decode(dc.cfg, dc.q_abs, dc.q_r, dc.pool, spec.num_blocks, dc.block_table,
-                     spec.max_blocks, dc.seq_lens, 1, 17, 0, dc.ws, dc.ws_bytes, dc.latent, dc.lse)
+                     spec.max_blocks, dc.seq_lens, 1, 65536, 0, dc.ws, dc.ws_bytes, dc.latent, dc.lse)
     assert e.value.code == -3
     bad = M.MlaConfig(128, 512, 128, 64, block_size=32)
     with pytest.raises(M.MlaError) as e:
