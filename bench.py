@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--workload", default="v2_decode")
     ap.add_argument("--kernel-impl", type=int, default=0, help="mla_config_t.impl (0 auto)")
     ap.add_argument("--max-splits", type=int, default=0)
+    ap.add_argument("--yarn", action="store_true",
+                    help="YaRN-scaled RoPE on k^R (s = 40, alpha = 1, beta = 32, 4K training length) "
+                         "and its attention temperature in the score scale")
     return ap.parse_args()
 
 
@@ -150,12 +153,22 @@ class ClockSampler:
 # the oracle arm
 # ---------------------------------------------------------------------------
 
-def oracle_sample_rate(spec, steps, warmup, heads_per_step=8, budget_s=None):
+# YaRN parameters of the long-context extension (4K -> 128K on k^R)
+YARN = dict(s=40.0, alpha=1.0, beta=32.0, orig_len=4096, coeff=0.0707)
+
+
+def oracle_sample_rate(spec, steps, warmup, heads_per_step=8, budget_s=None, yarn=False):
     """Time the fp64 oracle on `heads_per_step` heads of one sequence per step.
 
     Returns (tokens/s, seconds, description).  A token's output needs all n_h
     heads, so a step credits heads_per_step / n_h of each of its T_q tokens."""
     from oracle.evaluate import reference
+    kw = {}
+    if yarn:
+        from oracle import mla_oracle as O
+        kw = dict(inv_freq=O.yarn_inv_freq(spec.d_r, s=YARN["s"], alpha=YARN["alpha"], beta=YARN["beta"],
+                                           orig_len=YARN["orig_len"]),
+                  scale=O.yarn_score_scale(spec.d_h, spec.d_r, s=YARN["s"], coeff=YARN["coeff"]))
     b = 0
     heads_all = list(range(spec.n_h))
     heads_per_step = min(heads_per_step, spec.n_h)
@@ -163,7 +176,7 @@ def oracle_sample_rate(spec, steps, warmup, heads_per_step=8, budget_s=None):
     for i in range(warmup + steps):
         hs = [heads_all[(i * heads_per_step + j) % spec.n_h] for j in range(heads_per_step)]
         t0 = time.perf_counter()
-        reference(spec, b, heads=hs)
+        reference(spec, b, heads=hs, **kw)
         dt = time.perf_counter() - t0
         if i >= warmup:
             t_total += dt
@@ -192,13 +205,13 @@ def run_reference(args):
         return 0
     from mla_latent_kv_38_b200.workloads import workload_specs
     spec = workload_specs()[args.workload]
-    rate, secs, desc = oracle_sample_rate(spec, args.steps, args.warmup)
+    rate, secs, desc = oracle_sample_rate(spec, args.steps, args.warmup, yarn=args.yarn)
     line = {
         "metric": METRIC, "impl": "reference", "value": rate, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * secs / max(args.steps, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": spec.name},
+        "config": {"workload": spec.name, "rope": "yarn" if args.yarn else "plain"},
         "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -255,7 +268,8 @@ def run_ours(args):
     from mla_latent_kv_38_b200.workloads import workload_specs
 
     spec = workload_specs()[args.workload]
-    dc = DeviceCase(spec, impl=args.kernel_impl, max_splits=args.max_splits, device=f"cuda:{local}")
+    dc = DeviceCase(spec, impl=args.kernel_impl, max_splits=args.max_splits, device=f"cuda:{local}",
+                    yarn=YARN if args.yarn else None)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     launches_decode = M.mla_decode_launches(dc.cfg, spec.B, spec.T_q, args.max_splits)
@@ -459,7 +473,7 @@ def run_ours(args):
 
     cpu = None
     if world == 1:
-        rate, secs, desc = oracle_sample_rate(spec, steps=4, warmup=1, budget_s=20.0)
+        rate, secs, desc = oracle_sample_rate(spec, steps=4, warmup=1, budget_s=20.0, yarn=args.yarn)
         cpu = {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": desc}
 
@@ -472,7 +486,7 @@ def run_ours(args):
                    "d_c": spec.d_c, "d_r": spec.d_r, "block_size": spec.block_size,
                    "context": [int(spec.seq_lens.min()), int(spec.seq_lens.max())],
                    "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write)",
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": f"replicas x{world}", "rope": "yarn" if args.yarn else "plain"},
         "phases_us": phases_us, "phases_median_us": phases_med_us,
         "timing": "device passes replay CUDA graphs of the C-ABI calls; e2e calls the API directly",
         "host_enqueue_us_per_step": 1e6 * host_s / K,
