@@ -34,6 +34,9 @@ TID = {
     "w_uv": 6,
     "seq_lens": 7,
     "block_perm": 8,
+    "c_q": 9,
+    "w_uq": 10,
+    "w_o": 11,
 }
 
 

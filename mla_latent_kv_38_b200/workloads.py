@@ -35,6 +35,8 @@ class CaseSpec:
     permute_blocks: bool = False
     block_size: int = 64
     name: str = ""
+    d_cq: int = 1536                # query latent (W^UQ's input), DeepSeek-V2
+    d_model: int = 5120             # model width (W^O's output), DeepSeek-V2
 
     @property
     def B(self):
@@ -96,6 +98,18 @@ class CaseSpec:
     def w_uk(self):
         return synth.normal_bf16(self.seed, synth.TID["w_uk"], (self.n_h, self.d_h, self.d_c),
                                  std=synth.weight_std(self.d_c))
+
+    def c_q(self):
+        """Query latents c^Q (the input of W^UQ), one per token."""
+        return synth.normal_bf16(self.seed, synth.TID["c_q"], (self.n_tok, self.d_cq))
+
+    def w_uq(self):
+        return synth.normal_bf16(self.seed, synth.TID["w_uq"], (self.n_h, self.d_h, self.d_cq),
+                                 std=synth.weight_std(self.d_cq))
+
+    def w_o(self):
+        return synth.normal_bf16(self.seed, synth.TID["w_o"], (self.d_model, self.n_h, self.d_h),
+                                 std=synth.weight_std(self.n_h * self.d_h))
 
     def w_uv(self):
         return synth.normal_bf16(self.seed, synth.TID["w_uv"], (self.n_h, self.d_h, self.d_c),

@@ -28,7 +28,9 @@ the GPU receives:
 
 Also here, for tests that need them: the absorbed-query and value up-projection
 definitions (eq. 10/11 applied to a query or a latent, "Key에 대한 수식 전개",
-"Value에 대한 수식 전개"), the paged-cache index arithmetic, the log-sum-exp
+"Value에 대한 수식 전개"), the query up-projection and output projection on
+either side of the path and their folded weights (W^UK into W^UQ, W^UV into
+W^O, same sections), the paged-cache index arithmetic, the log-sum-exp
 merge of split partials, an emulation of the GPU's float32 RoPE arithmetic for
 the bit-exact append check, and the per-token cache-size formulas of the
 "Сколько получилось" table.
@@ -214,6 +216,60 @@ def up_v(latent: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
     for i in range(latent.shape[1]):
         out[:, i, :] = latent[:, i, :] @ w_uv[i].T
     return out
+
+
+# ---------------------------------------------------------------------------
+# The projections on either side of the path, and their folded forms
+# ("MLA 논문정리", "Key에 대한 수식 전개": W'^Q = (W^Q)^T W^UK, and "Value에
+# 대한 수식 전개": W'^O = W^O W^UV; "Техотчёт DeepSeek-V2 (2024)", "Идея 1")
+# ---------------------------------------------------------------------------
+
+
+def q_up(c_q: np.ndarray, w_uq: np.ndarray) -> np.ndarray:
+    """q^C[n, i, :] = W^UQ_i c^Q[n]: the query up-projection from the query latent.
+
+    c_q: (n_tok, d_cq); w_uq: (n_h, d_h, d_cq) -> (n_tok, n_h, d_h)."""
+    c_q = np.asarray(c_q, dtype=np.float64)
+    w_uq = np.asarray(w_uq, dtype=np.float64)
+    return np.einsum("hkd,nd->nhk", w_uq, c_q)
+
+
+def o_proj(o: np.ndarray, w_o: np.ndarray) -> np.ndarray:
+    """u[n] = W^O [o[n, 0, :]; ...; o[n, n_h - 1, :]] = sum_i W^O_i o[n, i, :].
+
+    o: (n_tok, n_h, d_h); w_o: (d_model, n_h, d_h) -> (n_tok, d_model)."""
+    o = np.asarray(o, dtype=np.float64)
+    w_o = np.asarray(w_o, dtype=np.float64)
+    return np.einsum("mhk,nhk->nm", w_o, o)
+
+
+def fold_q(w_uq: np.ndarray, w_uk: np.ndarray) -> np.ndarray:
+    """F_i = W^UK_i^T W^UQ_i, so that q_abs[n, i, :] = F_i c^Q[n] in one product.
+
+    w_uq: (n_h, d_h, d_cq); w_uk: (n_h, d_h, d_c) -> (n_h, d_c, d_cq)."""
+    w_uq = np.asarray(w_uq, dtype=np.float64)
+    w_uk = np.asarray(w_uk, dtype=np.float64)
+    return np.einsum("hkc,hkd->hcd", w_uk, w_uq)
+
+
+def fold_o(w_o: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
+    """G_i = W^O_i W^UV_i, so that u[n] = sum_i G_i latent[n, i, :]: one product
+    with K = n_h d_c over the whole latent output.
+
+    w_o: (d_model, n_h, d_h); w_uv: (n_h, d_h, d_c) -> (d_model, n_h, d_c)."""
+    w_o = np.asarray(w_o, dtype=np.float64)
+    w_uv = np.asarray(w_uv, dtype=np.float64)
+    return np.einsum("mhk,hkc->mhc", w_o, w_uv)
+
+
+def folded_q(c_q: np.ndarray, f: np.ndarray) -> np.ndarray:
+    """q_abs[n, i, :] = F_i c^Q[n]; c_q: (n_tok, d_cq), f: (n_h, d_c, d_cq)."""
+    return np.einsum("hcd,nd->nhc", np.asarray(f, dtype=np.float64), np.asarray(c_q, dtype=np.float64))
+
+
+def folded_o(latent: np.ndarray, g: np.ndarray) -> np.ndarray:
+    """u[n] = sum_i G_i latent[n, i, :]; latent: (n_tok, n_h, d_c), g: (d_model, n_h, d_c)."""
+    return np.einsum("mhc,nhc->nm", np.asarray(g, dtype=np.float64), np.asarray(latent, dtype=np.float64))
 
 
 # ---------------------------------------------------------------------------

@@ -49,6 +49,16 @@ MUTATIONS = {
     "yarn_ramp_reversed": ("return f * ((1.0 - gamma) / s + gamma)", "return f * (gamma / s + (1.0 - gamma))"),
     "yarn_temperature_not_squared": ("return yarn_sqrt_temperature(s, coeff) ** 2 / math.sqrt(d_h + d_r)",
                                      "return yarn_sqrt_temperature(s, coeff) / math.sqrt(d_h + d_r)"),
+    "fold_q_uses_query_weight_twice": ('return np.einsum("hkc,hkd->hcd", w_uk, w_uq)',
+                                       'return np.einsum("hkc,hkd->hcd", w_uq[..., :w_uk.shape[2]], w_uq)'),
+    "fold_o_head_mismatch": ('return np.einsum("mhk,hkc->mhc", w_o, w_uv)',
+                                  'return np.einsum("mhk,hkc->mhc", w_o, w_uv[::-1])'),
+    "q_up_transposed_contraction": ('return np.einsum("hkd,nd->nhk", w_uq, c_q)',
+                                    'return np.einsum("hkd,nd->nhk", w_uq[:, ::-1], c_q)'),
+    "o_proj_head_order": ('return np.einsum("mhk,nhk->nm", w_o, o)',
+                          'return np.einsum("mhk,nhk->nm", w_o, o[:, ::-1])'),
+    "folded_q_wrong_axis": ('return np.einsum("hcd,nd->nhc", np.asarray(f, dtype=np.float64)',
+                            'return np.einsum("hcd,nd->nhc", np.asarray(f[::-1], dtype=np.float64)'),
     "gather_wrong_slot": ("return int(block_table[b, pos // block_size]), pos % block_size",
                           "return int(block_table[b, pos // block_size]), (pos + 1) % block_size"),
 }

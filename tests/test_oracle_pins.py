@@ -479,3 +479,62 @@ def test_cache_sizes_printed_on_pages():
     code_mla = f("MLA", d_c=64, d_r=16, layers=1)
     assert code_mha == g["code_mha_numbers"] and code_mla == g["code_mla_numbers"]
     assert round(code_mha / code_mla) == g["code_ratio_approx"]
+
+
+# ---------------------------------------------------------------------------
+# Folded projections ("MLA 논문정리", "Key에 대한 수식 전개": W'^Q = (W^Q)^T W^UK;
+# "Value에 대한 수식 전개": W'^O = W^O W^UV).  Each definition is pinned by a
+# brute-force sum over its indices, written out here with plain loops, and the
+# folded forms by the identity with the two-step products they replace.
+# ---------------------------------------------------------------------------
+
+def _fold_case(seed=7, n_h=2, d_h=3, d_c=4, d_cq=5, d_model=6, n_tok=2):
+    r = np.random.default_rng(seed)
+    return dict(w_uq=r.standard_normal((n_h, d_h, d_cq)), w_uk=r.standard_normal((n_h, d_h, d_c)),
+                w_uv=r.standard_normal((n_h, d_h, d_c)), w_o=r.standard_normal((d_model, n_h, d_h)),
+                c_q=r.standard_normal((n_tok, d_cq)), lat=r.standard_normal((n_tok, n_h, d_c)),
+                o=r.standard_normal((n_tok, n_h, d_h)))
+
+
+def test_query_up_projection_and_output_projection_by_brute_force():
+    z = _fold_case()
+    n_h, d_h, d_cq = z["w_uq"].shape
+    d_model = z["w_o"].shape[0]
+    q = O.q_up(z["c_q"], z["w_uq"])
+    u = O.o_proj(z["o"], z["w_o"])
+    for n in range(z["c_q"].shape[0]):
+        for i in range(n_h):
+            for k in range(d_h):
+                want = sum(z["w_uq"][i, k, d] * z["c_q"][n, d] for d in range(d_cq))
+                assert abs(q[n, i, k] - want) < 1e-12
+        for m in range(d_model):
+            want = sum(z["w_o"][m, i, k] * z["o"][n, i, k] for i in range(n_h) for k in range(d_h))
+            assert abs(u[n, m] - want) < 1e-12
+
+
+def test_folded_weights_by_brute_force():
+    z = _fold_case()
+    n_h, d_h, d_cq = z["w_uq"].shape
+    d_c = z["w_uk"].shape[2]
+    d_model = z["w_o"].shape[0]
+    f = O.fold_q(z["w_uq"], z["w_uk"])
+    g = O.fold_o(z["w_o"], z["w_uv"])
+    assert f.shape == (n_h, d_c, d_cq) and g.shape == (d_model, n_h, d_c)
+    for i in range(n_h):
+        for c in range(d_c):
+            for d in range(d_cq):
+                want = sum(z["w_uk"][i, k, c] * z["w_uq"][i, k, d] for k in range(d_h))
+                assert abs(f[i, c, d] - want) < 1e-12
+            for m in range(d_model):
+                want = sum(z["w_o"][m, i, k] * z["w_uv"][i, k, c] for k in range(d_h))
+                assert abs(g[m, i, c] - want) < 1e-12
+
+
+def test_folded_projections_equal_the_two_step_products():
+    z = _fold_case(seed=11, n_h=4, d_h=8, d_c=16, d_cq=24, d_model=20, n_tok=5)
+    f = O.fold_q(z["w_uq"], z["w_uk"])
+    g = O.fold_o(z["w_o"], z["w_uv"])
+    two_step_q = O.absorb_q(O.q_up(z["c_q"], z["w_uq"]), z["w_uk"])
+    two_step_u = O.o_proj(O.up_v(z["lat"], z["w_uv"]), z["w_o"])
+    np.testing.assert_allclose(O.folded_q(z["c_q"], f), two_step_q, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(O.folded_o(z["lat"], g), two_step_u, rtol=1e-12, atol=1e-12)
