@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--workload", default="v2_decode")
     ap.add_argument("--kernel-impl", type=int, default=0, help="mla_config_t.impl (0 auto)")
     ap.add_argument("--max-splits", type=int, default=0)
+    ap.add_argument("--fold", action="store_true",
+                    help="the step with the folded projections: c^Q -> q_abs with W^UK folded into W^UQ, and "
+                         "latent -> u with W^UV folded into W^O (the model width)")
     ap.add_argument("--yarn", action="store_true",
                     help="YaRN-scaled RoPE on k^R (s = 40, alpha = 1, beta = 32, 4K training length) "
                          "and its attention temperature in the score scale")
@@ -274,6 +277,38 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     launches_decode = M.mla_decode_launches(dc.cfg, spec.B, spec.T_q, args.max_splits)
     launches_per_step = 3 + launches_decode       # absorb_q, rope_append, up_v + decode
+    fold = None
+    if args.fold:
+        # the folded weights, once (not timed), and the step's other ends: the
+        # query latent in, the model-width output out
+        def bits(a):
+            return torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)
+        fold = {"F": torch.empty((spec.n_h, spec.d_c, spec.d_cq), dtype=torch.bfloat16, device=dev),
+                "G": torch.empty((spec.d_model, spec.n_h, spec.d_c), dtype=torch.bfloat16, device=dev),
+                "h_c_q": spec.c_q()}
+        fold["c_q"] = bits(fold["h_c_q"])
+        fold["u"] = torch.empty((spec.n_tok, spec.d_model), dtype=torch.bfloat16, device=dev)
+        fold["ws"] = torch.zeros(M.mla_up_o_folded_workspace_bytes(dc.cfg, spec.d_model, spec.n_tok),
+                                 dtype=torch.uint8, device=dev)
+        M.mla_fold_weights(dc.cfg, spec.d_cq, spec.d_model, bits(spec.w_uq()), dc.w_uk, dc.w_uv, bits(spec.w_o()),
+                           fold["F"], fold["G"])
+        launches_per_step += 1                    # the output side adds its partials in a second kernel
+
+    def first_call(q_in, st=None):
+        if fold is None:
+            M.mla_absorb_q(dc.cfg, q_in, dc.w_uk, dc.q_abs, spec.n_tok, dc.status, st)
+        else:
+            M.mla_absorb_q_folded(dc.cfg, spec.d_cq, q_in, fold["F"], dc.q_abs, spec.n_tok, dc.status, st)
+
+    def last_call(out, st=None):
+        if fold is None:
+            M.mla_up_v(dc.cfg, dc.latent, dc.w_uv, out, spec.n_tok, dc.status, st)
+        else:
+            M.mla_up_o_folded(dc.cfg, spec.d_model, dc.latent, fold["G"], out, spec.n_tok, fold["ws"], dc.status,
+                              st)
+
+    q_in = dc.q_c if fold is None else fold["c_q"]
+    step_out = dc.out if fold is None else fold["u"]
 
     ranks = Ranks(pg, dev)
     barrier, max_over_ranks = ranks.barrier, ranks.max
@@ -281,7 +316,9 @@ def run_ours(args):
     # warm-up
     for _ in range(max(args.warmup, 3)):
         dc.reset_step_inputs()
-        dc.step()
+        first_call(q_in)
+        dc.step_middle()
+        last_call(step_out)
     torch.cuda.synchronize(dev)
     st = dc.decode_status() | dc.append_status()
     if st:
@@ -295,7 +332,7 @@ def run_ours(args):
         dc.q_r.copy_(dc.q_r_pre)
 
     def absorb():
-        M.mla_absorb_q(dc.cfg, dc.q_c, dc.w_uk, dc.q_abs, s.n_tok, dc.status)
+        first_call(q_in)
 
     def rope_append():
         M.mla_rope_append(dc.cfg, dc.q_r, dc.k_r_new, dc.c_kv_new, dc.positions, dc.rope_table,
@@ -303,7 +340,7 @@ def run_ours(args):
                           s.T_q, dc.status)
 
     def up_v():
-        M.mla_up_v(dc.cfg, dc.latent, dc.w_uv, dc.out, s.n_tok, dc.status)
+        last_call(step_out)
 
     # The device-timed passes replay the library calls from CUDA graphs
     # (captured from the same C-ABI calls), so that the host's enqueueing
@@ -356,7 +393,8 @@ def run_ours(args):
             evp[k][j + 1].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    names = ["absorb_q", "rope_append", "decode", "up_v"]
+    names = (["absorb_q", "rope_append", "decode", "up_v"] if fold is None else
+             ["absorb_q_folded", "rope_append", "decode", "up_o_folded"])
     phases = {n: [1e3 * e[j].elapsed_time(e[j + 1]) for e in evp] for j, n in enumerate(names)}
     phases_us = {n: sum(v) / K for n, v in phases.items()}
     phases_med_us = {n: statistics.median(v) for n, v in phases.items()}
@@ -375,8 +413,9 @@ def run_ours(args):
     # inputs and outputs are double-buffered and ordered by events.  No L2 flush runs
     # here (it would sit inside the timed region); the cache alone is larger
     # than L2.
+    h_q_in = dc.h_q_c if fold is None else fold["h_c_q"]
     parts = [a.view(np.uint8).reshape(-1) for a in
-             (dc.h_q_c, dc.h_q_r, dc.h_k_r_new, dc.h_c_kv_new, dc.h_positions)]
+             (h_q_in, dc.h_q_r, dc.h_k_r_new, dc.h_c_kv_new, dc.h_positions)]
     offs, tot = [], 0
     for a in parts:
         offs.append(tot)
@@ -385,14 +424,14 @@ def run_ours(args):
     for a, o in zip(parts, offs):
         h_stage[o:o + a.size].copy_(torch.from_numpy(a))
     d_stage = [torch.empty(tot, dtype=torch.uint8, device=dev) for _ in range(2)]
-    d_out = [torch.empty_like(dc.out) for _ in range(2)]
-    h_out = [torch.empty(dc.out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    d_out = [torch.empty_like(step_out) for _ in range(2)]
+    h_out = [torch.empty(step_out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
 
     def view(i, j, like):
         n = like.numel() * like.element_size()
         return d_stage[i][offs[j]:offs[j] + n].view(like.dtype).view(like.shape)
 
-    views = [tuple(view(i, j, t) for j, t in enumerate((dc.q_c, dc.q_r, dc.k_r_new, dc.c_kv_new, dc.positions)))
+    views = [tuple(view(i, j, t) for j, t in enumerate((q_in, dc.q_r, dc.k_r_new, dc.c_kv_new, dc.positions)))
              for i in range(2)]
     h2d = sum(a.size for a in parts)
     d2h = h_out[0].numel() * 2
@@ -427,12 +466,12 @@ def run_ours(args):
         stream.wait_event(ev_in[i])
         if k >= 2:
             stream.wait_event(ev_read[i])     # step k - 2's output has been read back
-        M.mla_absorb_q(dc.cfg, v_q_c, dc.w_uk, dc.q_abs, s.n_tok, dc.status, h_st)
+        first_call(v_q_c, h_st)
         M.mla_rope_append(dc.cfg, v_q_r, v_k_r, v_c_kv, v_pos, dc.rope_table, dc.max_pos, dc.block_table,
                           s.max_blocks, dc.pool, s.num_blocks, s.B, s.T_q, dc.status, h_st)
         M.mla_decode(dc.cfg, dc.q_abs, v_q_r, dc.pool, s.num_blocks, dc.block_table, s.max_blocks, dc.seq_lens,
                      s.B, s.T_q, dc.max_splits, dc.ws, dc.ws_bytes, dc.latent, dc.lse, h_st)
-        M.mla_up_v(dc.cfg, dc.latent, dc.w_uv, d_out[i], s.n_tok, dc.status, h_st)
+        last_call(d_out[i], h_st)
         ev_done[i].record(stream)
         s_down.wait_event(ev_done[i])
         cudart.cudaMemcpyAsync(h_out[i].data_ptr(), d_out[i].data_ptr(), d2h, 2, h_down)   # device -> host
@@ -465,6 +504,17 @@ def run_ours(args):
     roof["kernel"] = "mla_decode (decode + split merge)"
     roof["roofline_time_us"] = 1e6 * max(t_hbm, t_tc)
     roof["decode_us"] = decode_ms * 1e3
+    fold_line = None
+    if fold is not None:
+        # the folded products against the HBM peak: the weights once plus activations and outputs
+        n_tok = spec.n_tok
+        q_bytes = spec.n_h * spec.d_c * spec.d_cq * 2 + n_tok * spec.d_cq * 2 + n_tok * spec.n_h * spec.d_c * 2
+        o_bytes = spec.d_model * spec.n_h * spec.d_c * 2 + n_tok * spec.n_h * spec.d_c * 2 + n_tok * spec.d_model * 2
+        fold_line = {}
+        for key, nbytes, name in (("q", q_bytes, "absorb_q_folded"), ("o", o_bytes, "up_o_folded")):
+            t = phases_us[name] * 1e-6
+            fold_line[key] = {"us": phases_us[name], "bytes": nbytes, "achieved_gbs": nbytes / t / 1e9,
+                              "frac": nbytes / t / 1e9 / peaks["hbm_gbs"]}
 
     if rank != 0:
         if pg is not None:
@@ -486,8 +536,10 @@ def run_ours(args):
                    "d_c": spec.d_c, "d_r": spec.d_r, "block_size": spec.block_size,
                    "context": [int(spec.seq_lens.min()), int(spec.seq_lens.max())],
                    "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write)",
-                   "parallelism": f"replicas x{world}", "rope": "yarn" if args.yarn else "plain"},
+                   "parallelism": f"replicas x{world}", "rope": "yarn" if args.yarn else "plain",
+                   "projections": "folded" if fold is not None else "per head"},
         "phases_us": phases_us, "phases_median_us": phases_med_us,
+        **({"fold": fold_line} if fold_line is not None else {}),
         "timing": "device passes replay CUDA graphs of the C-ABI calls; e2e calls the API directly",
         "host_enqueue_us_per_step": 1e6 * host_s / K,
         "decode_hbm_tbs": hbm_gbs / 1e3, "decode_tflops": tflops,

@@ -269,6 +269,46 @@ int mla_decode_noalloc(const mla_config_t* cfg, const mla_bf16* q_abs, const mla
 int mla_up_v(const mla_config_t* cfg, const mla_bf16* latent, const mla_bf16* w_uv,
              mla_bf16* out, int n_tok, int32_t* dev_status, void* stream);
 
+/* Folded projections ([notes] "Key에 대한 수식 전개": the key up-projection
+ * folds into the query projection, W'^Q = (W^Q)^T W^UK; "Value에 대한 수식
+ * 전개": the value up-projection folds into the output projection,
+ * W'^O = W^O W^UV; [ru] "Идея 1").  With the query latent c^Q (d_cq columns,
+ * 1536 at DeepSeek-V2) and the model width d_model (5120 at DeepSeek-V2):
+ *   w_uq (n_h, d_h, d_cq): q^C[n, i, :] = w_uq[i] c_q[n]
+ *   w_o  (d_model, n_h, d_h): u[n] = sum_i w_o[:, i, :] o[n, i, :]
+ *   w_fold_q (n_h, d_c, d_cq): F_i = W^UK_i^T W^UQ_i
+ *   w_fold_o (d_model, n_h, d_c): G_i = W^O_i W^UV_i
+ * The fold multiplies the weight bytes a decode step reads (at DeepSeek-V2
+ * 3.0 x on the query side, 3.6 x on the output side); it pays only where
+ * the step is compute-bound.  All bf16, row-major, 16-byte aligned.
+ *
+ * mla_fold_weights: computes w_fold_q and/or w_fold_o (either may be null,
+ * not both; fp32 sums rounded to bf16, CUDA cores; once per weight set). */
+int mla_fold_weights(const mla_config_t* cfg, int d_cq, int d_model,
+                     const mla_bf16* w_uq, const mla_bf16* w_uk, const mla_bf16* w_uv,
+                     const mla_bf16* w_o, mla_bf16* w_fold_q, mla_bf16* w_fold_o, void* stream);
+
+/* q_abs[n, i, :] = F_i c_q[n] (the folded mla_absorb_q, from the query
+ * latent): c_q (n_tok, d_cq); q_abs (n_tok, n_h, d_c) as for mla_decode.
+ * tcgen05 kernels only: d_c a multiple of 128, d_cq of 64 (MLA_ERR_CONFIG
+ * otherwise).  dev_status as for mla_absorb_q. */
+int mla_absorb_q_folded(const mla_config_t* cfg, int d_cq, const mla_bf16* c_q,
+                        const mla_bf16* w_fold_q, mla_bf16* q_abs, int n_tok,
+                        int32_t* dev_status, void* stream);
+
+/* Bytes of workspace mla_up_o_folded needs (256-byte aligned pointer); 0 for
+ * invalid arguments. */
+size_t mla_up_o_folded_workspace_bytes(const mla_config_t* cfg, int d_model, int n_tok);
+
+/* u[n] = sum_i G_i latent[n, i, :] (the folded mla_up_v followed by the output
+ * projection): latent (n_tok, n_h, d_c) from mla_decode; u (n_tok, d_model).
+ * One product with K = n_h d_c, split over K; the fp32 partial sums go to the
+ * caller's workspace and are added by a second kernel.  tcgen05 kernels only:
+ * d_model a multiple of 128, n_h d_c of 64. */
+int mla_up_o_folded(const mla_config_t* cfg, int d_model, const mla_bf16* latent,
+                    const mla_bf16* w_fold_o, mla_bf16* u, int n_tok, void* workspace,
+                    size_t ws_bytes, int32_t* dev_status, void* stream);
+
 /* Zero a device status word (async on stream). */
 int mla_clear_status(int32_t* dev_status, void* stream);
 

@@ -29,6 +29,7 @@ EXPORTED = (
     "mla_yarn_score_scale", "mla_absorb_q",
     "mla_rope_append", "mla_decode_workspace_bytes", "mla_decode", "mla_decode_launches",
     "mla_decode_noalloc", "mla_decode_split_counts", "mla_test_arm_decode_timeout", "mla_up_v",
+    "mla_fold_weights", "mla_absorb_q_folded", "mla_up_o_folded_workspace_bytes", "mla_up_o_folded",
     "mla_clear_status", "mla_read_status",
 )
 
@@ -84,6 +85,11 @@ _lib.mla_decode_noalloc.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, 
 _lib.mla_decode_split_counts.argtypes = [_cfgp, _i, _i, _i, _vp, _vp, _i, _vp]
 _lib.mla_test_arm_decode_timeout.argtypes = [ctypes.c_uint64]
 _lib.mla_up_v.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp, _vp]
+_lib.mla_fold_weights.argtypes = [_cfgp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.mla_absorb_q_folded.argtypes = [_cfgp, _i, _vp, _vp, _vp, _i, _vp, _vp]
+_lib.mla_up_o_folded_workspace_bytes.restype = _sz
+_lib.mla_up_o_folded_workspace_bytes.argtypes = [_cfgp, _i, _i]
+_lib.mla_up_o_folded.argtypes = [_cfgp, _i, _vp, _vp, _vp, _i, _vp, _sz, _vp, _vp]
 _lib.mla_clear_status.argtypes = [_vp, _vp]
 _lib.mla_read_status.argtypes = [_vp, _vp, _vp]
 
@@ -204,6 +210,32 @@ def mla_test_arm_decode_timeout(wait_limit_ns: int):
 def mla_up_v(cfg: MlaConfig, latent, w_uv, out, n_tok: int, dev_status=None, stream=None):
     _check("mla_up_v", _lib.mla_up_v(ctypes.byref(cfg), _ptr(latent), _ptr(w_uv), _ptr(out),
                                      int(n_tok), _ptr(dev_status), _stream(stream)))
+
+
+def mla_fold_weights(cfg: MlaConfig, d_cq: int, d_model: int, w_uq, w_uk, w_uv, w_o, w_fold_q, w_fold_o,
+                     stream=None):
+    _check("mla_fold_weights", _lib.mla_fold_weights(
+        ctypes.byref(cfg), int(d_cq), int(d_model), _ptr(w_uq), _ptr(w_uk), _ptr(w_uv), _ptr(w_o),
+        _ptr(w_fold_q), _ptr(w_fold_o), _stream(stream)))
+
+
+def mla_absorb_q_folded(cfg: MlaConfig, d_cq: int, c_q, w_fold_q, q_abs, n_tok: int, dev_status=None,
+                        stream=None):
+    _check("mla_absorb_q_folded", _lib.mla_absorb_q_folded(
+        ctypes.byref(cfg), int(d_cq), _ptr(c_q), _ptr(w_fold_q), _ptr(q_abs), int(n_tok), _ptr(dev_status),
+        _stream(stream)))
+
+
+def mla_up_o_folded_workspace_bytes(cfg: MlaConfig, d_model: int, n_tok: int) -> int:
+    return int(_lib.mla_up_o_folded_workspace_bytes(ctypes.byref(cfg), int(d_model), int(n_tok)))
+
+
+def mla_up_o_folded(cfg: MlaConfig, d_model: int, latent, w_fold_o, u, n_tok: int, workspace, dev_status=None,
+                    stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("mla_up_o_folded", _lib.mla_up_o_folded(
+        ctypes.byref(cfg), int(d_model), _ptr(latent), _ptr(w_fold_o), _ptr(u), int(n_tok), _ptr(workspace),
+        ws_bytes, _ptr(dev_status), _stream(stream)))
 
 
 def mla_clear_status(dev_status, stream=None):

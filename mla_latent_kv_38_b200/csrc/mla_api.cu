@@ -10,6 +10,7 @@
 #include "kernels.h"
 #include "sm100_decode.h"
 #include "sm100_proj.h"
+#include "fold.h"
 
 namespace {
 
@@ -327,6 +328,56 @@ int mla_up_v(const mla_config_t* cfg, const mla_bf16* latent, const mla_bf16* w_
             mla::launch_up_v_sm100(latent, w_uv, out, n_tok, cfg->n_h, cfg->d_h, cfg->d_c, dev_status, st));
     }
     return cuda_rc(mla::launch_up_v_simt(latent, w_uv, out, n_tok, cfg->n_h, cfg->d_h, cfg->d_c, st));
+}
+
+int mla_fold_weights(const mla_config_t* cfg, int d_cq, int d_model, const mla_bf16* w_uq, const mla_bf16* w_uk,
+                     const mla_bf16* w_uv, const mla_bf16* w_o, mla_bf16* w_fold_q, mla_bf16* w_fold_o,
+                     void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!w_fold_q && !w_fold_o) return MLA_ERR_NULL;
+    if (w_fold_q && (!w_uq || !w_uk)) return MLA_ERR_NULL;
+    if (w_fold_o && (!w_uv || !w_o)) return MLA_ERR_NULL;
+    if (d_cq < 1 || d_cq > 65536 || d_model < 1 || d_model > 65536) return MLA_ERR_SIZE;
+    if (mla_check_device() != MLA_OK) return MLA_ERR_UNSUPPORTED;
+    return cuda_rc(mla::launch_fold_weights(w_uq, w_uk, w_uv, w_o, w_fold_q, w_fold_o, cfg->n_h, cfg->d_h, cfg->d_c,
+                                            d_cq, d_model, static_cast<cudaStream_t>(stream)));
+}
+
+int mla_absorb_q_folded(const mla_config_t* cfg, int d_cq, const mla_bf16* c_q, const mla_bf16* w_fold_q,
+                        mla_bf16* q_abs, int n_tok, int32_t* dev_status, void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!c_q || !w_fold_q || !q_abs) return MLA_ERR_NULL;
+    if (!aligned16(c_q) || !aligned16(w_fold_q) || !aligned16(q_abs)) return MLA_ERR_ALIGN;
+    if (dev_status && !aligned4(dev_status)) return MLA_ERR_ALIGN;
+    if (n_tok < 1 || n_tok > 65535 || d_cq < 64 || d_cq > 65536) return MLA_ERR_SIZE;
+    if (!mla::fold_q_supports(cfg->d_c, d_cq)) return MLA_ERR_CONFIG;
+    if (mla_check_device() != MLA_OK) return MLA_ERR_UNSUPPORTED;
+    return cuda_rc(mla::launch_q_folded(c_q, w_fold_q, q_abs, n_tok, cfg->n_h, cfg->d_c, d_cq, dev_status,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+size_t mla_up_o_folded_workspace_bytes(const mla_config_t* cfg, int d_model, int n_tok) {
+    if (check_config(cfg) || n_tok < 1 || n_tok > 65535 || d_model < 1) return 0;
+    if (!mla::fold_o_supports(cfg->n_h, cfg->d_c, d_model)) return 0;
+    return round256(mla::o_folded_workspace_bytes(cfg->n_h, cfg->d_c, d_model, n_tok));
+}
+
+int mla_up_o_folded(const mla_config_t* cfg, int d_model, const mla_bf16* latent, const mla_bf16* w_fold_o,
+                    mla_bf16* u, int n_tok, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!latent || !w_fold_o || !u || !workspace) return MLA_ERR_NULL;
+    if (!aligned16(latent) || !aligned16(w_fold_o) || !aligned16(u)) return MLA_ERR_ALIGN;
+    if (dev_status && !aligned4(dev_status)) return MLA_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLA_ERR_WORKSPACE;
+    if (n_tok < 1 || n_tok > 65535 || d_model < 1 || d_model > 65536) return MLA_ERR_SIZE;
+    if (!mla::fold_o_supports(cfg->n_h, cfg->d_c, d_model)) return MLA_ERR_CONFIG;
+    if (ws_bytes < mla::o_folded_workspace_bytes(cfg->n_h, cfg->d_c, d_model, n_tok)) return MLA_ERR_WORKSPACE;
+    if (mla_check_device() != MLA_OK) return MLA_ERR_UNSUPPORTED;
+    return cuda_rc(mla::launch_o_folded(latent, w_fold_o, u, n_tok, cfg->n_h, cfg->d_c, d_model, workspace,
+                                        dev_status, static_cast<cudaStream_t>(stream)));
 }
 
 int mla_clear_status(int32_t* dev_status, void* stream) {

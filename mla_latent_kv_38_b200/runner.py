@@ -118,13 +118,18 @@ class DeviceCase:
         """One pass of the whole hot path for the batch."""
         s = self.spec
         M.mla_absorb_q(self.cfg, self.q_c, self.w_uk, self.q_abs, s.n_tok, self.status, stream)
+        self.step_middle(stream)
+        M.mla_up_v(self.cfg, self.latent, self.w_uv, self.out, s.n_tok, self.status, stream)
+
+    def step_middle(self, stream=None):
+        """The step between the projections: RoPE + append, then the decode."""
+        s = self.spec
         M.mla_rope_append(self.cfg, self.q_r, self.k_r_new, self.c_kv_new, self.positions,
                           self.rope_table, self.max_pos, self.block_table, s.max_blocks, self.pool,
                           s.num_blocks, s.B, s.T_q, self.status, stream)
         M.mla_decode(self.cfg, self.q_abs, self.q_r, self.pool, s.num_blocks, self.block_table,
                      s.max_blocks, self.seq_lens, s.B, s.T_q, self.max_splits, self.ws,
                      self.ws_bytes, self.latent, self.lse, stream)
-        M.mla_up_v(self.cfg, self.latent, self.w_uv, self.out, s.n_tok, self.status, stream)
 
     def decode_only(self, stream=None):
         s = self.spec
