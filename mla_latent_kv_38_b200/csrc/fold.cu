@@ -152,6 +152,7 @@ constexpr int kRows = 128;                 // A rows per CTA (MMA M)
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint32_t kABytes = kRows * 128;  // one 64-column chunk of 128 rows (16 KB)
 constexpr size_t kRingLimit = 200 * 1024;
+constexpr int kMaxStages = 4;                 // two CTAs an SM at decode token counts
 
 struct KGemm {
     CUtensorMap tm_a;      // A [rows][K] bf16, boxes 64 x 128
@@ -359,12 +360,12 @@ int token_tile(int n_tok) {
     return want < 256 ? want : 256;
 }
 
-// As many stages as fit (at most 8; at least 2), leaving the first stage's
+// As many stages as fit (at most kMaxStages; at least 2), leaving the first stage's
 // bytes for the output tile (bf16: nt x 256 B, fp32: nt x 512 B).
 int ring_stages(int nt, bool f32_out) {
     const size_t stage = kABytes + static_cast<size_t>(nt) * 128;
     int s = static_cast<int>(kRingLimit / stage);
-    if (s > 8) s = 8;
+    if (s > kMaxStages) s = kMaxStages;
     const size_t out_bytes = static_cast<size_t>(nt) * (f32_out ? 512 : 256);
     while (static_cast<size_t>(s) * stage < out_bytes) ++s;
     return s < 2 ? 2 : s;
