@@ -20,7 +20,8 @@
 // shared memory and runs every token tile of its head against it.  One thread
 // issues the MMAs (cta_group::1, M = 128, N = token tile <= 256) into tensor
 // memory; four warps read the fp32 accumulator back (one TMEM lane per thread,
-// i.e. one output feature per thread) and store it as bf16.
+// i.e. one output feature per thread) into a bf16 tile in shared memory that
+// TMA bulk tensor stores write out.
 
 #include <cuda.h>
 
