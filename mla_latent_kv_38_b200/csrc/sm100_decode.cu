@@ -103,6 +103,7 @@ static_assert(4 * (5 * kInKernelUnits + 3 + kClusters + 1 + 48) <= static_cast<i
 static_assert(4 * (kClusters + 1) <= 320, "cut area");
 static_assert(kSRing % kSLaneGroups == 0, "each lane group keeps its own ring slots");
 static_assert(4 * kSLaneGroups <= 32, "lane groups of the S producer warp");
+static_assert(8 * 16384 <= kOffP, "the last epilogue's staging (16 KB per softmax warp) lies in the rings");
 
 enum {
     BAR_SR_FULL = 0,                         // + slot (leader: both CTAs' bytes)
@@ -987,16 +988,21 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                 const size_t grow = static_cast<size_t>(bt) * p.n_h + hb * 128 + head_in_unit;
                 const size_t slot = static_cast<size_t>(cluster) + t.u;
                 // This warp's 32 rows (consecutive heads) x the thread's 128
-                // latent columns go out through a 4 KB tile of the free P buffer,
-                // written in the 128-byte swizzled layout of a TMA store box (a
-                // thread's row of 128 bytes, 16-byte chunk k at k ^ (row & 7)),
-                // so each round is one bulk tensor store: 4 rounds of 32 fp32
-                // columns for a partial, 2 rounds of 64 bf16 columns otherwise.
+                // latent columns go out through 4 KB tiles written in the
+                // 128-byte swizzled layout of a TMA store box (a thread's row of
+                // 128 bytes, 16-byte chunk k at k ^ (row & 7)), each tile one
+                // bulk tensor store: 4 stores of 32 fp32 columns for a partial,
+                // 2 of 64 bf16 columns otherwise.  Between tiles the staging is
+                // one 4 KB tile of the free P buffer per warp, reused store
+                // after store; after the CTA's last tile no load or MMA touches
+                // the rings any more, so every store gets its own tile there
+                // and none waits for the one before.
+                const bool final_tile = w.done();
                 const int h = cg;   // this thread's 128 O columns
                 const int col0 = 128 * h + (hi ? 256 : 0);
-                unsigned char* stage = smem + kOffP + sw * 4096;
-                const uint32_t stage_u = sbase + kOffP + sw * 4096;
-                unsigned char* my_row = stage + lane * 128;
+                const uint32_t stage_off = final_tile ? kOffSRing + sw * 16384u : kOffP + sw * 4096u;
+                unsigned char* stage = smem + stage_off;
+                const uint32_t stage_u = sbase + stage_off;
                 const int x7 = lane & 7;
                 const int row0 = whole ? static_cast<int>(grow - lane)
                                        : static_cast<int>(slot * 128 + head_in_unit - lane);
@@ -1005,7 +1011,10 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                     uint32_t o[32];
                     ptx::tmem_ld32(t_lane + kTmemO + 128 * h + 32 * q, o);
                     ptx::tmem_wait_ld();
-                    if (!whole || (q & 1) == 0) {
+                    const int tile_k = whole ? (q >> 1) : q;   // this round's store
+                    const uint32_t tile_off = final_tile ? 4096u * tile_k : 0u;
+                    unsigned char* my_row = stage + tile_off + lane * 128;
+                    if (!final_tile && (!whole || (q & 1) == 0)) {
                         if (lane == 0) ptx::bulk_wait_read_all();   // the previous store has read the tile
                         __syncwarp();
                     }
@@ -1024,7 +1033,7 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                             ptx::fence_proxy_async_smem();
                             __syncwarp();
                             if (lane == 0) {
-                                ptx::tma_store_2d(&p.tm_out, stage_u, col0 + 64 * (q >> 1), row0);
+                                ptx::tma_store_2d(&p.tm_out, stage_u + tile_off, col0 + 64 * (q >> 1), row0);
                                 ptx::bulk_commit_group();
                             }
                         }
@@ -1037,13 +1046,15 @@ mla_decode_sm100_kernel(const __grid_constant__ Sm100Params p) {
                         ptx::fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            ptx::tma_store_2d(&p.tm_part, stage_u, col0 + 32 * q, row0);
+                            ptx::tma_store_2d(&p.tm_part, stage_u + tile_off, col0 + 32 * q, row0);
                             ptx::bulk_commit_group();
                         }
                     }
                 }
-                if (lane == 0) ptx::bulk_wait_read_all();   // the P buffer is written again by the next tile
-                __syncwarp();
+                if (!final_tile) {
+                    if (lane == 0) ptx::bulk_wait_read_all();   // the P buffer is written again by the next tile
+                    __syncwarp();
+                }
                 if (!hi && cg == 0) {
                     if (whole) p.out_lse[grow] = lse;
                     else p.part_lse[slot * 128 + head_in_unit] = lse;
@@ -1159,17 +1170,17 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, 
 // The partial rows were written by the decode kernel just before and are read
 // from L2 (ld.global.cg).  The first two slots' rows are fetched together with
 // the log-sum-exps, so that a row split in two takes two dependent round trips
-// (metadata, then everything else); further slots follow two at a time.  At
-// most 64 registers a thread: 8 warps of every SM's 4 blocks are resident at
-// once, one wave for the 4,096 rows of 32 split units.
-__global__ void __launch_bounds__(256, 4)
+// (metadata, then everything else); further slots follow two at a time.
+// Blocks of 4 warps, 7 per SM (up to 72 registers a thread, no spills): the
+// 4,096 rows of 32 split units are 1,024 blocks, one wave on 148 SMs.
+__global__ void __launch_bounds__(128, 7)
 mla_sm100_merge_kernel(const int4* __restrict__ unit_meta, const float* __restrict__ part_o,
                        const float* __restrict__ part_lse, uint16_t* __restrict__ out_latent,
                        float* __restrict__ out_lse, int n_h, int n_hb, int B, int T_q, int U) {
     griddep_launch_dependents();
     griddep_wait();
     const int lane = threadIdx.x & 31;
-    const int wg = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int wg = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int u = wg >> 7, row = wg & 127;
     if (u >= U) return;
     const int4 meta = unit_meta[u];
@@ -1350,7 +1361,7 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int max_splits,
     e = launch_pdl(mla_decode_sm100_kernel, dim3(2 * kClusters), dim3(kThreads), kSmemBytes, stream, k);
     if (e != cudaSuccess) return e;
     const int rows = U * 128;
-    return launch_pdl(mla_sm100_merge_kernel, dim3((rows + 7) / 8), dim3(256), 0, stream,
+    return launch_pdl(mla_sm100_merge_kernel, dim3((rows + 3) / 4), dim3(128), 0, stream,
                       static_cast<const int4*>(k.unit_meta), static_cast<const float*>(k.part_o),
                       static_cast<const float*>(k.part_lse), P.out_latent, P.out_lse, P.n_h, n_hb, P.B, P.T_q, U);
 }

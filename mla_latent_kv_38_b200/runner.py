@@ -2,7 +2,7 @@
 
 :class:`DeviceCase` allocates a workload's buffers with torch, fills the paged
 latent cache with the history rows (through ``mla_rope_append``), and runs the
-step ``mla_absorb_q -> mla_rope_append -> mla_decode -> mla_up_v``.  Used by
+step ``mla_rope_append -> mla_absorb_q -> mla_decode -> mla_up_v``.  Used by
 the GPU tests, the benchmark and the smoke check.
 """
 
@@ -115,21 +115,23 @@ class DeviceCase:
         self.q_r.copy_(self.q_r_pre)
 
     def step(self, stream=None):
-        """One pass of the whole hot path for the batch."""
+        """One pass of the whole hot path for the batch.
+
+        RoPE + append and the query absorption read disjoint inputs, so either
+        may go first; the append goes first: the absorption's CTAs then start
+        while it runs and fetch their weight tiles before they wait for it."""
         s = self.spec
+        self.rope_append(stream)
         M.mla_absorb_q(self.cfg, self.q_c, self.w_uk, self.q_abs, s.n_tok, self.status, stream)
-        self.step_middle(stream)
+        self.decode_only(stream)
         M.mla_up_v(self.cfg, self.latent, self.w_uv, self.out, s.n_tok, self.status, stream)
 
-    def step_middle(self, stream=None):
-        """The step between the projections: RoPE + append, then the decode."""
+    def rope_append(self, stream=None):
+        """RoPE on q^R in place and the new cache rows appended."""
         s = self.spec
         M.mla_rope_append(self.cfg, self.q_r, self.k_r_new, self.c_kv_new, self.positions,
                           self.rope_table, self.max_pos, self.block_table, s.max_blocks, self.pool,
                           s.num_blocks, s.B, s.T_q, self.status, stream)
-        M.mla_decode(self.cfg, self.q_abs, self.q_r, self.pool, s.num_blocks, self.block_table,
-                     s.max_blocks, self.seq_lens, s.B, s.T_q, self.max_splits, self.ws,
-                     self.ws_bytes, self.latent, self.lse, stream)
 
     def decode_only(self, stream=None):
         s = self.spec
