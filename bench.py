@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MLA decode tokens/s + achieved HBM TB/s & TFLOP/s vs roofline (1×B200)"
 L2_FLUSH_BYTES = 256 << 20
+ALU_CLOCK_GHZ = 1.965   # B200 clocks.max.sm
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -47,6 +48,8 @@ def parse():
     ap.add_argument("--fold", action="store_true",
                     help="the step with the folded projections: c^Q -> q_abs with W^UK folded into W^UQ, and "
                          "latent -> u with W^UV folded into W^O (the model width)")
+    ap.add_argument("--cache", choices=["bf16", "e4m3"], default="bf16",
+                    help="latent cache format: bf16 rows, or the low-bit e4m3 rows (portable decode kernel)")
     ap.add_argument("--yarn", action="store_true",
                     help="YaRN-scaled RoPE on k^R (s = 40, alpha = 1, beta = 32, 4K training length) "
                          "and its attention temperature in the score scale")
@@ -160,16 +163,16 @@ class ClockSampler:
 YARN = dict(s=40.0, alpha=1.0, beta=32.0, orig_len=4096, coeff=0.0707)
 
 
-def oracle_sample_rate(spec, steps, warmup, heads_per_step=8, budget_s=None, yarn=False):
+def oracle_sample_rate(spec, steps, warmup, heads_per_step=8, budget_s=None, yarn=False, cache="bf16"):
     """Time the fp64 oracle on `heads_per_step` heads of one sequence per step.
 
     Returns (tokens/s, seconds, description).  A token's output needs all n_h
     heads, so a step credits heads_per_step / n_h of each of its T_q tokens."""
     from oracle.evaluate import reference
-    kw = {}
+    kw = {"cache": cache}
     if yarn:
         from oracle import mla_oracle as O
-        kw = dict(inv_freq=O.yarn_inv_freq(spec.d_r, s=YARN["s"], alpha=YARN["alpha"], beta=YARN["beta"],
+        kw.update(inv_freq=O.yarn_inv_freq(spec.d_r, s=YARN["s"], alpha=YARN["alpha"], beta=YARN["beta"],
                                            orig_len=YARN["orig_len"]),
                   scale=O.yarn_score_scale(spec.d_h, spec.d_r, s=YARN["s"], coeff=YARN["coeff"]))
     b = 0
@@ -208,13 +211,13 @@ def run_reference(args):
         return 0
     from mla_latent_kv_38_b200.workloads import workload_specs
     spec = workload_specs()[args.workload]
-    rate, secs, desc = oracle_sample_rate(spec, args.steps, args.warmup, yarn=args.yarn)
+    rate, secs, desc = oracle_sample_rate(spec, args.steps, args.warmup, yarn=args.yarn, cache=args.cache)
     line = {
         "metric": METRIC, "impl": "reference", "value": rate, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * secs / max(args.steps, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": spec.name, "rope": "yarn" if args.yarn else "plain"},
+        "config": {"workload": spec.name, "rope": "yarn" if args.yarn else "plain", "cache": args.cache},
         "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -272,10 +275,14 @@ def run_ours(args):
 
     spec = workload_specs()[args.workload]
     dc = DeviceCase(spec, impl=args.kernel_impl, max_splits=args.max_splits, device=f"cuda:{local}",
-                    yarn=YARN if args.yarn else None)
+                    yarn=YARN if args.yarn else None, cache=args.cache)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    launches_decode = M.mla_decode_launches(dc.cfg, spec.B, spec.T_q, args.max_splits)
+    if args.cache == "bf16":
+        launches_decode = M.mla_decode_launches(dc.cfg, spec.B, spec.T_q, args.max_splits)
+    else:   # the portable kernel (and its merge when the rows are split)
+        portable = M.MlaConfig(spec.n_h, spec.d_c, spec.d_h, spec.d_r, spec.block_size, dc.cfg.scale, M.IMPL_SIMT)
+        launches_decode = M.mla_decode_launches(portable, spec.B, spec.T_q, args.max_splits)
     launches_per_step = 3 + launches_decode       # absorb_q, rope_append, up_v + decode
     fold = None
     if args.fold:
@@ -336,9 +343,7 @@ def run_ours(args):
         first_call(q_in)
 
     def rope_append():
-        M.mla_rope_append(dc.cfg, dc.q_r, dc.k_r_new, dc.c_kv_new, dc.positions, dc.rope_table,
-                          dc.max_pos, dc.block_table, s.max_blocks, dc.pool, s.num_blocks, s.B,
-                          s.T_q, dc.status)
+        dc.rope_append()
 
     def up_v():
         last_call(step_out)
@@ -453,6 +458,8 @@ def run_ours(args):
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
     ev_read = [torch.cuda.Event() for _ in range(2)]
+    append_fn = M.mla_rope_append if args.cache == "bf16" else M.mla_rope_append_e4m3
+    decode_fn = M.mla_decode if args.cache == "bf16" else M.mla_decode_e4m3
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
     barrier()
@@ -469,11 +476,11 @@ def run_ours(args):
         stream.wait_event(ev_in[i])
         if k >= 2:
             stream.wait_event(ev_read[i])     # step k - 2's output has been read back
-        M.mla_rope_append(dc.cfg, v_q_r, v_k_r, v_c_kv, v_pos, dc.rope_table, dc.max_pos, dc.block_table,
-                          s.max_blocks, dc.pool, s.num_blocks, s.B, s.T_q, dc.status, h_st)
+        append_fn(dc.cfg, v_q_r, v_k_r, v_c_kv, v_pos, dc.rope_table, dc.max_pos, dc.block_table,
+                  s.max_blocks, dc.pool, s.num_blocks, s.B, s.T_q, dc.status, h_st)
         first_call(v_q_c, h_st)
-        M.mla_decode(dc.cfg, dc.q_abs, v_q_r, dc.pool, s.num_blocks, dc.block_table, s.max_blocks, dc.seq_lens,
-                     s.B, s.T_q, dc.max_splits, dc.ws, dc.ws_bytes, dc.latent, dc.lse, h_st)
+        decode_fn(dc.cfg, dc.q_abs, v_q_r, dc.pool, s.num_blocks, dc.block_table, s.max_blocks, dc.seq_lens,
+                  s.B, s.T_q, dc.max_splits, dc.ws, dc.ws_bytes, dc.latent, dc.lse, h_st)
         last_call(d_out[i], h_st)
         ev_done[i].record(stream)
         s_down.wait_event(ev_done[i])
@@ -487,7 +494,8 @@ def run_ours(args):
     e2e_value = aggregate_rate(world, tokens_per_step, K, e2e_ms)
 
     peaks, peak_src = load_peaks()
-    bytes_alg = spec.algorithmic_bytes()
+    row_bytes = None if args.cache == "bf16" else M.mla_e4m3_row_bytes(spec.d_c, spec.d_r)
+    bytes_alg = spec.algorithmic_bytes(row_bytes=row_bytes)
     flops_alg = spec.algorithmic_flops()
     dec_s = decode_ms / 1e3
     hbm_gbs = bytes_alg / dec_s / 1e9
@@ -495,16 +503,25 @@ def run_ours(args):
     t_hbm = bytes_alg / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops_alg / (peaks["bf16_tflops"] * 1e12)
     bound = "hbm" if t_hbm >= t_tc else "tensor"
-    if bound == "hbm":
+    if args.cache == "e4m3":
+        # the portable kernel: float32 FMAs on the CUDA cores, 148 SMs x 128
+        # lanes x 2 FLOP per cycle at the highest SM clock
+        alu_tflops = 148 * 128 * 2 * ALU_CLOCK_GHZ / 1e3
+        t_alu = flops_alg / (alu_tflops * 1e12)
+        roof = {"bound": "alu", "achieved": tflops, "peak": alu_tflops, "unit": "TFLOP/s",
+                "frac": tflops / alu_tflops, "hbm_frac": hbm_gbs / peaks["hbm_gbs"]}
+        t_tc = max(t_tc, t_alu)
+    elif bound == "hbm":
         roof = {"bound": "hbm", "achieved": hbm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": hbm_gbs / peaks["hbm_gbs"]}
     else:
         roof = {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"]}
     khash = decode_source_hash()
-    roof["traffic"] = profiled_traffic(args.workload, khash)
+    roof["traffic"] = profiled_traffic(args.workload, khash) if args.cache == "bf16" else None
     roof["peak_source"] = f"MEASURED_PEAKS.json ({peak_src})"
-    roof["kernel"] = "mla_decode (decode + split merge)"
+    roof["kernel"] = ("mla_decode (decode + split merge)" if args.cache == "bf16" else
+                      "mla_decode_e4m3 (portable decode + split merge)")
     roof["roofline_time_us"] = 1e6 * max(t_hbm, t_tc)
     roof["decode_us"] = decode_ms * 1e3
     fold_line = None
@@ -526,7 +543,8 @@ def run_ours(args):
 
     cpu = None
     if world == 1:
-        rate, secs, desc = oracle_sample_rate(spec, steps=4, warmup=1, budget_s=20.0, yarn=args.yarn)
+        rate, secs, desc = oracle_sample_rate(spec, steps=4, warmup=1, budget_s=20.0, yarn=args.yarn,
+                                              cache=args.cache)
         cpu = {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": desc}
 
@@ -534,13 +552,14 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": step_ms / K,
         "ms_per_step_median": statistics.median(step_each), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if args.cache == "bf16" else "f32",
+        "data": "synthetic",
         "config": {"workload": spec.name, "B": spec.B, "T_q": spec.T_q, "n_h": spec.n_h,
                    "d_c": spec.d_c, "d_r": spec.d_r, "block_size": spec.block_size,
                    "context": [int(spec.seq_lens.min()), int(spec.seq_lens.max())],
                    "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write)",
                    "parallelism": f"replicas x{world}", "rope": "yarn" if args.yarn else "plain",
-                   "projections": "folded" if fold is not None else "per head"},
+                   "projections": "folded" if fold is not None else "per head", "cache": args.cache},
         "phases_us": phases_us, "phases_median_us": phases_med_us,
         **({"fold": fold_line} if fold_line is not None else {}),
         "timing": "device passes replay CUDA graphs of the C-ABI calls; e2e calls the API directly",

@@ -309,6 +309,58 @@ int mla_up_o_folded(const mla_config_t* cfg, int d_model, const mla_bf16* latent
                     const mla_bf16* w_fold_o, mla_bf16* u, int n_tok, void* workspace,
                     size_t ws_bytes, int32_t* dev_status, void* stream);
 
+/* ---- Low-bit latent cache ------------------------------------------------
+ * The pages quote a KV cache of about 6 bits per element for the served model
+ * ("DeepSeek-V2 review", 4.2 Evaluation, "Inference efficiency"; [ru]
+ * "Откуда берутся 93,3%") and give no format.  This library's format: the
+ * latent c^KV as OCP FP8 E4M3 codes with one float32 scale per
+ * MLA_E4M3_GROUP latent columns; the rotated RoPE key k^R stays bf16 (its
+ * rotation carries the position, [ru] "Идея 2").  One cache row, bytes:
+ *   [0, d_c)                          e4m3 codes of c^KV
+ *   [S, S + 4 d_c / 64)               float32 scales,  S = d_c rounded up to 16
+ *   [R, R + 2 d_r)                    bf16 RoPE key,   R = end of the scales
+ *                                                        rounded up to 16
+ *   padding to mla_e4m3_row_bytes(d_c, d_r) (a multiple of 16), zero.
+ * At DeepSeek-V2 (d_c 512, d_r 64) a row is 672 bytes against 1,152 in bf16.
+ * Quantisation of a group x (the bf16 latent values as float32): amax =
+ * max |x|; inv = 448 / amax and scale = amax / 448 (float32 divisions,
+ * round to nearest even); code = e4m3(x * inv) (float32 product, then round
+ * to nearest even with saturation at +-448).  amax = 0 stores scale 0 and
+ * zero codes.  A cached value reads back as e4m3(code) * scale.  Inputs must
+ * be finite.  Pool: (num_blocks, block_size, mla_e4m3_row_bytes) bytes,
+ * 16-byte aligned.  Shapes: d_c a multiple of 64 (MLA_ERR_CONFIG otherwise). */
+#define MLA_E4M3_GROUP 64
+
+/* Bytes of one cache row in the e4m3 format; 0 for an unsupported shape. */
+size_t mla_e4m3_row_bytes(int d_c, int d_r);
+
+/* mla_rope_append into an e4m3 pool: the same RoPE of q^R (in place) and
+ * k^R, the same positions, block table and status bits; the appended row is
+ * the quantised latent, its scales and the rotated bf16 key. */
+int mla_rope_append_e4m3(const mla_config_t* cfg, mla_bf16* q_r, const mla_bf16* k_r,
+                         const mla_bf16* c_kv, const int32_t* positions,
+                         const float* rope_table, int max_pos,
+                         const int32_t* block_table, int max_blocks_per_seq,
+                         uint8_t* pool, int num_blocks, int B, int T_q,
+                         int32_t* dev_status, void* stream);
+
+/* Workspace bytes of mla_decode_e4m3 (256-byte aligned pointer required);
+ * 0 for invalid arguments. */
+size_t mla_decode_e4m3_workspace_bytes(const mla_config_t* cfg, int B, int T_q, int max_splits);
+
+/* mla_decode over an e4m3 pool: the same scores, mask, softmax, outputs and
+ * size limits, with every cached latent value read back as e4m3(code) *
+ * scale (in float32) and the key's RoPE part as stored.  Runs the portable
+ * CUDA-core decode kernel (cfg->impl 0 or 1; 2 returns MLA_ERR_CONFIG) with
+ * exactly max_splits key-range parts per query row (0: a count from B, T_q,
+ * n_h), merged by the log-sum-exp reduction.  The workspace starts with the
+ * device status word. */
+int mla_decode_e4m3(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q_r,
+                    const uint8_t* pool, int num_blocks, const int32_t* block_table,
+                    int max_blocks_per_seq, const int32_t* seq_lens, int B, int T_q,
+                    int max_splits, void* workspace, size_t ws_bytes,
+                    mla_bf16* out_latent, float* out_lse, void* stream);
+
 /* Zero a device status word (async on stream). */
 int mla_clear_status(int32_t* dev_status, void* stream);
 

@@ -30,6 +30,7 @@ EXPORTED = (
     "mla_rope_append", "mla_decode_workspace_bytes", "mla_decode", "mla_decode_launches",
     "mla_decode_noalloc", "mla_decode_split_counts", "mla_test_arm_decode_timeout", "mla_up_v",
     "mla_fold_weights", "mla_absorb_q_folded", "mla_up_o_folded_workspace_bytes", "mla_up_o_folded",
+    "mla_e4m3_row_bytes", "mla_rope_append_e4m3", "mla_decode_e4m3_workspace_bytes", "mla_decode_e4m3",
     "mla_clear_status", "mla_read_status",
 )
 
@@ -90,6 +91,12 @@ _lib.mla_absorb_q_folded.argtypes = [_cfgp, _i, _vp, _vp, _vp, _i, _vp, _vp]
 _lib.mla_up_o_folded_workspace_bytes.restype = _sz
 _lib.mla_up_o_folded_workspace_bytes.argtypes = [_cfgp, _i, _i]
 _lib.mla_up_o_folded.argtypes = [_cfgp, _i, _vp, _vp, _vp, _i, _vp, _sz, _vp, _vp]
+_lib.mla_e4m3_row_bytes.restype = _sz
+_lib.mla_e4m3_row_bytes.argtypes = [_i, _i]
+_lib.mla_rope_append_e4m3.argtypes = [_cfgp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, _vp, _vp]
+_lib.mla_decode_e4m3_workspace_bytes.restype = _sz
+_lib.mla_decode_e4m3_workspace_bytes.argtypes = [_cfgp, _i, _i, _i]
+_lib.mla_decode_e4m3.argtypes = [_cfgp, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, _vp, _sz, _vp, _vp, _vp]
 _lib.mla_clear_status.argtypes = [_vp, _vp]
 _lib.mla_read_status.argtypes = [_vp, _vp, _vp]
 
@@ -236,6 +243,32 @@ def mla_up_o_folded(cfg: MlaConfig, d_model: int, latent, w_fold_o, u, n_tok: in
     _check("mla_up_o_folded", _lib.mla_up_o_folded(
         ctypes.byref(cfg), int(d_model), _ptr(latent), _ptr(w_fold_o), _ptr(u), int(n_tok), _ptr(workspace),
         ws_bytes, _ptr(dev_status), _stream(stream)))
+
+
+def mla_e4m3_row_bytes(d_c: int, d_r: int) -> int:
+    return int(_lib.mla_e4m3_row_bytes(int(d_c), int(d_r)))
+
+
+def mla_rope_append_e4m3(cfg: MlaConfig, q_r, k_r, c_kv, positions, rope_table, max_pos: int,
+                         block_table, max_blocks_per_seq: int, pool, num_blocks: int, B: int, T_q: int,
+                         dev_status=None, stream=None):
+    _check("mla_rope_append_e4m3", _lib.mla_rope_append_e4m3(
+        ctypes.byref(cfg), _ptr(q_r), _ptr(k_r), _ptr(c_kv), _ptr(positions), _ptr(rope_table),
+        int(max_pos), _ptr(block_table), int(max_blocks_per_seq), _ptr(pool), int(num_blocks),
+        int(B), int(T_q), _ptr(dev_status), _stream(stream)))
+
+
+def mla_decode_e4m3_workspace_bytes(cfg: MlaConfig, B: int, T_q: int, max_splits: int = 0) -> int:
+    return int(_lib.mla_decode_e4m3_workspace_bytes(ctypes.byref(cfg), int(B), int(T_q), int(max_splits)))
+
+
+def mla_decode_e4m3(cfg: MlaConfig, q_abs, q_r, pool, num_blocks: int, block_table,
+                    max_blocks_per_seq: int, seq_lens, B: int, T_q: int, max_splits: int,
+                    workspace, ws_bytes: int, out_latent, out_lse, stream=None):
+    _check("mla_decode_e4m3", _lib.mla_decode_e4m3(
+        ctypes.byref(cfg), _ptr(q_abs), _ptr(q_r), _ptr(pool), int(num_blocks), _ptr(block_table),
+        int(max_blocks_per_seq), _ptr(seq_lens), int(B), int(T_q), int(max_splits), _ptr(workspace),
+        int(ws_bytes), _ptr(out_latent), _ptr(out_lse), _stream(stream)))
 
 
 def mla_clear_status(dev_status, stream=None):

@@ -39,6 +39,38 @@ __device__ __forceinline__ void unpack8(const uint4& v, float* f) {
     }
 }
 
+// Two float32 values -> two OCP FP8 E4M3 codes (round to nearest even,
+// saturating at +-448); lo in the low byte.
+__device__ __forceinline__ uint16_t e4m3x2_from_f32(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two E4M3 codes (low byte first) -> their values as float32 (exact).
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint16_t codes) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(codes));
+    float lo, hi;
+    asm("{\n\t.reg .f16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+        : "=f"(lo), "=f"(hi) : "r"(h));
+    return make_float2(lo, hi);
+}
+
+// Byte offsets of one e4m3 cache row (layout in include/mla.h): the group
+// scales, the bf16 RoPE key, and the row's size.
+struct E4m3Row {
+    int scale_off, kr_off, bytes;
+};
+
+__host__ __device__ __forceinline__ E4m3Row e4m3_row(int d_c, int d_r) {
+    E4m3Row r;
+    r.scale_off = (d_c + 15) / 16 * 16;
+    r.kr_off = (r.scale_off + 4 * (d_c / MLA_E4M3_GROUP) + 15) / 16 * 16;
+    r.bytes = (r.kr_off + 2 * d_r + 15) / 16 * 16;
+    return r;
+}
+
 // 2^x on the special-function unit (PTX ex2.approx; 2^-inf = +0)
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -111,6 +143,7 @@ struct DecodeParams {
     const uint16_t* q_abs;      // (n_tok, n_h, d_c)
     const uint16_t* q_r;        // (n_tok, n_h, d_r)
     const uint16_t* pool;       // (num_blocks, block_size, d_c + d_r)
+    const uint8_t* pool8 = nullptr;   // e4m3 pool (portable kernel only), else null
     const int32_t* block_table; // (B, max_blocks)
     const int32_t* seq_lens;    // (B)
     uint16_t* out_latent;       // (n_tok, n_h, d_c)

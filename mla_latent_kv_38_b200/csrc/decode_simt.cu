@@ -11,6 +11,10 @@
 // Layout of the work: grid (split, token, head group of 8).  Each warp owns one
 // head; the 8 warps share each 32-row key tile staged in shared memory with
 // 16-byte loads.  Online softmax in the exp2 domain.
+//
+// With an e4m3 pool (the low-bit cache of include/mla.h) the tile is staged as
+// float32: each latent value is e4m3(code) * its group's scale, the RoPE key
+// is widened from bf16; the rest of the kernel is the same.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -20,13 +24,31 @@ namespace mla {
 constexpr int kSimtHeads = 8;
 constexpr int kSimtKeys = 32;
 
+// Eight consecutive values of staged key row `row` from value 8 v on.
+template <bool kE4m3>
+__device__ __forceinline__ void load8(const unsigned char* tile, int row_stride, int row, int v, float* f) {
+    if constexpr (kE4m3) {
+        const float4* p = reinterpret_cast<const float4*>(tile + static_cast<size_t>(row) * row_stride) + 2 * v;
+        const float4 a = p[0], b = p[1];
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    } else {
+        unpack8(reinterpret_cast<const uint4*>(tile + static_cast<size_t>(row) * row_stride)[v], f);
+    }
+}
+
+// Bytes of one staged key row: bf16 values plus 16 bytes, or float32 values
+// plus 16 bytes (the padding spreads the rows over the shared-memory banks).
+__host__ __device__ __forceinline__ int staged_row_bytes(int D, bool e4m3) { return (e4m3 ? 4 : 2) * D + 16; }
+
+template <bool kE4m3>
 __global__ void __launch_bounds__(256)
 decode_simt_kernel(DecodeParams P) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int D = P.d_c + P.d_r;
-    const int row_vec = D / 8 + 1;                       // padded row, in uint4
-    uint4* Ks = reinterpret_cast<uint4*>(smem_raw);      // [32][row_vec]
-    float* Qs = reinterpret_cast<float*>(Ks + kSimtKeys * row_vec);  // [8][D]
+    const int row_bytes = staged_row_bytes(D, kE4m3);
+    unsigned char* tile = smem_raw;                                          // [32][row_bytes]
+    float* Qs = reinterpret_cast<float*>(smem_raw + kSimtKeys * row_bytes);  // [8][D]
 
     const int split = blockIdx.x, n = blockIdx.y, hg = blockIdx.z;
     const int b = n / P.T_q, t = n - b * P.T_q;
@@ -65,35 +87,87 @@ decode_simt_kernel(DecodeParams P) {
     float m_run = -INFINITY, l_run = 0.f;
     const float* q = Qs + warp * D;
 
-    for (int tile = tile0; tile < tile1; ++tile) {
+    for (int kt = tile0; kt < tile1; ++kt) {
         __syncthreads();
         // cooperative load of 32 cache rows through the block table
-        for (int e = threadIdx.x; e < kSimtKeys * (D / 8); e += blockDim.x) {
-            const int j = e / (D / 8), v = e - j * (D / 8);
-            const int key = tile * kSimtKeys + j;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (key < kv_len) {
-                const int blk = P.block_table[static_cast<size_t>(b) * P.max_blocks + key / P.block_size];
-                if (blk >= 0 && blk < P.num_blocks) {
-                    const uint4* src = reinterpret_cast<const uint4*>(
-                        P.pool + (static_cast<size_t>(blk) * P.block_size + key % P.block_size) * D);
-                    val = src[v];
-                } else if (v == 0) {
-                    raise_status(P.status, MLA_STATUS_BAD_BLOCK);
+        if constexpr (kE4m3) {
+            // work item: 16 latent codes (with their group's scale) or 8 RoPE-key values
+            const E4m3Row L = e4m3_row(P.d_c, P.d_r);
+            const int per_row = P.d_c / 16 + P.d_r / 8;
+            for (int e = threadIdx.x; e < kSimtKeys * per_row; e += blockDim.x) {
+                const int j = e / per_row, v = e - j * per_row;
+                const int key = kt * kSimtKeys + j;
+                const unsigned char* src = nullptr;
+                if (key < kv_len) {
+                    const int blk = P.block_table[static_cast<size_t>(b) * P.max_blocks + key / P.block_size];
+                    if (blk >= 0 && blk < P.num_blocks)
+                        src = P.pool8 + (static_cast<size_t>(blk) * P.block_size + key % P.block_size) * L.bytes;
+                    else if (v == 0)
+                        raise_status(P.status, MLA_STATUS_BAD_BLOCK);
+                }
+                float4* dst = reinterpret_cast<float4*>(tile + static_cast<size_t>(j) * row_bytes);
+                if (v < P.d_c / 16) {
+                    float f[16];
+                    if (src != nullptr) {
+                        const uint4 c = reinterpret_cast<const uint4*>(src)[v];
+                        const float sc = reinterpret_cast<const float*>(src + L.scale_off)[v >> 2];
+                        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float2 lo = e4m3x2_to_f32(static_cast<uint16_t>(w[k] & 0xFFFFu));
+                            const float2 hi = e4m3x2_to_f32(static_cast<uint16_t>(w[k] >> 16));
+                            f[4 * k] = lo.x * sc;
+                            f[4 * k + 1] = lo.y * sc;
+                            f[4 * k + 2] = hi.x * sc;
+                            f[4 * k + 3] = hi.y * sc;
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) f[k] = 0.f;
+                    }
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        dst[4 * v + k] = make_float4(f[4 * k], f[4 * k + 1], f[4 * k + 2], f[4 * k + 3]);
+                } else {
+                    const int r = v - P.d_c / 16;   // 8 key values from column d_c + 8 r
+                    float f[8];
+                    if (src != nullptr) {
+                        unpack8(reinterpret_cast<const uint4*>(src + L.kr_off)[r], f);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) f[k] = 0.f;
+                    }
+                    dst[P.d_c / 4 + 2 * r] = make_float4(f[0], f[1], f[2], f[3]);
+                    dst[P.d_c / 4 + 2 * r + 1] = make_float4(f[4], f[5], f[6], f[7]);
                 }
             }
-            Ks[j * row_vec + v] = val;
+        } else {
+            for (int e = threadIdx.x; e < kSimtKeys * (D / 8); e += blockDim.x) {
+                const int j = e / (D / 8), v = e - j * (D / 8);
+                const int key = kt * kSimtKeys + j;
+                uint4 val = make_uint4(0, 0, 0, 0);
+                if (key < kv_len) {
+                    const int blk = P.block_table[static_cast<size_t>(b) * P.max_blocks + key / P.block_size];
+                    if (blk >= 0 && blk < P.num_blocks) {
+                        const uint4* src = reinterpret_cast<const uint4*>(
+                            P.pool + (static_cast<size_t>(blk) * P.block_size + key % P.block_size) * D);
+                        val = src[v];
+                    } else if (v == 0) {
+                        raise_status(P.status, MLA_STATUS_BAD_BLOCK);
+                    }
+                }
+                reinterpret_cast<uint4*>(tile + static_cast<size_t>(j) * row_bytes)[v] = val;
+            }
         }
         __syncthreads();
         if (!head_ok) continue;
 
         // scores: lane j scores key j
-        const int key = tile * kSimtKeys + lane;
+        const int key = kt * kSimtKeys + lane;
         float s = 0.f;
-        const uint4* krow = Ks + lane * row_vec;
         for (int v = 0; v < D / 8; ++v) {
             float kf[8];
-            unpack8(krow[v], kf);
+            load8<kE4m3>(tile, row_bytes, lane, v, kf);
             const float4 qa = *reinterpret_cast<const float4*>(q + 8 * v);
             const float4 qb = *reinterpret_cast<const float4*>(q + 8 * v + 4);
             s = fmaf(qa.x, kf[0], s); s = fmaf(qa.y, kf[1], s);
@@ -114,13 +188,12 @@ decode_simt_kernel(DecodeParams P) {
         for (int j = 0; j < kSimtKeys; ++j) {
             const float pj = __shfl_sync(0xffffffffu, p, j);
             if (pj == 0.f) continue;   // warp-uniform
-            const uint4* vrow = Ks + j * row_vec;
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int ch = lane + 32 * u;
                 if (ch < nchunk) {
                     float vf[8];
-                    unpack8(vrow[ch], vf);
+                    load8<kE4m3>(tile, row_bytes, j, ch, vf);
 #pragma unroll
                     for (int k = 0; k < 8; ++k) o[u][k] = fmaf(pj, vf[k], o[u][k]);
                 }
@@ -196,18 +269,19 @@ merge_splits_kernel(const float* __restrict__ part_o, const float* __restrict__ 
     if (threadIdx.x == 0) out_lse[row] = z > 0.f ? m + logf(z) : -INFINITY;
 }
 
-size_t simt_smem_bytes(int d_c, int d_r) {
+size_t simt_smem_bytes(int d_c, int d_r, bool e4m3) {
     const int D = d_c + d_r;
-    return static_cast<size_t>(kSimtKeys) * (D / 8 + 1) * 16 + static_cast<size_t>(kSimtHeads) * D * 4;
+    return static_cast<size_t>(kSimtKeys) * staged_row_bytes(D, e4m3) + static_cast<size_t>(kSimtHeads) * D * 4;
 }
 
 cudaError_t launch_decode_simt(const DecodeParams& P, cudaStream_t stream) {
-    const size_t smem = simt_smem_bytes(P.d_c, P.d_r);
-    cudaError_t e = cudaFuncSetAttribute(decode_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    const bool e4m3 = P.pool8 != nullptr;
+    const size_t smem = simt_smem_bytes(P.d_c, P.d_r, e4m3);
+    auto kernel = e4m3 ? decode_simt_kernel<true> : decode_simt_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     dim3 grid(P.splits, P.n_tok, (P.n_h + kSimtHeads - 1) / kSimtHeads);
-    decode_simt_kernel<<<grid, 256, smem, stream>>>(P);
+    kernel<<<grid, 256, smem, stream>>>(P);
     e = cudaGetLastError();
     if (e != cudaSuccess || P.splits == 1) return e;
     return launch_merge(P.part_o, P.part_lse, P.out_latent, P.out_lse, P.n_tok * P.n_h, P.d_c,

@@ -44,13 +44,9 @@ struct WsLayout {
     size_t part_o, part_lse, sm100, total;
 };
 
-WsLayout ws_layout(const mla_config_t* c, int B, int T_q, int max_splits) {
+WsLayout ws_layout_simt(const mla_config_t* c, int B, int T_q, int max_splits) {
     WsLayout w;
     w.part_o = w.part_lse = w.sm100 = 256;
-    if (uses_sm100(c)) {
-        w.total = w.sm100 + round256(mla::sm100_workspace_bytes(c->n_h, c->d_c, B, T_q));
-        return w;
-    }
     const int splits = choose_splits(c, B, T_q, max_splits);
     const size_t rows = static_cast<size_t>(B) * T_q * c->n_h;
     const size_t simt_o = splits > 1 ? round256(static_cast<size_t>(splits) * rows * c->d_c * 4) : 0;
@@ -59,6 +55,17 @@ WsLayout ws_layout(const mla_config_t* c, int B, int T_q, int max_splits) {
     w.total = w.part_lse + simt_l;
     return w;
 }
+
+WsLayout ws_layout(const mla_config_t* c, int B, int T_q, int max_splits) {
+    if (!uses_sm100(c)) return ws_layout_simt(c, B, T_q, max_splits);
+    WsLayout w;
+    w.part_o = w.part_lse = w.sm100 = 256;
+    w.total = w.sm100 + round256(mla::sm100_workspace_bytes(c->n_h, c->d_c, B, T_q));
+    return w;
+}
+
+// Shapes of the e4m3 cache format: whole 64-column groups of the latent.
+bool e4m3_shape(const mla_config_t* c) { return c->d_c % MLA_E4M3_GROUP == 0; }
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_LAUNCH; }
 
@@ -205,7 +212,7 @@ int mla_rope_append(const mla_config_t* cfg, mla_bf16* q_r, const mla_bf16* k_r,
     if (B < 1 || T_q < 1 || static_cast<long>(B) * T_q > (1L << 24)) return MLA_ERR_SIZE;
     if (max_pos < 1 || max_blocks_per_seq < 1 || num_blocks < 1) return MLA_ERR_SIZE;
     return cuda_rc(mla::launch_rope_append(q_r, k_r, c_kv, positions, rope_table, max_pos, block_table,
-                                           max_blocks_per_seq, pool, num_blocks, B * T_q, T_q,
+                                           max_blocks_per_seq, pool, false, num_blocks, B * T_q, T_q,
                                            cfg->n_h, cfg->d_c, cfg->d_r, cfg->block_size, dev_status,
                                            static_cast<cudaStream_t>(stream)));
 }
@@ -378,6 +385,86 @@ int mla_up_o_folded(const mla_config_t* cfg, int d_model, const mla_bf16* latent
     if (mla_check_device() != MLA_OK) return MLA_ERR_UNSUPPORTED;
     return cuda_rc(mla::launch_o_folded(latent, w_fold_o, u, n_tok, cfg->n_h, cfg->d_c, d_model, workspace,
                                         dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+size_t mla_e4m3_row_bytes(int d_c, int d_r) {
+    if (d_c < MLA_E4M3_GROUP || d_c > 512 || d_c % MLA_E4M3_GROUP) return 0;
+    if (d_r < 8 || d_r > 64 || d_r % 8) return 0;
+    return static_cast<size_t>(mla::e4m3_row(d_c, d_r).bytes);
+}
+
+int mla_rope_append_e4m3(const mla_config_t* cfg, mla_bf16* q_r, const mla_bf16* k_r,
+                         const mla_bf16* c_kv, const int32_t* positions, const float* rope_table,
+                         int max_pos, const int32_t* block_table, int max_blocks_per_seq,
+                         uint8_t* pool, int num_blocks, int B, int T_q, int32_t* dev_status,
+                         void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!e4m3_shape(cfg)) return MLA_ERR_CONFIG;
+    if (!k_r || !c_kv || !positions || !rope_table || !block_table || !pool) return MLA_ERR_NULL;
+    if ((q_r && !aligned16(q_r)) || !aligned16(k_r) || !aligned16(c_kv) || !aligned16(pool))
+        return MLA_ERR_ALIGN;
+    if (!aligned4(positions) || !aligned4(rope_table) || !aligned4(block_table) ||
+        (dev_status && !aligned4(dev_status)))
+        return MLA_ERR_ALIGN;
+    if (B < 1 || T_q < 1 || static_cast<long>(B) * T_q > (1L << 24)) return MLA_ERR_SIZE;
+    if (max_pos < 1 || max_blocks_per_seq < 1 || num_blocks < 1) return MLA_ERR_SIZE;
+    return cuda_rc(mla::launch_rope_append(q_r, k_r, c_kv, positions, rope_table, max_pos, block_table,
+                                           max_blocks_per_seq, pool, true, num_blocks, B * T_q, T_q,
+                                           cfg->n_h, cfg->d_c, cfg->d_r, cfg->block_size, dev_status,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+size_t mla_decode_e4m3_workspace_bytes(const mla_config_t* cfg, int B, int T_q, int max_splits) {
+    if (check_config(cfg) || !e4m3_shape(cfg) || cfg->impl == 2 || max_splits < 0) return 0;
+    if (B < 1 || T_q < 1 || static_cast<long>(B) * T_q > 65535) return 0;
+    return ws_layout_simt(cfg, B, T_q, max_splits).total;
+}
+
+int mla_decode_e4m3(const mla_config_t* cfg, const mla_bf16* q_abs, const mla_bf16* q_r,
+                    const uint8_t* pool, int num_blocks, const int32_t* block_table,
+                    int max_blocks_per_seq, const int32_t* seq_lens, int B, int T_q, int max_splits,
+                    void* workspace, size_t ws_bytes, mla_bf16* out_latent, float* out_lse,
+                    void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!e4m3_shape(cfg) || cfg->impl == 2) return MLA_ERR_CONFIG;
+    if (!q_abs || !q_r || !pool || !block_table || !seq_lens || !workspace || !out_latent || !out_lse)
+        return MLA_ERR_NULL;
+    if (!aligned16(q_abs) || !aligned16(q_r) || !aligned16(pool) || !aligned16(out_latent) ||
+        !aligned4(out_lse) || !aligned4(block_table) || !aligned4(seq_lens))
+        return MLA_ERR_ALIGN;
+    if (B < 1 || T_q < 1 || static_cast<long>(B) * T_q > 65535) return MLA_ERR_SIZE;
+    if (num_blocks < 1 || max_blocks_per_seq < 1 || max_splits < 0) return MLA_ERR_SIZE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLA_ERR_WORKSPACE;
+    const WsLayout w = ws_layout_simt(cfg, B, T_q, max_splits);
+    if (ws_bytes < w.total) return MLA_ERR_WORKSPACE;
+
+    char* ws = static_cast<char*>(workspace);
+    DecodeParams P;
+    P.q_abs = q_abs;
+    P.q_r = q_r;
+    P.pool = nullptr;
+    P.pool8 = pool;
+    P.block_table = block_table;
+    P.seq_lens = seq_lens;
+    P.out_latent = out_latent;
+    P.out_lse = out_lse;
+    P.part_o = reinterpret_cast<float*>(ws + w.part_o);
+    P.part_lse = reinterpret_cast<float*>(ws + w.part_lse);
+    P.status = reinterpret_cast<int32_t*>(ws);
+    P.n_h = cfg->n_h;
+    P.d_c = cfg->d_c;
+    P.d_r = cfg->d_r;
+    P.block_size = cfg->block_size;
+    P.num_blocks = num_blocks;
+    P.max_blocks = max_blocks_per_seq;
+    P.B = B;
+    P.T_q = T_q;
+    P.n_tok = B * T_q;
+    P.splits = choose_splits(cfg, B, T_q, max_splits);
+    P.scale_log2 = effective_scale(cfg) * mla::kLog2e;
+    return cuda_rc(mla::launch_decode_simt(P, static_cast<cudaStream_t>(stream)));
 }
 
 int mla_clear_status(int32_t* dev_status, void* stream) {

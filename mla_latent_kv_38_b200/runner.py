@@ -28,10 +28,14 @@ class DeviceCase:
 
     def __init__(self, spec: CaseSpec, impl: int = M.IMPL_AUTO, max_splits: int = 0,
                  device: str = "cuda:0", rope_base: float = 10000.0, fill_history: bool = True,
-                 yarn=None):
+                 yarn=None, cache: str = "bf16"):
         """yarn: None (plain RoPE, scale 1/sqrt(d_h + d_r)) or a dict of
         mla_rope_table_yarn / mla_yarn_score_scale arguments (s, alpha, beta,
-        orig_len, coeff); the library builds the table and the scale."""
+        orig_len, coeff); the library builds the table and the scale.
+        cache: "bf16" (rows of d_c + d_r bf16 values) or "e4m3" (the low-bit
+        rows of mla_rope_append_e4m3 / mla_decode_e4m3)."""
+        assert cache in ("bf16", "e4m3")
+        self.cache = cache
         self.spec = spec
         self.dev = torch.device(device)
         self.impl = impl
@@ -54,9 +58,15 @@ class DeviceCase:
         self.block_table_np = s.block_table()
         self.block_table = torch.from_numpy(self.block_table_np).to(dev)
         self.seq_lens = torch.from_numpy(s.seq_lens.astype(np.int32)).to(dev)
-        # Unwritten cache slots hold NaN so that any read past a sequence's end shows.
-        self.pool = torch.full((s.num_blocks, s.block_size, s.D), NAN_BF16, dtype=torch.int16,
-                               device=dev).view(torch.bfloat16)
+        # Unwritten cache slots hold NaN so that any read past a sequence's end
+        # shows (e4m3: NaN codes, scales and key values of 0x7F7F... bytes).
+        if cache == "bf16":
+            self.pool = torch.full((s.num_blocks, s.block_size, s.D), NAN_BF16, dtype=torch.int16,
+                                   device=dev).view(torch.bfloat16)
+        else:
+            self.row_bytes = M.mla_e4m3_row_bytes(s.d_c, s.d_r)
+            self.pool = torch.full((s.num_blocks, s.block_size, self.row_bytes), 0x7F, dtype=torch.uint8,
+                                   device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.w_uk = _bits_to_dev(s.w_uk(), dev)
         self.w_uv = _bits_to_dev(s.w_uv(), dev)
@@ -82,7 +92,8 @@ class DeviceCase:
         self.latent = torch.empty((n, s.n_h, s.d_c), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((n, s.n_h), dtype=torch.float32, device=dev)
         self.out = torch.empty((n, s.n_h, s.d_h), dtype=torch.bfloat16, device=dev)
-        self.ws_bytes = M.mla_decode_workspace_bytes(self.cfg, s.B, s.T_q, max_splits)
+        self.ws_bytes = (M.mla_decode_workspace_bytes(self.cfg, s.B, s.T_q, max_splits) if cache == "bf16" else
+                         M.mla_decode_e4m3_workspace_bytes(self.cfg, s.B, s.T_q, max_splits))
         self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev)
         if fill_history:
             self.fill_history()
@@ -104,9 +115,12 @@ class DeviceCase:
                 k = synth.normal_bf16_torch(s.seed, synth.TID["k_r"], (j1 - j0) * s.d_r,
                                             start=base * s.d_r, device=self.dev)
                 pos = torch.arange(j0, j1, dtype=torch.int32, device=self.dev)
-                M.mla_rope_append(self.cfg, None, k, c, pos, self.rope_table, self.max_pos,
-                                  self.block_table[b:b + 1], s.max_blocks, self.pool, s.num_blocks,
-                                  1, j1 - j0, self.status)
+                self._append()(self.cfg, None, k, c, pos, self.rope_table, self.max_pos,
+                               self.block_table[b:b + 1], s.max_blocks, self.pool, s.num_blocks,
+                               1, j1 - j0, self.status)
+
+    def _append(self):
+        return M.mla_rope_append if self.cache == "bf16" else M.mla_rope_append_e4m3
 
     # -- the step -------------------------------------------------------------
 
@@ -129,15 +143,16 @@ class DeviceCase:
     def rope_append(self, stream=None):
         """RoPE on q^R in place and the new cache rows appended."""
         s = self.spec
-        M.mla_rope_append(self.cfg, self.q_r, self.k_r_new, self.c_kv_new, self.positions,
-                          self.rope_table, self.max_pos, self.block_table, s.max_blocks, self.pool,
-                          s.num_blocks, s.B, s.T_q, self.status, stream)
+        self._append()(self.cfg, self.q_r, self.k_r_new, self.c_kv_new, self.positions,
+                       self.rope_table, self.max_pos, self.block_table, s.max_blocks, self.pool,
+                       s.num_blocks, s.B, s.T_q, self.status, stream)
 
     def decode_only(self, stream=None):
         s = self.spec
-        M.mla_decode(self.cfg, self.q_abs, self.q_r, self.pool, s.num_blocks, self.block_table,
-                     s.max_blocks, self.seq_lens, s.B, s.T_q, self.max_splits, self.ws,
-                     self.ws_bytes, self.latent, self.lse, stream)
+        decode = M.mla_decode if self.cache == "bf16" else M.mla_decode_e4m3
+        decode(self.cfg, self.q_abs, self.q_r, self.pool, s.num_blocks, self.block_table,
+               s.max_blocks, self.seq_lens, s.B, s.T_q, self.max_splits, self.ws,
+               self.ws_bytes, self.latent, self.lse, stream)
 
     def decode_status(self) -> int:
         return M.mla_read_status(self.ws)

@@ -123,9 +123,10 @@ class CaseSpec:
     def visible_keys(self):
         return sum(int(L) - self.T_q + t + 1 for L in self.seq_lens for t in range(self.T_q))
 
-    def algorithmic_bytes(self):
-        """Cache read once + q (bf16) + latent out (bf16) + lse (fp32)."""
-        cache = int(np.sum(self.seq_lens)) * self.D * 2
+    def algorithmic_bytes(self, row_bytes=None):
+        """Cache read once + q (bf16) + latent out (bf16) + lse (fp32); a cache
+        row is D bf16 values unless row_bytes says otherwise (the e4m3 rows)."""
+        cache = int(np.sum(self.seq_lens)) * (self.D * 2 if row_bytes is None else int(row_bytes))
         q = self.n_tok * self.n_h * self.D * 2
         out = self.n_tok * self.n_h * (self.d_c * 2 + 4)
         return cache + q + out

@@ -29,17 +29,23 @@ def _key(spec):
             tuple(int(x) for x in spec.seq_lens))
 
 
-def reference(spec, b: int, heads=None, want_p=False, inv_freq=None, scale=None):
+def reference(spec, b: int, heads=None, want_p=False, inv_freq=None, scale=None, cache="bf16"):
     """Oracle outputs for sequence b: dict(o, latent, lse[, p]) over `heads`.
 
     inv_freq / scale: RoPE frequencies and score scale other than the
-    defaults (YaRN: mla_oracle.yarn_inv_freq, mla_oracle.yarn_score_scale)."""
+    defaults (YaRN: mla_oracle.yarn_inv_freq, mla_oracle.yarn_score_scale).
+    cache "e4m3": every cached latent row is read back from its e4m3 codes and
+    group scales (``lowbit_cache``); the RoPE key as in the bf16 cache."""
     L = int(spec.seq_lens[b])
     T_q = spec.T_q
     c = O.bf16_to_f64(spec.c_kv_rows(b, 0, L))
+    if cache == "e4m3":
+        from . import lowbit_cache as LB
+        c = LB.dequantize_latent(*LB.quantize_latent(spec.c_kv_rows(b, 0, L)))
     k = O.bf16_to_f64(spec.k_r_rows(b, 0, L))
     w_uk, w_uv = _cached("w", spec)
     q_c, q_r = _cached("q", spec)
     sl = slice(b * T_q, (b + 1) * T_q)
     return O.mla_decode_reference(c, k, q_c[sl], q_r[sl], w_uk, w_uv, scale=scale, inv_freq=inv_freq, heads=heads,
                                   want_p=want_p)
+

@@ -250,3 +250,48 @@ def test_yarn_table_and_scale_match_the_oracle(M):
                       ctypes.c_double(32.0), ctypes.c_double(1.0), 4096, buf) == -3      # beta <= alpha
     with pytest.raises(M.MlaError):
         M.mla_yarn_score_scale(128, 64, 0.5)
+
+
+def test_e4m3_row_bytes_match_the_oracle_layout(M):
+    from oracle import lowbit_cache as LB
+    for d_c in (64, 128, 192, 256, 512):
+        for d_r in (8, 16, 32, 64):
+            assert M.mla_e4m3_row_bytes(d_c, d_r) == LB.row_layout(d_c, d_r)[2], (d_c, d_r)
+    for d_c, d_r in ((0, 64), (100, 64), (576, 64), (512, 0), (512, 12), (512, 72)):
+        assert M.mla_e4m3_row_bytes(d_c, d_r) == 0, (d_c, d_r)
+
+
+def test_e4m3_host_validation(M):
+    raw = M.raw_call
+    cfg = _cfg(M)
+    p = ctypes.c_void_p(FAKE)
+
+    def append(c=cfg, q_r=p, k_r=p, c_kv=p, pos=p, table=p, max_pos=4096, bt=p, mbps=64,
+               pool=p, num_blocks=2048, B=32, T_q=1, status=None):
+        return raw("mla_rope_append_e4m3", ctypes.byref(c), q_r, k_r, c_kv, pos, table, max_pos, bt, mbps,
+                   pool, num_blocks, B, T_q, status, None)
+
+    def decode(c=cfg, q_abs=p, q_r=p, pool=p, num_blocks=2048, bt=p, mbps=64, lens=p, B=32, T_q=1,
+               max_splits=0, ws=p, ws_bytes=1 << 30, out=p, lse=p):
+        return raw("mla_decode_e4m3", ctypes.byref(c), q_abs, q_r, pool, num_blocks, bt, mbps, lens, B, T_q,
+                   max_splits, ws, ctypes.c_size_t(ws_bytes), out, lse, None)
+
+    assert append(c=_cfg(M, d_c=96)) == -2 and decode(c=_cfg(M, d_c=96)) == -2   # not whole 64-column groups
+    assert decode(c=_cfg(M, impl=2)) == -2                                        # portable kernels only
+    for name in ("k_r", "c_kv", "pos", "table", "bt", "pool"):
+        assert append(**{name: None}) == -1, name
+    for name in ("q_abs", "q_r", "pool", "bt", "lens", "ws", "out", "lse"):
+        assert decode(**{name: None}) == -1, name
+    odd16 = ctypes.c_void_p(FAKE + 8)
+    assert append(pool=odd16) == -7 and decode(pool=odd16) == -7 and decode(out=odd16) == -7
+    assert append(B=0) == -3 and decode(B=0) == -3 and decode(B=65536) == -3
+    assert decode(ws=ctypes.c_void_p(FAKE + 16)) == -4                            # not 256-byte aligned
+    need = M.mla_decode_e4m3_workspace_bytes(cfg, 32, 1, 0)
+    assert need > 0 and decode(ws_bytes=need - 1) == -4
+    assert M.mla_decode_e4m3_workspace_bytes(_cfg(M, d_c=96), 32, 1, 0) == 0
+    assert M.mla_decode_e4m3_workspace_bytes(_cfg(M, impl=2), 32, 1, 0) == 0
+    # the portable kernel's split partials: splits x rows x (4 d_c + 4) bytes after the status word
+    rows, splits = 32 * 128, 3
+    r256 = lambda x: (x + 255) // 256 * 256
+    assert M.mla_decode_e4m3_workspace_bytes(cfg, 32, 1, splits) == 256 + r256(splits * rows * 512 * 4) + \
+        r256(splits * rows * 4)
