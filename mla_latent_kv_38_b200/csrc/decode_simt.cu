@@ -8,9 +8,10 @@
 // afterwards by mla_up_v).  The causal limit of query t is
 // seq_len - T_q + t ("MLA 코드 구현", generalised causal mask).
 //
-// Layout of the work: grid (split, token, head group of 8).  Each warp owns one
-// head; the 8 warps share each 32-row key tile staged in shared memory with
-// 16-byte loads.  Online softmax in the exp2 domain.
+// Layout of the work: grid (split, token, head group of 16).  Each warp owns
+// two heads, so a staged key row is read from shared memory once for both; the
+// 8 warps share each 32-row key tile staged in shared memory with 16-byte
+// loads.  Online softmax in the exp2 domain.
 //
 // With an e4m3 pool (the low-bit cache of include/mla.h) the tile is staged as
 // float32: each latent value is e4m3(code) * its group's scale, the RoPE key
@@ -21,7 +22,8 @@
 
 namespace mla {
 
-constexpr int kSimtHeads = 8;
+constexpr int kHeadsPerWarp = 2;
+constexpr int kSimtHeads = 8 * kHeadsPerWarp;   // heads per CTA
 constexpr int kSimtKeys = 32;
 
 // Eight consecutive values of staged key row `row` from value 8 v on.
@@ -48,13 +50,13 @@ decode_simt_kernel(DecodeParams P) {
     const int D = P.d_c + P.d_r;
     const int row_bytes = staged_row_bytes(D, kE4m3);
     unsigned char* tile = smem_raw;                                          // [32][row_bytes]
-    float* Qs = reinterpret_cast<float*>(smem_raw + kSimtKeys * row_bytes);  // [8][D]
+    float* Qs = reinterpret_cast<float*>(smem_raw + kSimtKeys * row_bytes);  // [16][D]
 
     const int split = blockIdx.x, n = blockIdx.y, hg = blockIdx.z;
     const int b = n / P.T_q, t = n - b * P.T_q;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int head = hg * kSimtHeads + warp;
-    const bool head_ok = head < P.n_h;
+    const int head0 = hg * kSimtHeads + warp * kHeadsPerWarp;   // this warp's heads: head0, head0 + 1
+    const bool warp_ok = head0 < P.n_h;
 
     int L = P.seq_lens[b];
     const bool len_ok = L >= P.T_q && L <= P.max_blocks * P.block_size;
@@ -79,13 +81,18 @@ decode_simt_kernel(DecodeParams P) {
     }
 
     const int nchunk = P.d_c >> 3;                      // 8-column latent chunks
-    float o[2][8];
+    float o[kHeadsPerWarp][2][8];
+    float m_run[kHeadsPerWarp], l_run[kHeadsPerWarp];
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
+    for (int h = 0; h < kHeadsPerWarp; ++h) {
+        m_run[h] = -INFINITY;
+        l_run[h] = 0.f;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) o[u][k] = 0.f;
-    float m_run = -INFINITY, l_run = 0.f;
-    const float* q = Qs + warp * D;
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) o[h][u][k] = 0.f;
+    }
+    const float* q = Qs + warp * kHeadsPerWarp * D;     // the warp's query rows, one after the other
 
     for (int kt = tile0; kt < tile1; ++kt) {
         __syncthreads();
@@ -160,34 +167,51 @@ decode_simt_kernel(DecodeParams P) {
             }
         }
         __syncthreads();
-        if (!head_ok) continue;
+        if (!warp_ok) continue;
 
-        // scores: lane j scores key j
+        // scores: lane j scores key j against both of the warp's heads
         const int key = kt * kSimtKeys + lane;
-        float s = 0.f;
+        float s[kHeadsPerWarp];
+#pragma unroll
+        for (int h = 0; h < kHeadsPerWarp; ++h) s[h] = 0.f;
         for (int v = 0; v < D / 8; ++v) {
             float kf[8];
             load8<kE4m3>(tile, row_bytes, lane, v, kf);
-            const float4 qa = *reinterpret_cast<const float4*>(q + 8 * v);
-            const float4 qb = *reinterpret_cast<const float4*>(q + 8 * v + 4);
-            s = fmaf(qa.x, kf[0], s); s = fmaf(qa.y, kf[1], s);
-            s = fmaf(qa.z, kf[2], s); s = fmaf(qa.w, kf[3], s);
-            s = fmaf(qb.x, kf[4], s); s = fmaf(qb.y, kf[5], s);
-            s = fmaf(qb.z, kf[6], s); s = fmaf(qb.w, kf[7], s);
+#pragma unroll
+            for (int h = 0; h < kHeadsPerWarp; ++h) {
+                const float4 qa = *reinterpret_cast<const float4*>(q + h * D + 8 * v);
+                const float4 qb = *reinterpret_cast<const float4*>(q + h * D + 8 * v + 4);
+                float a = s[h];
+                a = fmaf(qa.x, kf[0], a); a = fmaf(qa.y, kf[1], a);
+                a = fmaf(qa.z, kf[2], a); a = fmaf(qa.w, kf[3], a);
+                a = fmaf(qb.x, kf[4], a); a = fmaf(qb.y, kf[5], a);
+                a = fmaf(qb.z, kf[6], a); a = fmaf(qb.w, kf[7], a);
+                s[h] = a;
+            }
         }
-        if (key >= kv_len) s = -INFINITY;
-        const float m_new = fmaxf(m_run, warp_max(s));
-        const float alpha = ex2(m_run - m_new);
-        const float p = ex2(s - m_new);
-        l_run = l_run * alpha + warp_sum(p);
-        m_run = m_new;
+        float p[kHeadsPerWarp];
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
+        for (int h = 0; h < kHeadsPerWarp; ++h) {
+            if (key >= kv_len) s[h] = -INFINITY;
+            const float m_new = fmaxf(m_run[h], warp_max(s[h]));   // finite: key kt * 32 is visible
+            const float alpha = ex2(m_run[h] - m_new);
+            p[h] = ex2(s[h] - m_new);
+            l_run[h] = l_run[h] * alpha + warp_sum(p[h]);
+            m_run[h] = m_new;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) o[u][k] *= alpha;
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) o[h][u][k] *= alpha;
+        }
         for (int j = 0; j < kSimtKeys; ++j) {
-            const float pj = __shfl_sync(0xffffffffu, p, j);
-            if (pj == 0.f) continue;   // warp-uniform
+            float pj[kHeadsPerWarp];
+            bool any = false;
+#pragma unroll
+            for (int h = 0; h < kHeadsPerWarp; ++h) {
+                pj[h] = __shfl_sync(0xffffffffu, p[h], j);
+                any = any || pj[h] != 0.f;
+            }
+            if (!any) continue;   // warp-uniform
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int ch = lane + 32 * u;
@@ -195,43 +219,51 @@ decode_simt_kernel(DecodeParams P) {
                     float vf[8];
                     load8<kE4m3>(tile, row_bytes, j, ch, vf);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) o[u][k] = fmaf(pj, vf[k], o[u][k]);
+                    for (int h = 0; h < kHeadsPerWarp; ++h)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) o[h][u][k] = fmaf(pj[h], vf[k], o[h][u][k]);
                 }
             }
         }
     }
 
-    if (!head_ok) return;
-    const size_t row = static_cast<size_t>(n) * P.n_h + head;
-    const bool empty = l_run == 0.f;
-    const float inv_l = empty ? 0.f : 1.f / l_run;
-    const float lse = empty ? -INFINITY : (m_run + __log2f(l_run)) * kLn2;
-    if (P.splits == 1) {
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int ch = lane + 32 * u;
-            if (ch < nchunk) {
-                uint4 w;
-                w.x = pack_bf16x2(o[u][0] * inv_l, o[u][1] * inv_l);
-                w.y = pack_bf16x2(o[u][2] * inv_l, o[u][3] * inv_l);
-                w.z = pack_bf16x2(o[u][4] * inv_l, o[u][5] * inv_l);
-                w.w = pack_bf16x2(o[u][6] * inv_l, o[u][7] * inv_l);
-                reinterpret_cast<uint4*>(P.out_latent + row * P.d_c)[ch] = w;
-            }
-        }
-        if (lane == 0) P.out_lse[row] = lse;
-    } else {
-        float* po = P.part_o + (static_cast<size_t>(split) * P.n_tok * P.n_h + row) * P.d_c;
+    for (int h = 0; h < kHeadsPerWarp; ++h) {
+        const int head = head0 + h;
+        if (head >= P.n_h) break;
+        const size_t row = static_cast<size_t>(n) * P.n_h + head;
+        const bool empty = l_run[h] == 0.f;
+        const float inv_l = empty ? 0.f : 1.f / l_run[h];
+        const float lse = empty ? -INFINITY : (m_run[h] + __log2f(l_run[h])) * kLn2;
+        if (P.splits == 1) {
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int ch = lane + 32 * u;
-            if (ch < nchunk) {
-                float4* d = reinterpret_cast<float4*>(po + 8 * ch);
-                d[0] = make_float4(o[u][0] * inv_l, o[u][1] * inv_l, o[u][2] * inv_l, o[u][3] * inv_l);
-                d[1] = make_float4(o[u][4] * inv_l, o[u][5] * inv_l, o[u][6] * inv_l, o[u][7] * inv_l);
+            for (int u = 0; u < 2; ++u) {
+                const int ch = lane + 32 * u;
+                if (ch < nchunk) {
+                    uint4 w;
+                    w.x = pack_bf16x2(o[h][u][0] * inv_l, o[h][u][1] * inv_l);
+                    w.y = pack_bf16x2(o[h][u][2] * inv_l, o[h][u][3] * inv_l);
+                    w.z = pack_bf16x2(o[h][u][4] * inv_l, o[h][u][5] * inv_l);
+                    w.w = pack_bf16x2(o[h][u][6] * inv_l, o[h][u][7] * inv_l);
+                    reinterpret_cast<uint4*>(P.out_latent + row * P.d_c)[ch] = w;
+                }
             }
+            if (lane == 0) P.out_lse[row] = lse;
+        } else {
+            float* po = P.part_o + (static_cast<size_t>(split) * P.n_tok * P.n_h + row) * P.d_c;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int ch = lane + 32 * u;
+                if (ch < nchunk) {
+                    float4* d = reinterpret_cast<float4*>(po + 8 * ch);
+                    d[0] = make_float4(o[h][u][0] * inv_l, o[h][u][1] * inv_l, o[h][u][2] * inv_l,
+                                       o[h][u][3] * inv_l);
+                    d[1] = make_float4(o[h][u][4] * inv_l, o[h][u][5] * inv_l, o[h][u][6] * inv_l,
+                                       o[h][u][7] * inv_l);
+                }
+            }
+            if (lane == 0) P.part_lse[static_cast<size_t>(split) * P.n_tok * P.n_h + row] = lse;
         }
-        if (lane == 0) P.part_lse[static_cast<size_t>(split) * P.n_tok * P.n_h + row] = lse;
     }
 }
 

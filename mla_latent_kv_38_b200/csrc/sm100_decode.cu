@@ -1171,16 +1171,18 @@ mla_sm100_schedule_kernel(const int32_t* __restrict__ seq_lens, int B, int T_q, 
 // from L2 (ld.global.cg).  The first two slots' rows are fetched together with
 // the log-sum-exps, so that a row split in two takes two dependent round trips
 // (metadata, then everything else); further slots follow two at a time.
-// Blocks of 4 warps, 7 per SM (up to 72 registers a thread, no spills): the
-// 4,096 rows of 32 split units are 1,024 blocks, one wave on 148 SMs.
-__global__ void __launch_bounds__(128, 7)
+// Blocks of 8 warps, at most 64 registers a thread: 4 blocks per SM, one wave
+// for the 4,096 rows of 32 split units.  (Blocks of 4 warps doubled the merge
+// at prefill sizes, where most of the U x 128 rows belong to whole units and
+// the time goes into scheduling blocks that exit at once.)
+__global__ void __launch_bounds__(256, 4)
 mla_sm100_merge_kernel(const int4* __restrict__ unit_meta, const float* __restrict__ part_o,
                        const float* __restrict__ part_lse, uint16_t* __restrict__ out_latent,
                        float* __restrict__ out_lse, int n_h, int n_hb, int B, int T_q, int U) {
     griddep_launch_dependents();
     griddep_wait();
     const int lane = threadIdx.x & 31;
-    const int wg = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int wg = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int u = wg >> 7, row = wg & 127;
     if (u >= U) return;
     const int4 meta = unit_meta[u];
@@ -1361,7 +1363,7 @@ cudaError_t launch_decode_sm100(const DecodeParams& P, void* ws, int max_splits,
     e = launch_pdl(mla_decode_sm100_kernel, dim3(2 * kClusters), dim3(kThreads), kSmemBytes, stream, k);
     if (e != cudaSuccess) return e;
     const int rows = U * 128;
-    return launch_pdl(mla_sm100_merge_kernel, dim3((rows + 3) / 4), dim3(128), 0, stream,
+    return launch_pdl(mla_sm100_merge_kernel, dim3((rows + 7) / 8), dim3(256), 0, stream,
                       static_cast<const int4*>(k.unit_meta), static_cast<const float*>(k.part_o),
                       static_cast<const float*>(k.part_lse), P.out_latent, P.out_lse, P.n_h, n_hb, P.B, P.T_q, U);
 }

@@ -1,6 +1,6 @@
 """Run a workload's decode step a fixed number of times, for profilers.
 
-    python -m mla_latent_kv_38_b200.profile_case --workload v2_decode --iters 4 [--impl 0]
+    python -m mla_latent_kv_38_b200.profile_case --workload v2_decode --iters 4 [--impl 0] [--cache e4m3]
 
 Sets up the workload (cache history appended through the library), then runs
 `--iters` full steps (absorb_q, rope_append, decode, up_v) back to back and
@@ -21,8 +21,9 @@ def main():
     ap.add_argument("--iters", type=int, default=4)
     ap.add_argument("--impl", type=int, default=0)
     ap.add_argument("--decode-only", action="store_true")
+    ap.add_argument("--cache", choices=["bf16", "e4m3"], default="bf16")
     a = ap.parse_args()
-    dc = DeviceCase(workload_specs()[a.workload], impl=a.impl)
+    dc = DeviceCase(workload_specs()[a.workload], impl=a.impl, cache=a.cache)
     for _ in range(a.iters):
         dc.reset_step_inputs()
         if a.decode_only:
