@@ -9,6 +9,11 @@
  *                    weighted sum of the latent rows (split-KV + LSE merge)
  *   mla_up_v         o = W^UV latent, per head
  *
+ * and, around them: the folded projections (mla_fold_weights,
+ * mla_absorb_q_folded, mla_up_o_folded), the YaRN-scaled RoPE table and score
+ * scale, and a low-bit cache format with its own append and decode
+ * (mla_rope_append_e4m3, mla_decode_e4m3).
+ *
  * Sources (page title, section / equation):
  *   [notes]  "MLA(Multi-head Latent Attention): DeepSeek-V2 논문정리":
  *            eq. (9)-(11); "Key에 대한 수식 전개"; "Value에 대한 수식 전개";
