@@ -1,6 +1,8 @@
 """Planted-mistake check of the low-bit cache pins (CPU only): each entry plants
 one plausible slip in a private copy of the oracle module and asserts that at
-least one pin in ``test_oracle_lowbit_pins`` fails on it."""
+least one pin in ``test_oracle_lowbit_pins`` fails on it, and, where the slip
+is in the quantiser, that the exact-arithmetic check in
+``test_oracle_lowbit_exact`` fails too."""
 
 import inspect
 import os
@@ -8,6 +10,7 @@ import types
 
 import pytest
 
+import tests.test_oracle_lowbit_exact as exact
 import tests.test_oracle_lowbit_pins as pins
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(__file__)), "oracle", "lowbit_cache.py")
@@ -56,3 +59,24 @@ def test_pins_catch_planted_mistake(name, monkeypatch):
         except Exception:
             failures += 1
     assert failures >= 1, f"no pin caught mutation {name}"
+
+
+# slips in the quantiser's arithmetic (not in the layout or the decoder), which
+# the exact-rounding check must catch on its own
+QUANTISER = ("encode_truncates", "encode_bias_8", "encode_subnormal_step", "encode_drops_sign",
+             "scale_stored_inverted", "one_scale_per_row", "product_in_double", "divide_by_scale")
+
+
+@pytest.mark.parametrize("name", QUANTISER)
+def test_exact_check_catches_planted_mistake(name, monkeypatch):
+    mod = _mutated_module(*MUTATIONS[name])
+    monkeypatch.setattr(exact, "L", mod)
+    failures = 0
+    for fname, fn in inspect.getmembers(exact, inspect.isfunction):
+        if not fname.startswith("test_"):
+            continue
+        try:
+            fn()
+        except Exception:
+            failures += 1
+    assert failures >= 1, f"the exact check missed mutation {name}"
