@@ -205,6 +205,16 @@ def blas_threads():
         return os.cpu_count()
 
 
+def bench_config(spec, args, world):
+    """The workload description both arms print (the same keys and values)."""
+    return {"workload": spec.name, "B": spec.B, "T_q": spec.T_q, "n_h": spec.n_h,
+            "d_c": spec.d_c, "d_r": spec.d_r, "block_size": spec.block_size,
+            "context": [int(spec.seq_lens.min()), int(spec.seq_lens.max())],
+            "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write)",
+            "parallelism": f"replicas x{world}", "rope": "yarn" if args.yarn else "plain",
+            "projections": "folded" if args.fold else "per head", "cache": args.cache}
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
@@ -217,7 +227,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * secs / max(args.steps, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": spec.name, "rope": "yarn" if args.yarn else "plain", "cache": args.cache},
+        "config": bench_config(spec, args, world),
         "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -554,12 +564,7 @@ def run_ours(args):
         "ms_per_step_median": statistics.median(step_each), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if args.cache == "bf16" else "f32",
         "data": "synthetic",
-        "config": {"workload": spec.name, "B": spec.B, "T_q": spec.T_q, "n_h": spec.n_h,
-                   "d_c": spec.d_c, "d_r": spec.d_r, "block_size": spec.block_size,
-                   "context": [int(spec.seq_lens.min()), int(spec.seq_lens.max())],
-                   "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write)",
-                   "parallelism": f"replicas x{world}", "rope": "yarn" if args.yarn else "plain",
-                   "projections": "folded" if fold is not None else "per head", "cache": args.cache},
+        "config": bench_config(spec, args, world),
         "phases_us": phases_us, "phases_median_us": phases_med_us,
         **({"fold": fold_line} if fold_line is not None else {}),
         "timing": "device passes replay CUDA graphs of the C-ABI calls; e2e calls the API directly",
