@@ -8,10 +8,12 @@
 // afterwards by mla_up_v).  The causal limit of query t is
 // seq_len - T_q + t ("MLA 코드 구현", generalised causal mask).
 //
-// Layout of the work: grid (split, token, head group of 16).  Each warp owns
-// two heads, so a staged key row is read from shared memory once for both; the
-// 8 warps share each 32-row key tile staged in shared memory with 16-byte
-// loads.  Online softmax in the exp2 domain.
+// Layout of the work: grid (split, token, head group of 32).  Each warp owns
+// four heads, so a staged key row is read from shared memory once for all of
+// them; the 8 warps share each 32-row key tile staged in shared memory with
+// 16-byte loads.  The query rows stay bf16 in shared memory (the score scale
+// multiplies each finished dot product), which with at most 128 registers a
+// thread keeps two CTAs on an SM.  Online softmax in the exp2 domain.
 //
 // With an e4m3 pool (the low-bit cache of include/mla.h) the tile is staged as
 // float32: each latent value is e4m3(code) * its group's scale, the RoPE key
@@ -22,7 +24,7 @@
 
 namespace mla {
 
-constexpr int kHeadsPerWarp = 2;
+constexpr int kHeadsPerWarp = 4;
 constexpr int kSimtHeads = 8 * kHeadsPerWarp;   // heads per CTA
 constexpr int kSimtKeys = 32;
 
@@ -44,13 +46,13 @@ __device__ __forceinline__ void load8(const unsigned char* tile, int row_stride,
 __host__ __device__ __forceinline__ int staged_row_bytes(int D, bool e4m3) { return (e4m3 ? 4 : 2) * D + 16; }
 
 template <bool kE4m3>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 decode_simt_kernel(DecodeParams P) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int D = P.d_c + P.d_r;
     const int row_bytes = staged_row_bytes(D, kE4m3);
     unsigned char* tile = smem_raw;                                          // [32][row_bytes]
-    float* Qs = reinterpret_cast<float*>(smem_raw + kSimtKeys * row_bytes);  // [16][D]
+    uint16_t* Qs = reinterpret_cast<uint16_t*>(smem_raw + kSimtKeys * row_bytes);  // [heads][D] bf16
 
     const int split = blockIdx.x, n = blockIdx.y, hg = blockIdx.z;
     const int b = n / P.T_q, t = n - b * P.T_q;
@@ -68,16 +70,16 @@ decode_simt_kernel(DecodeParams P) {
     const int tile0 = split * per;
     const int tile1 = min(ntiles, tile0 + per);
 
-    // stage the query rows, pre-multiplied by scale*log2(e)
+    // stage the query rows as bf16 (the score scale is applied to each dot product)
     for (int e = threadIdx.x; e < kSimtHeads * D; e += blockDim.x) {
         const int w = e / D, c = e - w * D;
         const int hh = hg * kSimtHeads + w;
-        float v = 0.f;
+        uint16_t v = 0;
         if (hh < P.n_h) {
-            v = c < P.d_c ? bf2f(P.q_abs[(static_cast<size_t>(n) * P.n_h + hh) * P.d_c + c])
-                          : bf2f(P.q_r[(static_cast<size_t>(n) * P.n_h + hh) * P.d_r + (c - P.d_c)]);
+            v = c < P.d_c ? P.q_abs[(static_cast<size_t>(n) * P.n_h + hh) * P.d_c + c]
+                          : P.q_r[(static_cast<size_t>(n) * P.n_h + hh) * P.d_r + (c - P.d_c)];
         }
-        Qs[e] = v * P.scale_log2;
+        Qs[e] = v;
     }
 
     const int nchunk = P.d_c >> 3;                      // 8-column latent chunks
@@ -92,7 +94,7 @@ decode_simt_kernel(DecodeParams P) {
 #pragma unroll
             for (int k = 0; k < 8; ++k) o[h][u][k] = 0.f;
     }
-    const float* q = Qs + warp * kHeadsPerWarp * D;     // the warp's query rows, one after the other
+    const uint16_t* q = Qs + warp * kHeadsPerWarp * D;  // the warp's query rows, one after the other
 
     for (int kt = tile0; kt < tile1; ++kt) {
         __syncthreads();
@@ -179,16 +181,16 @@ decode_simt_kernel(DecodeParams P) {
             load8<kE4m3>(tile, row_bytes, lane, v, kf);
 #pragma unroll
             for (int h = 0; h < kHeadsPerWarp; ++h) {
-                const float4 qa = *reinterpret_cast<const float4*>(q + h * D + 8 * v);
-                const float4 qb = *reinterpret_cast<const float4*>(q + h * D + 8 * v + 4);
+                float qf[8];
+                unpack8(*reinterpret_cast<const uint4*>(q + h * D + 8 * v), qf);
                 float a = s[h];
-                a = fmaf(qa.x, kf[0], a); a = fmaf(qa.y, kf[1], a);
-                a = fmaf(qa.z, kf[2], a); a = fmaf(qa.w, kf[3], a);
-                a = fmaf(qb.x, kf[4], a); a = fmaf(qb.y, kf[5], a);
-                a = fmaf(qb.z, kf[6], a); a = fmaf(qb.w, kf[7], a);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) a = fmaf(qf[k], kf[k], a);
                 s[h] = a;
             }
         }
+#pragma unroll
+        for (int h = 0; h < kHeadsPerWarp; ++h) s[h] *= P.scale_log2;
         float p[kHeadsPerWarp];
 #pragma unroll
         for (int h = 0; h < kHeadsPerWarp; ++h) {
@@ -303,7 +305,7 @@ merge_splits_kernel(const float* __restrict__ part_o, const float* __restrict__ 
 
 size_t simt_smem_bytes(int d_c, int d_r, bool e4m3) {
     const int D = d_c + d_r;
-    return static_cast<size_t>(kSimtKeys) * staged_row_bytes(D, e4m3) + static_cast<size_t>(kSimtHeads) * D * 4;
+    return static_cast<size_t>(kSimtKeys) * staged_row_bytes(D, e4m3) + static_cast<size_t>(kSimtHeads) * D * 2;
 }
 
 cudaError_t launch_decode_simt(const DecodeParams& P, cudaStream_t stream) {

@@ -24,10 +24,10 @@ bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Portable kernels: key-range parts per query row -- the caller's bound, or
-// enough (token, 16-head group) CTAs for about 8 per SM.
+// enough (token, 32-head group) CTAs for about 8 per SM.
 int choose_splits(const mla_config_t* c, int B, int T_q, int max_splits) {
     if (max_splits > 0) return max_splits < kMaxSplits ? max_splits : kMaxSplits;
-    const long work = static_cast<long>(B) * T_q * ((c->n_h + 15) / 16);
+    const long work = static_cast<long>(B) * T_q * ((c->n_h + 31) / 32);
     long s = (8L * kB200Sms + work - 1) / work;
     if (s < 1) s = 1;
     if (s > 64) s = 64;
