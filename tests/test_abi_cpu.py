@@ -295,3 +295,21 @@ def test_e4m3_host_validation(M):
     r256 = lambda x: (x + 255) // 256 * 256
     assert M.mla_decode_e4m3_workspace_bytes(cfg, 32, 1, splits) == 256 + r256(splits * rows * 512 * 4) + \
         r256(splits * rows * 4)
+
+
+def test_portable_split_choice(M):
+    """The portable kernels' automatic split count: enough (token, 32-head
+    group) CTAs for about 8 per SM, between 1 and 64 parts; visible through
+    the workspace size of the e4m3 decode (splits x rows x (4 d_c + 4) bytes)."""
+    r256 = lambda x: (x + 255) // 256 * 256
+
+    def ws(n_h, d_c, B, T_q):
+        rows = B * T_q * n_h
+        work = B * T_q * ((n_h + 31) // 32)
+        s = min(64, max(1, -(-8 * 148 // work)))
+        return 256 + (r256(s * rows * d_c * 4) + r256(s * rows * 4) if s > 1 else 0)
+
+    for n_h, d_c, B, T_q in ((128, 512, 32, 1), (128, 512, 1, 1), (4, 64, 1, 1), (128, 512, 64, 4),
+                             (12, 128, 2, 1), (128, 512, 512, 4)):
+        cfg = _cfg(M, n_h=n_h, d_c=d_c, d_r=64 if d_c == 512 else 16)
+        assert M.mla_decode_e4m3_workspace_bytes(cfg, B, T_q, 0) == ws(n_h, d_c, B, T_q), (n_h, d_c, B, T_q)
